@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of one SparsePR attention call on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload wide]
+
+A step is one whole call (partition -> route -> block-sparse attention with
+exact probes -> ridge fit -> corrected output) on the wide call: B=1, H=40,
+N=75600 (grid 21x45x80), d=128, bf16, 22% executed-pair density including 512
+exact probes per head.  Inputs are seeded synthetic video-grid tensors that
+stay resident in HBM; at 2.3 GB they are far larger than L2, so no flush is
+needed between steps.  The device time of K steps is taken with CUDA events on
+the launching stream between barriers and synchronisations; the metric is
+milliseconds per call (lower is better).
+
+Under torchrun each rank runs its own call on its own GPU (independent heads
+need no exchange, so there is no collective on the data path): weak scaling,
+job value = max-rank time / (K * ranks).
+
+`--impl reference` times the fp64 CPU oracle (the reference arm) on the host
+cores on a bounded sample of the same call and prints the same JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per SparsePR attention call (executed-pair density 22% incl. probes)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wide")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="skip the dense/e2e/accuracy extras")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.gpu)], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- inputs
+def device_inputs(w, device):
+    import torch
+    from synthetic import generate_inputs
+    q, k, v = generate_inputs(w, bits=True)
+    if w.dtype == "bf16":
+        return [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device) for a in (q, k, v)]
+    return [torch.from_numpy(a).to(device) for a in (q, k, v)]
+
+
+# --------------------------------------------------------------------- oracle (CPU)
+def oracle_sample(w, budget_s: float = 20.0):
+    """The oracle on a bounded sample of the call: one head, timed stage by
+    stage.  Stages whose full cost exceeds the budget are timed on a
+    contiguous part (k-means: one assignment+update, scaled by the iteration
+    count it takes; attention: a prefix of the query groups, scaled by their
+    share of pairs).  Returns (ms per call, threads, description)."""
+    import oracle as O
+    from synthetic import generate_head
+    q, k, v = (a.astype(np.float64) for a in generate_head(w, 0, 0))
+    kw = O.workload_kwargs(w)
+    N, d = q.shape
+    t_total = 0.0
+    t0 = time.perf_counter()
+    idx = O.sample_indices(N, w.Ms)
+    F = O.key_factor(O.key_metric(q, idx), w.rK, len(idx))
+    phi = k @ F
+    t_total += time.perf_counter() - t0
+    # one k-means iteration (assign + update) on the full head, scaled by max iterations
+    c = phi[O.kmeans_init_indices(w.seed, 0, 0, w.Ck, N)]
+    t0 = time.perf_counter()
+    lab, _ = O.kmeans_assign(phi, c)
+    c = O.kmeans_update(phi, lab, c)
+    t_iter_k = time.perf_counter() - t0
+    kv_raw, _, it_k, _ = O.kmeans(phi, O.kmeans_init_indices(w.seed, 0, 0, w.Ck, N), 2, 0)
+    kv, Ck2, kv_sizes = O.compact_labels(kv_raw, w.Ck)
+    t0 = time.perf_counter()
+    kbar = O.group_means(k, kv, Ck2)
+    vbar = O.group_means(v, kv, Ck2)
+    F_Q = O.query_factor(O.query_metric(kbar), O.query_rank(w.rQ, d, Ck2))
+    phiq = O.query_coords(q, F_Q, w.eps_rms)
+    t_total += time.perf_counter() - t0
+    cq = phiq[O.kmeans_init_indices(w.seed, 0, 1, w.Cq, N)]
+    t0 = time.perf_counter()
+    lq, _ = O.kmeans_assign(phiq, cq)
+    cq = O.kmeans_update(phiq, lq, cq)
+    t_iter_q = time.perf_counter() - t0
+    t_total += (t_iter_k + t_iter_q) * w.kmeans_iters
+    ql, Cq2, q_sizes = O.compact_labels(lq, w.Cq)
+    t0 = time.perf_counter()
+    qbar = O.group_means(q, ql, Cq2)
+    O.query_distances(phiq, ql, Cq2)
+    n_route = max(1, min(Cq2, 8))
+    O.routing_score(qbar[:n_route], k, v, kbar, vbar, kv)
+    t_route = (time.perf_counter() - t0) * Cq2 / n_route
+    t_total += t_route
+    s = O.routing_score(qbar[:n_route], k, v, kbar, vbar, kv)
+    beta = O.key_budget(w.density, min(w.M, N), N, N)
+    mask, _ = O.route(s, kv_sizes, q_sizes[:n_route], beta)
+    # sparse attention on the first query groups, scaled by rows (equal key budgets)
+    t0 = time.perf_counter()
+    rows_done = 0
+    for a in range(n_route):
+        rows = np.nonzero(ql == a)[0]
+        keys = np.nonzero(mask[a][kv])[0]
+        O.dense_attention(q[rows], k[keys], v[keys])
+        rows_done += len(rows)
+    t_total += (time.perf_counter() - t0) * N / max(rows_done, 1)
+    # probes: 16 dense rows scaled to M; fit on M rows
+    t0 = time.perf_counter()
+    O.dense_attention(q[:16], k, v)
+    t_total += (time.perf_counter() - t0) * min(w.M, N) / 16
+    X = np.random.default_rng(0).standard_normal((min(w.M, N), d))
+    t0 = time.perf_counter()
+    al = np.full(len(X), 1.0 / len(X))
+    f = O.ridge_fit(X, X * 0.01, al, al * len(X), w.lam, w.eps_std)
+    O.apply_correction(q, np.arange(4), q[:4], f)
+    t_total += time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    desc = (f"fp64 numpy oracle on head 0 of {w.B * w.H}, x{w.B * w.H}; k-means timed as one assign+update per "
+            f"partition x {w.kmeans_iters} iterations; routing score and sparse attention timed on the first "
+            f"{n_route} of {Cq2} query groups and scaled by rows; 16 of {min(w.M, N)} probe rows scaled")
+    return t_total * 1e3 * w.B * w.H, cores, desc
+
+
+def run_reference(args, w):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        ms, cores, desc = oracle_sample(w)
+        if i >= args.warmup:
+            times.append(ms)
+    v = float(np.mean(times))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms/call", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w), "cpu_baseline": {"value": v, "unit": "ms/call", "cores": cores,
+                                                      "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "ms/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    T, Y, X = w.grid
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} ({T}x{Y}x{X}) d={w.d} {w.dtype}", "B": w.B, "H": w.H,
+            "N": w.N, "d": w.d, "density": w.density, "probes": w.M, "sampled_queries": w.Ms, "Cq": w.Cq,
+            "Ck": w.Ck, "rK": w.rK, "rQ": w.rQ, "kmeans_iters": w.kmeans_iters, "lambda": w.lam,
+            "l2_between_steps": "inputs (2.3 GB) larger than L2; no flush"}
+
+
+# --------------------------------------------------------------------- ours
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    import free_block_sparse_sampled_b200 as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(minutes=15))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cfg = S.SparsePRConfig.from_workload(w)
+    q, k, v = device_inputs(w, dev)
+    ws = S.alloc_workspace(cfg, dev)
+    out = torch.empty(cfg.B, cfg.H, cfg.N, cfg.d, dtype=torch.float32, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        S.call(cfg, q, k, v, ws, out)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        S.call(cfg, q, k, v, ws, out)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    total_ms = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = total_ms / args.steps
+    status = S.device_status(ws)
+
+    # per-stage breakdown, pair counts and launch count (separate, synchronising calls)
+    br = []
+    for _ in range(3):
+        _, st = S.call(cfg, q, k, v, ws, out, stats=True)
+        br.append(st)
+    st = {k_: float(np.mean([b[k_] for b in br])) for k_ in br[0]}
+    pairs_exec, pairs_route = int(br[0]["pairs_exec"]), int(br[0]["pairs_route"])
+    launches = int(br[0]["launches"])
+
+    # dominant kernel: the attention stage alone (staged API), CUDA events on its stream
+    part = S.partition(cfg, q, k, v, ws)
+    rt = S.route(cfg, part, ws)
+    for _ in range(2):
+        S.attention(cfg, part, rt, ws)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_attn = max(3, args.steps)
+    a0.record()
+    for _ in range(n_attn):
+        O_sp, pd, ps = S.attention(cfg, part, rt, ws)
+    a1.record()
+    torch.cuda.synchronize()
+    ms_attn = a0.elapsed_time(a1) / n_attn
+    attn_flops = 4.0 * cfg.d * pairs_exec          # QK^T and PV on every executed pair
+    peaks, peak_kind = measured_peaks()
+    achieved = attn_flops / (ms_attn * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "kernel": "attention_tc_kernel<128> (+ work list and probe gathers)",
+                "peak_source": f"{peak_kind} bf16 dense (burst)"}
+
+    extras = {}
+    if not args.quick:
+        # dense flash-attention call of the same shape (library SDPA, timing reference only)
+        import torch.nn.functional as Fn
+        for _ in range(2):
+            Fn.scaled_dot_product_attention(q, k, v)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record()
+        for _ in range(3):
+            Fn.scaled_dot_product_attention(q, k, v)
+        d1.record()
+        torch.cuda.synchronize()
+        ms_dense = d0.elapsed_time(d1) / 3
+        extras["dense_sdpa_ms"] = ms_dense
+        extras["speedup_vs_dense_sdpa"] = ms_dense / ms_step
+        # accuracy on unprobed rows: 2048 evenly spaced rows per head vs fp32 dense
+        S.call(cfg, q, k, v, ws, out)
+        rows = torch.linspace(0, cfg.N - 1, 2048, device=dev).long()
+        ref = Fn.scaled_dot_product_attention(q[:, :, rows].float(), k.float(), v.float())
+        got = out[:, :, rows]
+        probes = rt["probe_idx"].view(cfg.B, cfg.H, -1)
+        sp = torch.zeros(cfg.B, cfg.H, cfg.N, dtype=torch.bool, device=dev)
+        sp.scatter_(2, probes.long().clamp_min(0), True)
+        keep = ~sp[:, :, rows]
+        err = (got - ref).norm(dim=-1) / (ref.norm(dim=-1) + 1e-8)
+        osp = O_sp.view(cfg.B, cfg.H, cfg.N, cfg.d)[:, :, :][:, :, :]
+        pos = part["pos_q"].view(cfg.B, cfg.H, cfg.N).long()
+        osp_rows = torch.gather(osp, 2, pos[:, :, rows].unsqueeze(-1).expand(-1, -1, -1, cfg.d))
+        err_sp = (osp_rows - ref).norm(dim=-1) / (ref.norm(dim=-1) + 1e-8)
+        e, esp = err[keep].double(), err_sp[keep].double()
+        extras["rel_l2_unprobed"] = {"mean": float(e.mean()), "p99": float(torch.quantile(e, 0.99)),
+                                     "mean_before_correction": float(esp.mean()),
+                                     "p99_before_correction": float(torch.quantile(esp, 0.99)),
+                                     "rows": "2048 evenly spaced rows per head, probes excluded"}
+    e2e = None
+    if not args.no_e2e and not args.quick:
+        hq = [t.cpu().pin_memory() for t in (q, k, v)]
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dq = [torch.empty_like(t) for t in (q, k, v)]
+        for _ in range(2):
+            for dst, src in zip(dq, hq):
+                dst.copy_(src, non_blocking=True)
+            S.call(cfg, *dq, ws, out)
+            hout.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 5))
+        h0.record()
+        for _ in range(n_e2e):
+            for dst, src in zip(dq, hq):
+                dst.copy_(src, non_blocking=True)
+            S.call(cfg, *dq, ws, out)
+            hout.copy_(out, non_blocking=True)
+        h1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(h0.elapsed_time(h1) / n_e2e)
+        e2e = {"value": e2e_ms / world, "unit": "ms/call", "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in hq)),
+               "d2h_bytes_per_step": int(hout.numel() * hout.element_size())}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms_cpu, cores, desc = oracle_sample(w)
+        cpu = {"value": ms_cpu, "unit": "ms/call", "cores": cores, "kind": "oracle", "sample": desc}
+
+    line = {"metric": METRIC, "value": ms_step / world, "unit": "ms/call", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded video-grid generator)",
+            "config": config_of(w), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches * args.steps, "clocks": clocks,
+            "exec_pair_tflops": 4.0 * cfg.d * pairs_exec / (ms_step * 1e-3) / 1e12,
+            "attention_exec_pair_tflops": achieved, "attention_ms": ms_attn,
+            "rho_exec": st["rho_exec"], "pairs_route": pairs_route, "pairs_exec": pairs_exec,
+            "pairs_visited": int(br[0]["pairs_visited"]),
+            "breakdown_ms": {k_: st[k_] for k_ in ("ms_partition", "ms_route", "ms_attention", "ms_fit",
+                                                   "ms_apply", "ms_total")},
+            "kmeans_iters_run": part["kmeans_iters_run"].float().mean(0).tolist(),
+            "device_status": status, **extras}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    from synthetic import get_workload
+    w = get_workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

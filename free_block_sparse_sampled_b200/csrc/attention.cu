@@ -1,0 +1,654 @@
+// Block-sparse attention over group-permuted Q/K/V and exact probe rows
+// ("Partition the Support, Reconstruct the Residual", §3 Eq. (2), §4.3).
+//
+// Work items are query tiles of at most 128 rows that never cross a query
+// group, plus tiles of probe rows.  A sparse item attends to the rows of
+// every K/V group selected for its query group; a probe item attends to all N
+// keys.  Softmax is renormalised over exactly those keys.
+//
+// bf16, block 128: tcgen05 kernel.  Warps 0-3 own the 128 query rows (TMEM
+// lanes) and run the online softmax; warp 4 streams K/V with TMA in 8-row
+// slots (one 1 KB box per 8 keys x 64 channels, 128-byte swizzle) so ragged
+// K/V groups pack into 128-key tiles with little padding (partially used
+// slots are masked); warp 5 issues S = Q K^T and O += P V into TMEM.
+// Every wait is bounded; on timeout the kernel records SPARSEPR_TIMEOUT, lets
+// in-flight copies and MMAs finish, frees TMEM and returns.
+//
+// fp32 inputs (or the SIMT flag): CUDA-core kernel with the same work items.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace spr {
+
+// ---------------------------------------------------------------- work items
+__global__ void __launch_bounds__(1024) build_work_kernel(const int32_t* __restrict__ q_off,
+                                                          const int32_t* __restrict__ ng, int Cq, int BM,
+                                                          int4* __restrict__ items,
+                                                          int32_t* __restrict__ counter) {
+    __shared__ int cnt[kMaxGroups];
+    __shared__ int scratch[33];
+    __shared__ int base;
+    const int bh = blockIdx.x;
+    const int Cqp = ng[bh * 2 + 0];
+    const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
+    for (int a = threadIdx.x; a < Cqp; a += blockDim.x) cnt[a] = (qo[a + 1] - qo[a] + BM - 1) / BM;
+    __syncthreads();
+    const int total = block_exclusive_scan(cnt, Cqp, scratch);
+    if (threadIdx.x == 0) base = atomicAdd(counter, total);
+    __syncthreads();
+    for (int a = threadIdx.x; a < Cqp; a += blockDim.x) {
+        const int s = qo[a], size = qo[a + 1] - qo[a];
+        const int n = (size + BM - 1) / BM;
+        for (int t = 0; t < n; ++t)
+            items[base + cnt[a] + t] = make_int4(bh, a, s + t * BM, min(BM, size - t * BM));
+    }
+}
+
+struct Item {
+    int bh, a, row0, nrows;
+};
+
+__device__ __forceinline__ bool decode_item(int item, const int4* items, const int32_t* counter,
+                                            int n_probe_items, int BM, int Mp, Item& it) {
+    if (item < n_probe_items) {
+        const int per = (Mp + BM - 1) / BM;
+        it.bh = item / per;
+        it.a = -1;
+        it.row0 = (item % per) * BM;
+        it.nrows = min(BM, Mp - it.row0);
+        return true;
+    }
+    const int k = item - n_probe_items;
+    if (k >= *counter) return false;
+    const int4 w = items[k];
+    it.bh = w.x;
+    it.a = w.y;
+    it.row0 = w.z;
+    it.nrows = w.w;
+    return true;
+}
+
+
+// Walks the 8-row key slots of an item: every selected K/V group (or all N
+// keys for a probe item) is cut into slots of 8 rows; the last slot of a
+// group holds fewer valid rows.  Slots past the end are padding (v = 0).
+struct SlotCursor {
+    const int32_t* sg;
+    const int32_t* ko;
+    int n_groups, gi, r_start, r_len, r_off, probe_next, N;
+    bool probe, have;
+    __device__ __forceinline__ SlotCursor(const Item& it, const int32_t* sel_groups, const int32_t* sel_count,
+                                          const int32_t* kv_off, int Cq, int Ck, int N_)
+        : gi(0), r_start(0), r_len(0), r_off(0), probe_next(0), N(N_), have(false) {
+        probe = it.a < 0;
+        sg = sel_groups + ((size_t)it.bh * Cq + (probe ? 0 : it.a)) * Ck;
+        ko = kv_off + (size_t)it.bh * (Ck + 1);
+        n_groups = probe ? 0 : sel_count[(size_t)it.bh * Cq + it.a];
+    }
+    __device__ __forceinline__ void next(int& row, int& v) {
+        row = -1;
+        v = 0;
+        if (probe) {
+            if (probe_next < N) {
+                row = probe_next;
+                v = min(8, N - probe_next);
+                probe_next += 8;
+            }
+            return;
+        }
+        while (!have && gi < n_groups) {
+            const int b = sg[gi++];
+            r_start = ko[b];
+            r_len = ko[b + 1] - r_start;
+            r_off = 0;
+            have = r_len > 0;
+        }
+        if (have) {
+            row = r_start + r_off;
+            v = min(8, r_len - r_off);
+            r_off += 8;
+            if (r_off >= r_len) have = false;
+        }
+    }
+};
+
+// ---------------------------------------------------------------- gathers
+template <typename T>
+__global__ void gather_probe_rows_kernel(const T* __restrict__ src, const int32_t* __restrict__ probe_idx,
+                                         const int32_t* __restrict__ pos_q, int BH, int N, int Mp, int d,
+                                         T* __restrict__ dst) {
+    const int chunks = d * (int)sizeof(T) / 16;
+    const size_t total = (size_t)BH * Mp * chunks;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const size_t r = e / chunks;
+        const int c = (int)(e - r * chunks);
+        const size_t bh = r / Mp;
+        const size_t p = bh * N + pos_q[bh * N + probe_idx[r]];
+        reinterpret_cast<uint4*>(dst)[r * chunks + c] = reinterpret_cast<const uint4*>(src)[p * chunks + c];
+    }
+}
+
+// ---------------------------------------------------------------- SIMT kernel
+// Two threads per query row (each owns half of the channels); keys staged
+// 32 at a time in shared memory; online softmax in the log2 domain.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) attention_simt_kernel(
+    const T* __restrict__ Qp, const T* __restrict__ Kp, const T* __restrict__ Vp,
+    const T* __restrict__ Qprobe, const int4* __restrict__ items, const int32_t* __restrict__ counter,
+    int n_probe_items, int BM, int N, int Mp, int Cq, int Ck, const int32_t* __restrict__ kv_off,
+    const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_groups,
+    float* __restrict__ O_sp, float* __restrict__ probe_dense, unsigned long long* __restrict__ visited,
+    float scale_log2) {
+    constexpr int H = D / 2, KC = 32;
+    __shared__ float ks[KC][D];
+    __shared__ float vs[KC][D];
+    Item it;
+    if (!decode_item(blockIdx.x, items, counter, n_probe_items, BM, Mp, it)) return;
+    const int r = threadIdx.x >> 1, h = threadIdx.x & 1;
+    const bool active = r < it.nrows;
+    const T* qrow = (it.a < 0) ? Qprobe + ((size_t)it.bh * Mp + it.row0 + r) * D
+                               : Qp + ((size_t)it.bh * N + it.row0 + r) * D;
+    float q[H], o[H];
+#pragma unroll
+    for (int t = 0; t < H; ++t) {
+        q[t] = active ? ldf(qrow + h * H + t) * scale_log2 : 0.f;
+        o[t] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+    const int n_ranges = (it.a < 0) ? 1 : sel_count[(size_t)it.bh * Cq + it.a];
+    const int32_t* sg = sel_groups + ((size_t)it.bh * Cq + (it.a < 0 ? 0 : it.a)) * Ck;
+    const int32_t* ko = kv_off + (size_t)it.bh * (Ck + 1);
+    for (int g = 0; g < n_ranges; ++g) {
+        int s, e;
+        if (it.a < 0) {
+            s = 0;
+            e = N;
+        } else {
+            const int b = sg[g];
+            s = ko[b];
+            e = ko[b + 1];
+        }
+        for (int c0 = s; c0 < e; c0 += KC) {
+            const int n = min(KC, e - c0);
+            __syncthreads();
+            for (int x = threadIdx.x; x < KC * D; x += blockDim.x) {
+                const int j = x / D, t = x % D;
+                const bool ok = j < n;
+                ks[j][t] = ok ? ldf(Kp + ((size_t)it.bh * N + c0 + j) * D + t) : 0.f;
+                vs[j][t] = ok ? ldf(Vp + ((size_t)it.bh * N + c0 + j) * D + t) : 0.f;
+            }
+            __syncthreads();
+            float sc[KC];
+            float cm = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < KC; ++j) {
+                float part = 0.f;
+#pragma unroll
+                for (int t = 0; t < H; ++t) part = fmaf(q[t], ks[j][h * H + t], part);
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                sc[j] = (j < n) ? part : -INFINITY;
+                cm = fmaxf(cm, sc[j]);
+            }
+            const float mn = fmaxf(m, cm);
+            const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+            l *= alpha;
+#pragma unroll
+            for (int t = 0; t < H; ++t) o[t] *= alpha;
+            m = mn;
+#pragma unroll
+            for (int j = 0; j < KC; ++j) {
+                if (j < n) {
+                    const float p = exp2f(sc[j] - m);
+                    l += p;
+#pragma unroll
+                    for (int t = 0; t < H; ++t) o[t] = fmaf(p, vs[j][h * H + t], o[t]);
+                }
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        unsigned long long keys = 0;
+        for (int g = 0; g < n_ranges; ++g)
+            keys += (it.a < 0) ? (unsigned long long)N : (unsigned long long)(ko[sg[g] + 1] - ko[sg[g]]);
+        atomicAdd(visited, keys * (unsigned long long)BM);
+    }
+    if (!active) return;
+    float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + it.row0 + r) * D
+                            : O_sp + ((size_t)it.bh * N + it.row0 + r) * D;
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int t = 0; t < H; ++t) out[h * H + t] = o[t] * inv;
+}
+
+// ---------------------------------------------------------------- tcgen05 kernel
+namespace tc {
+constexpr int BM = 128, BN = 128, NS = 2;
+constexpr uint32_t kSpin = 1u << 20;   // polls of mbarrier.try_wait before giving up
+enum { B_Q = 0, B_KF = 1, B_KE = B_KF + NS, B_VF = B_KE + NS, B_VE = B_VF + NS, B_SF = B_VE + NS,
+       B_SE = B_SF + 2, B_PF = B_SE + 2, B_OD = B_PF + 1, B_DR = B_OD + 1, N_BAR = B_DR + 1 };
+
+template <int D>
+struct Layout {
+    static constexpr int QB = BM * D * 2;          // Q tile bytes
+    static constexpr int KB = BN * D * 2;          // one K (or V) stage
+    static constexpr int PB = BM * BN * 2;         // P tile
+    static constexpr int oQ = 0;
+    static constexpr int oK = oQ + QB;
+    static constexpr int oV = oK + NS * KB;
+    static constexpr int oP = oV + NS * KB;
+    static constexpr int oBar = oP + PB;
+    static constexpr int oMisc = oBar + N_BAR * 8;
+    static constexpr int bytes = oMisc + 64;
+    static constexpr int smem = bytes + 1024;      // slack for 1024-byte alignment
+};
+}  // namespace tc
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) attention_tc_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQP,
+    const int4* __restrict__ items, const int32_t* __restrict__ counter, int n_probe_items, int N,
+    int Mp, int Cq, int Ck, const int32_t* __restrict__ kv_off, const int32_t* __restrict__ sel_count,
+    const int32_t* __restrict__ sel_groups, float* __restrict__ O_sp, float* __restrict__ probe_dense,
+    DevStatus* status, unsigned long long* __restrict__ visited, float scale_log2) {
+    using namespace tc;
+    using namespace sm100;
+    using L = Layout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    Item it;
+    if (!decode_item(blockIdx.x, items, counter, n_probe_items, BM, Mp, it)) return;
+    // once any block has given up, the rest of the launch returns at once
+    if (*reinterpret_cast<volatile const int32_t*>(&status->code) != 0) return;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t s_base = smem_u32(sm);
+    const uint32_t sQ = s_base + L::oQ, sK = s_base + L::oK, sV = s_base + L::oV, sP = s_base + L::oP;
+    auto bar = [&](int i) -> uint32_t { return s_base + L::oBar + 8 * i; };
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::oMisc);   // [0] tmem, [1] abort, [2] n_tiles
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+    if (tid == 0) {
+        mbar_init(bar(B_Q), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(B_KF + s), 1);
+            mbar_init(bar(B_KE + s), 1);
+            mbar_init(bar(B_VF + s), 1);
+            mbar_init(bar(B_VE + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_SF + s), 1);
+            mbar_init(bar(B_SE + s), 128);
+        }
+        mbar_init(bar(B_PF), 128);
+        mbar_init(bar(B_OD), 1);
+        mbar_init(bar(B_DR), 1);
+        fence_barrier_init();
+        misc[1] = 0;
+    }
+    if (warp == 0) {   // number of 128-key tiles = ceil(slots / 16)
+        long long slots = 0;
+        if (it.a < 0) {
+            slots = lane == 0 ? (N + 7) / 8 : 0;
+        } else {
+            const int cnt = sel_count[(size_t)it.bh * Cq + it.a];
+            const int32_t* sg = sel_groups + ((size_t)it.bh * Cq + it.a) * Ck;
+            const int32_t* ko = kv_off + (size_t)it.bh * (Ck + 1);
+            for (int g = lane; g < cnt; g += 32) {
+                const int b = sg[g];
+                slots += (ko[b + 1] - ko[b] + 7) / 8;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) slots += __shfl_xor_sync(0xffffffffu, slots, o);
+        if (lane == 0) {
+            misc[2] = (uint32_t)((slots + 15) / 16);
+            atomicAdd(visited, (unsigned long long)((slots + 15) / 16) * (unsigned long long)(BM * BN));
+        }
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(misc), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const int n_tiles = (int)misc[2];
+
+    if (warp == 4) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const CUtensorMap* tq = (it.a < 0) ? &tmQP : &tmQ;
+            prefetch_tmap(tq);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            const int qrow = (it.a < 0) ? it.bh * Mp + it.row0 : it.bh * N + it.row0;
+            mbar_arrive_expect_tx(bar(B_Q), L::QB);
+            for (int u = 0; u < 16; ++u)
+                for (int hh = 0; hh < D / 64; ++hh)
+                    tma_load_2d(sQ + hh * BM * 128 + u * 1024, tq, bar(B_Q), hh * 64, qrow + 8 * u);
+            SlotCursor cur(it, sel_groups, sel_count, kv_off, Cq, Ck, N);
+            int pad_row = -1, issued_k = 0, issued_v = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int stage = j % NS, use = j / NS;
+                if (j >= NS && !mbar_wait(bar(B_KE + stage), (use - 1) & 1, abort_flag, kSpin)) {
+                    record_status(status, SPARSEPR_TIMEOUT, 41);
+                    *abort_flag = 1;
+                    break;
+                }
+                int rows[16];
+                for (int u = 0; u < 16; ++u) {
+                    int row, v;
+                    cur.next(row, v);
+                    if (pad_row < 0) pad_row = row;
+                    rows[u] = row >= 0 ? row : pad_row;
+                }
+                mbar_arrive_expect_tx(bar(B_KF + stage), L::KB);
+                for (int u = 0; u < 16; ++u)
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        tma_load_2d(sK + stage * L::KB + hh * BN * 128 + u * 1024, &tmK, bar(B_KF + stage),
+                                    hh * 64, it.bh * N + rows[u]);
+                issued_k = j + 1;
+                if (j >= NS && !mbar_wait(bar(B_VE + stage), (use - 1) & 1, abort_flag, kSpin)) {
+                    record_status(status, SPARSEPR_TIMEOUT, 42);
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(bar(B_VF + stage), L::KB);
+                for (int u = 0; u < 16; ++u)
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        tma_load_2d(sV + stage * L::KB + hh * BN * 128 + u * 1024, &tmV, bar(B_VF + stage),
+                                    hh * 64, it.bh * N + rows[u]);
+                issued_v = j + 1;
+            }
+            // every copy this CTA issued lands before the CTA can exit (abort or not)
+            mbar_wait(bar(B_Q), 0, nullptr, kSpin);
+            for (int t = max(0, issued_k - NS); t < issued_k; ++t)
+                mbar_wait(bar(B_KF + t % NS), (t / NS) & 1, nullptr, kSpin);
+            for (int t = max(0, issued_v - NS); t < issued_v; ++t)
+                mbar_wait(bar(B_VF + t % NS), (t / NS) & 1, nullptr, kSpin);
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
+            auto issue_pv = [&](int t) -> bool {
+                const int stage = t % NS;
+                if (!mbar_wait(bar(B_PF), t & 1, abort_flag, kSpin)) return false;
+                if (!mbar_wait(bar(B_VF + stage), (t / NS) & 1, abort_flag, kSpin)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t a = smem_desc(sP + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
+                    const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
+                    mma_bf16_ss(tO, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(B_OD));
+                mma_commit(bar(B_VE + stage));
+                return true;
+            };
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int stage = j % NS, sb = j & 1;
+                if (!mbar_wait(bar(B_KF + stage), (j / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
+                if (j >= 2 && !mbar_wait(bar(B_SE + sb), ((j - 2) / 2) & 1, abort_flag, kSpin)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t tS = sb ? tS1 : tS0;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t a = smem_desc(sQ + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
+                    const uint64_t b = smem_desc(sK + stage * L::KB + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
+                    mma_bf16_ss(tS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(B_SF + sb));
+                mma_commit(bar(B_KE + stage));
+                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+            }
+            if (ok && n_tiles > 0) ok = issue_pv(n_tiles - 1);
+            if (!ok) {
+                record_status(status, SPARSEPR_TIMEOUT, 43);
+                *abort_flag = 1;
+            }
+            // every MMA issued above completes before TMEM is released
+            mma_commit(bar(B_DR));
+            mbar_wait(bar(B_DR), 0, nullptr, kSpin);
+        }
+    } else {
+        // ------------------------------------------------ softmax warpgroup (rows = TMEM lanes)
+        const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t tO = t_row + 256;
+        const int r = tid;   // 0..127
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        uint8_t* prow = sm + L::oP + r * 128;
+        SlotCursor cur(it, sel_groups, sel_count, kv_off, Cq, Ck, N);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int sb = j & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + sb), (j / 2) & 1, abort_flag, kSpin));
+            if (!ok) break;
+            tc_fence_after();
+            float s[128];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float v[32];
+                tmem_ld32(t_row + sb * 128 + c4 * 32, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) s[c4 * 32 + i] = v[i];
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(B_SE + sb));
+            float mx = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                int row_unused, v;
+                cur.next(row_unused, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float x = (i < v) ? s[u * 8 + i] * scale_log2 : -INFINITY;
+                    s[u * 8 + i] = x;
+                    mx = fmaxf(mx, x);
+                }
+            }
+            const float m_new = fmaxf(m_ref, mx);
+            const bool need = (j > 0) && (m_new > m_ref + 8.f);
+            if (j == 0) m_ref = m_new;
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD), (j - 1) & 1, abort_flag, kSpin));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            if (__any_sync(0xffffffffu, need)) {
+                const float alpha = need ? exp2f(m_ref - m_new) : 1.f;
+                if (need) {
+                    m_ref = m_new;
+                    l *= alpha;
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    float v[32];
+                    tmem_ld32(tO + c4 * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st32(tO + c4 * 32, v);
+                }
+                tmem_wait_st();
+            }
+            // P = exp2(s - m_ref) as bf16 into the swizzled K-major P tile
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __nv_bfloat162 pr = __floats2bfloat162_rn(exp2f(s[u * 8 + 2 * i] - m_ref),
+                                                                    exp2f(s[u * 8 + 2 * i + 1] - m_ref));
+                    const float2 back = __bfloat1622float2(pr);
+                    l += back.x + back.y;
+                    w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+                }
+                const int chunk = u >> 3, unit = u & 7;
+                uint4* dst = reinterpret_cast<uint4*>(prow + chunk * (BM * 128) + ((unit ^ (r & 7)) << 4));
+                *dst = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(B_PF));
+        }
+        if (ok && n_tiles > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD), (n_tiles - 1) & 1, abort_flag, kSpin));
+            if (ok) {
+                tc_fence_after();
+                float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + it.row0 + r) * D
+                                        : O_sp + ((size_t)it.bh * N + it.row0 + r) * D;
+                const float inv = 1.f / l;
+#pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    float v[32];
+                    tmem_ld32(tO + c4 * 32, v);
+                    tmem_wait_ld();
+                    if (r < it.nrows) {
+                        float4* o4 = reinterpret_cast<float4*>(out + c4 * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            o4[i] = make_float4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv,
+                                                v[4 * i + 3] * inv);
+                    }
+                }
+            }
+        }
+        if (!ok) {
+            record_status(status, SPARSEPR_TIMEOUT, 44);
+            *abort_flag = 1;
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ================================================================ host side
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [rows, d] bf16 row-major, boxes of 8 rows x 64 channels, 128-byte swizzle.
+bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr || rows == 0) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64, 8};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int grid_for(size_t total, int threads) {
+    size_t g = (total + threads - 1) / threads;
+    return (int)(g > 148 * 64 ? 148 * 64 : (g == 0 ? 1 : g));
+}
+
+}  // namespace
+
+bool attention_uses_tc(const sparsepr_params& p) {
+    return p.dtype == SPARSEPR_BF16 && p.block == 128 && (p.d == 64 || p.d == 128) &&
+           !(p.flags & SPARSEPR_FLAG_SIMT_ATTENTION);
+}
+
+sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
+                              const sparsepr_route_out& r, float* O_sp, float* probe_dense,
+                              float* probe_sparse, void* ws, cudaStream_t st) {
+    const int BH = pl.BH, N = pl.N, d = pl.d, Mp = pl.Mp;
+    int32_t* counter = at<int32_t>(ws, pl.o_work);
+    int4* items = at<int4>(ws, pl.o_work + 256);
+    void* qprobe = at<void>(ws, pl.o_qprobe);
+    DevStatus* status = at<DevStatus>(ws, pl.o_status);
+    unsigned long long* visited = at<unsigned long long>(ws, pl.o_work + 8);
+    cudaMemsetAsync(counter, 0, 16, st);
+    count_launch(), build_work_kernel<<<BH, 1024, 0, st>>>(part.q_offsets, part.n_groups, pl.Cq, pl.BM, items, counter);
+    if (Mp > 0) {
+        const int chunks = d * pl.esz / 16;
+        if (p.dtype == SPARSEPR_BF16)
+            count_launch(), gather_probe_rows_kernel<__nv_bfloat16><<<grid_for((size_t)BH * Mp * chunks, 256), 256, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(part.Qp), r.probe_idx, part.pos_q, BH, N, Mp, d,
+                static_cast<__nv_bfloat16*>(qprobe));
+        else
+            count_launch(), gather_probe_rows_kernel<float><<<grid_for((size_t)BH * Mp * chunks, 256), 256, 0, st>>>(
+                static_cast<const float*>(part.Qp), r.probe_idx, part.pos_q, BH, N, Mp, d,
+                static_cast<float*>(qprobe));
+    }
+    const int grid = pl.n_probe_items + pl.n_items_max;
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+    if (attention_uses_tc(p)) {
+        CUtensorMap mQ, mK, mV, mQP;
+        bool ok = make_rows_map(&mQ, part.Qp, (uint64_t)BH * N, d) && make_rows_map(&mK, part.Kp, (uint64_t)BH * N, d) &&
+                  make_rows_map(&mV, part.Vp, (uint64_t)BH * N, d);
+        if (!ok) return SPARSEPR_CUDA_ERROR;
+        if (Mp > 0) {
+            if (!make_rows_map(&mQP, qprobe, (uint64_t)BH * Mp, d)) return SPARSEPR_CUDA_ERROR;
+        } else {
+            mQP = mQ;
+        }
+        if (d == 128) {
+            auto k = attention_tc_kernel<128>;
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<128>::smem);
+            count_launch(), k<<<grid, 192, tc::Layout<128>::smem, st>>>(mQ, mK, mV, mQP, items, counter, pl.n_probe_items, N, Mp,
+                                                       pl.Cq, pl.Ck, part.kv_offsets, r.sel_count, r.sel_groups,
+                                                       O_sp, probe_dense, status, visited, scale_log2);
+        } else {
+            auto k = attention_tc_kernel<64>;
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<64>::smem);
+            count_launch(), k<<<grid, 192, tc::Layout<64>::smem, st>>>(mQ, mK, mV, mQP, items, counter, pl.n_probe_items, N, Mp,
+                                                      pl.Cq, pl.Ck, part.kv_offsets, r.sel_count, r.sel_groups,
+                                                      O_sp, probe_dense, status, visited, scale_log2);
+        }
+    } else {
+        const int threads = 2 * pl.BM;
+#define SPR_SIMT(T, D)                                                                                        \
+    count_launch(), attention_simt_kernel<T, D><<<grid, threads, 0, st>>>(                                                    \
+        static_cast<const T*>(part.Qp), static_cast<const T*>(part.Kp), static_cast<const T*>(part.Vp),     \
+        static_cast<const T*>(qprobe), items, counter, pl.n_probe_items, pl.BM, N, Mp, pl.Cq, pl.Ck,        \
+        part.kv_offsets, r.sel_count, r.sel_groups, O_sp, probe_dense, visited, scale_log2)
+        if (p.dtype == SPARSEPR_BF16) {
+            if (d == 128) SPR_SIMT(__nv_bfloat16, 128); else SPR_SIMT(__nv_bfloat16, 64);
+        } else {
+            if (d == 128) SPR_SIMT(float, 128); else SPR_SIMT(float, 64);
+        }
+#undef SPR_SIMT
+    }
+    if (Mp > 0) {
+        const int chunks = d * 4 / 16;
+        count_launch(), gather_probe_rows_kernel<float><<<grid_for((size_t)BH * Mp * chunks, 256), 256, 0, st>>>(
+            O_sp, r.probe_idx, part.pos_q, BH, N, Mp, d, probe_sparse);
+    }
+    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+}
+
+}  // namespace spr

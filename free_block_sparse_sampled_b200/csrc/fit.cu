@@ -1,0 +1,301 @@
+// Probe-fitted residual reconstruction ("Partition the Support, Reconstruct
+// the Residual", §4.2, A.2, A.3, D.3).
+//
+//   w_p = |G_a| / m_a,  alpha_p = w_p / sum w,  w~_p = M alpha_p
+//   mu_X = sum alpha x_p,  sigma = sqrt(sum alpha (x_p - mu_X)^2 + eps),
+//   Xbar = (X - mu_X)/sigma,  mu_R = sum alpha R_p,  Rbar = R - mu_R
+//   B = (Xbar^T W Xbar + lambda I)^-1 Xbar^T W Rbar     (Cholesky)
+//   O^_i = O^dense_i for probes,  O^sp_i + mu_R + Xbar_i B otherwise.
+//
+// The fit is small (M x d and d x d per head) and runs in fp64; B and the
+// statistics are stored in fp32 for the fp32 apply.
+#include "common.cuh"
+#include "internal.h"
+
+namespace spr {
+
+__device__ __forceinline__ double probe_alpha(int p, const int32_t* pg, const int32_t* alloc, const int32_t* qo,
+                                              double sum_w) {
+    const int a = pg[p];
+    return ((double)(qo[a + 1] - qo[a]) / (double)alloc[a]) / sum_w;
+}
+
+// Weighted statistics; one thread per channel j.
+__global__ void fit_stats_kernel(const float* __restrict__ Xs, const float* __restrict__ Xd,
+                                 const int32_t* __restrict__ probe_group, const int32_t* __restrict__ alloc,
+                                 const int32_t* __restrict__ q_off, const int32_t* __restrict__ ng,
+                                 int32_t* __restrict__ psum, int Cq, int Mp, int d, float eps_std,
+                                 double* __restrict__ fstat, float* __restrict__ mu_x, float* __restrict__ sigma,
+                                 float* __restrict__ mu_r) {
+    const int bh = blockIdx.x, j = threadIdx.x;
+    __shared__ int sum_w;
+    if (j == 0) {   // sum_p w_p = sum of |G_a| over groups holding probes
+        int s = 0;
+        const int Cqp = ng[bh * 2 + 0];
+        for (int a = 0; a < Cqp; ++a)
+            if (alloc[(size_t)bh * Cq + a] > 0) s += q_off[(size_t)bh * (Cq + 1) + a + 1] - q_off[(size_t)bh * (Cq + 1) + a];
+        sum_w = s;
+        psum[bh] = s;
+    }
+    __syncthreads();
+    const float* X = Xs + (size_t)bh * Mp * d;
+    const float* D = Xd + (size_t)bh * Mp * d;
+    const int32_t* pg = probe_group + (size_t)bh * Mp;
+    const int32_t* al = alloc + (size_t)bh * Cq;
+    const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
+    const double sw = (double)sum_w;
+    double mx = 0.0, mr = 0.0;
+    for (int p = 0; p < Mp; ++p) {
+        const double al_p = probe_alpha(p, pg, al, qo, sw);
+        const double x = X[(size_t)p * d + j];
+        mx += al_p * x;
+        mr += al_p * ((double)D[(size_t)p * d + j] - x);
+    }
+    double var = 0.0;
+    for (int p = 0; p < Mp; ++p) {
+        const double al_p = probe_alpha(p, pg, al, qo, sw);
+        const double c = (double)X[(size_t)p * d + j] - mx;
+        var += al_p * c * c;
+    }
+    const double sg = sqrt(var + (double)eps_std);
+    double* fs = fstat + (size_t)bh * 3 * d;
+    fs[j] = mx;
+    fs[d + j] = sg;
+    fs[2 * d + j] = mr;
+    mu_x[(size_t)bh * d + j] = (float)mx;
+    sigma[(size_t)bh * d + j] = (float)sg;
+    mu_r[(size_t)bh * d + j] = (float)mr;
+}
+
+// Rows i0..i0+7 of G = Xbar^T W Xbar + lambda I and of RHS = Xbar^T W Rbar.
+__global__ void fit_gram_kernel(const float* __restrict__ Xs, const float* __restrict__ Xd,
+                                const int32_t* __restrict__ probe_group, const int32_t* __restrict__ alloc,
+                                const int32_t* __restrict__ q_off, const int32_t* __restrict__ psum, int Cq, int Mp,
+                                int d, double lambda, const double* __restrict__ fstat, double* __restrict__ G,
+                                double* __restrict__ rhs) {
+    constexpr int RI = 8;
+    const int bh = blockIdx.y, i0 = blockIdx.x * RI, j = threadIdx.x;
+    const float* X = Xs + (size_t)bh * Mp * d;
+    const float* D = Xd + (size_t)bh * Mp * d;
+    const int32_t* pg = probe_group + (size_t)bh * Mp;
+    const int32_t* al = alloc + (size_t)bh * Cq;
+    const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
+    const double* fs = fstat + (size_t)bh * 3 * d;
+    const double sw = (double)psum[bh];
+    const double mxj = fs[j], sgj = fs[d + j], mrj = fs[2 * d + j];
+    double mxi[RI], sgi[RI];
+#pragma unroll
+    for (int u = 0; u < RI; ++u) {
+        mxi[u] = fs[i0 + u];
+        sgi[u] = fs[d + i0 + u];
+    }
+    double g[RI], h[RI];
+#pragma unroll
+    for (int u = 0; u < RI; ++u) g[u] = h[u] = 0.0;
+    for (int p = 0; p < Mp; ++p) {
+        const double wt = (double)Mp * probe_alpha(p, pg, al, qo, sw);
+        const double xj = (double)X[(size_t)p * d + j];
+        const double xbj = (xj - mxj) / sgj;
+        const double rbj = ((double)D[(size_t)p * d + j] - xj) - mrj;
+#pragma unroll
+        for (int u = 0; u < RI; ++u) {
+            const double xbi = wt * (((double)X[(size_t)p * d + i0 + u] - mxi[u]) / sgi[u]);
+            g[u] += xbi * xbj;
+            h[u] += xbi * rbj;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < RI; ++u) {
+        const int i = i0 + u;
+        G[((size_t)bh * d + i) * d + j] = g[u] + (i == j ? lambda : 0.0);
+        rhs[((size_t)bh * d + i) * d + j] = h[u];
+    }
+}
+
+// Cholesky G = L L^T in shared memory, then each thread solves one column
+// of B = G^-1 RHS by forward and back substitution (RHS overwritten in place).
+__global__ void fit_solve_kernel(const double* __restrict__ G, double* __restrict__ rhs, int d,
+                                 float* __restrict__ Bout, DevStatus* status) {
+    extern __shared__ double Ls[];
+    __shared__ int fail;
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    const int ld = d + 1;
+    const double* Gh = G + (size_t)bh * d * d;
+    for (int e = tid; e < d * d; e += blockDim.x) Ls[(e / d) * ld + (e % d)] = Gh[e];
+    if (tid == 0) fail = 0;
+    __syncthreads();
+    for (int k = 0; k < d; ++k) {
+        if (tid == 0) {
+            const double piv = Ls[k * ld + k];
+            if (!(piv > 0.0)) {
+                fail = 1;
+                record_status(status, SPARSEPR_NUMERIC, 60);
+            } else {
+                Ls[k * ld + k] = sqrt(piv);
+            }
+        }
+        __syncthreads();
+        if (fail) break;
+        const double lkk = Ls[k * ld + k];
+        for (int i = k + 1 + tid; i < d; i += blockDim.x) Ls[i * ld + k] /= lkk;
+        __syncthreads();
+        for (int i = k + 1 + tid; i < d; i += blockDim.x) {
+            const double lik = Ls[i * ld + k];
+            for (int j = k + 1; j <= i; ++j) Ls[i * ld + j] -= lik * Ls[j * ld + k];
+        }
+        __syncthreads();
+    }
+    if (fail) {
+        for (int e = tid; e < d * d; e += blockDim.x) Bout[(size_t)bh * d * d + e] = 0.f;
+        return;
+    }
+    double* R = rhs + (size_t)bh * d * d;
+    for (int j = tid; j < d; j += blockDim.x) {
+        for (int i = 0; i < d; ++i) {   // L y = rhs_j
+            double acc = R[(size_t)i * d + j];
+            for (int k = 0; k < i; ++k) acc -= Ls[i * ld + k] * R[(size_t)k * d + j];
+            R[(size_t)i * d + j] = acc / Ls[i * ld + i];
+        }
+        for (int i = d - 1; i >= 0; --i) {   // L^T b = y
+            double acc = R[(size_t)i * d + j];
+            for (int k = i + 1; k < d; ++k) acc -= Ls[k * ld + i] * R[(size_t)k * d + j];
+            R[(size_t)i * d + j] = acc / Ls[i * ld + i];
+        }
+        for (int i = 0; i < d; ++i) Bout[((size_t)bh * d + i) * d + j] = (float)R[(size_t)i * d + j];
+    }
+}
+
+// O_out[perm_q[p]] for 64 permuted rows per block: probe rows copy O^dense,
+// the others get O^sp + mu_R + ((O^sp - mu_X)/sigma) B.
+template <int D>
+__global__ void __launch_bounds__(256) apply_kernel(const float* __restrict__ O_sp, const float* __restrict__ Bm,
+                                                    const float* __restrict__ mu_x, const float* __restrict__ sigma,
+                                                    const float* __restrict__ mu_r, const int32_t* __restrict__ pslot,
+                                                    const float* __restrict__ probe_dense,
+                                                    const int32_t* __restrict__ perm_q, int N, int Mp,
+                                                    float* __restrict__ O_out) {
+    constexpr int RT = 64, CG = D / 16;   // rows per block, columns per thread
+    extern __shared__ float sm[];
+    float* Bs = sm;                 // [D][D]
+    float* Xs = Bs + D * D;         // [RT][D+4]
+    float* st = Xs + RT * (D + 4);  // mu_x, sigma, mu_r
+    const int bh = blockIdx.y, p0 = blockIdx.x * RT, tid = threadIdx.x;
+    const float* Bh = Bm + (size_t)bh * D * D;
+    for (int e = tid; e < D * D; e += blockDim.x) Bs[e] = Bh[e];
+    for (int e = tid; e < D; e += blockDim.x) {
+        st[e] = mu_x[(size_t)bh * D + e];
+        st[D + e] = sigma[(size_t)bh * D + e];
+        st[2 * D + e] = mu_r[(size_t)bh * D + e];
+    }
+    __syncthreads();
+    for (int e = tid; e < RT * D; e += blockDim.x) {
+        const int r = e / D, t = e % D;
+        const int p = p0 + r;
+        Xs[r * (D + 4) + t] = (p < N) ? (O_sp[((size_t)bh * N + p) * D + t] - st[t]) / st[D + t] : 0.f;
+    }
+    __syncthreads();
+    const int rg = tid / 16, cg = tid % 16;
+    float acc[4][CG];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < CG; ++v) acc[u][v] = 0.f;
+    for (int t = 0; t < D; ++t) {
+        float xb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) xb[u] = Xs[(rg * 4 + u) * (D + 4) + t];
+        const float* br = Bs + t * D + cg * CG;
+#pragma unroll
+        for (int v = 0; v < CG; ++v) {
+            const float b = br[v];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u][v] = fmaf(xb[u], b, acc[u][v]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int p = p0 + rg * 4 + u;
+        if (p >= N) continue;
+        const size_t src = (size_t)bh * N + p;
+        const int slot = pslot[src];
+        float* dst = O_out + ((size_t)bh * N + perm_q[src]) * D + cg * CG;
+        if (slot >= 0) {
+            const float* pd = probe_dense + ((size_t)bh * Mp + slot) * D + cg * CG;
+#pragma unroll
+            for (int v = 0; v < CG; ++v) dst[v] = pd[v];
+        } else {
+            const float* x = O_sp + src * D + cg * CG;
+#pragma unroll
+            for (int v = 0; v < CG; ++v) dst[v] = x[v] + st[2 * D + cg * CG + v] + acc[u][v];
+        }
+    }
+}
+
+// pslot[permuted row] = probe slot, for the probe rows.
+__global__ void probe_slot_kernel(const int32_t* __restrict__ probe_idx, const int32_t* __restrict__ pos_q, int BH,
+                                  int N, int Mp, int32_t* __restrict__ pslot) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= BH * Mp) return;
+    const size_t bh = e / Mp;
+    pslot[bh * N + pos_q[bh * N + probe_idx[e]]] = e - (int)bh * Mp;
+}
+
+__global__ void fill_kernel(float* __restrict__ x, int n, float v) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) x[i] = v;
+}
+
+// ================================================================ host side
+sparsepr_status run_fit(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
+                        const sparsepr_route_out& r, const float* probe_sparse, const float* probe_dense,
+                        const sparsepr_fit_out& f, void* ws, cudaStream_t st) {
+    const int BH = pl.BH, d = pl.d, Mp = pl.Mp;
+    double* fstat = at<double>(ws, pl.o_fstat);
+    double* G = at<double>(ws, pl.o_G);
+    double* rhs = at<double>(ws, pl.o_rhs);
+    const int32_t* alloc = r.probe_alloc;
+    int32_t* psum = at<int32_t>(ws, pl.o_psum);
+    DevStatus* status = at<DevStatus>(ws, pl.o_status);
+    if (Mp == 0) {   // no probes: no correction (B = 0, mu = 0, sigma = 1)
+        cudaMemsetAsync(f.B, 0, (size_t)BH * d * d * 4, st);
+        cudaMemsetAsync(f.mu_x, 0, (size_t)BH * d * 4, st);
+        cudaMemsetAsync(f.mu_r, 0, (size_t)BH * d * 4, st);
+        count_launch(), fill_kernel<<<(BH * d + 255) / 256, 256, 0, st>>>(f.sigma, BH * d, 1.f);
+        return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+    }
+    count_launch(), fit_stats_kernel<<<BH, d, 0, st>>>(probe_sparse, probe_dense, r.probe_group, alloc, part.q_offsets,
+                                       part.n_groups, psum, pl.Cq, Mp, d, p.eps_std, fstat, f.mu_x, f.sigma,
+                                       f.mu_r);
+    count_launch(), fit_gram_kernel<<<dim3(d / 8, BH), d, 0, st>>>(probe_sparse, probe_dense, r.probe_group, alloc, part.q_offsets,
+                                                   psum, pl.Cq, Mp, d, p.lambda, fstat, G, rhs);
+    const size_t smem = (size_t)d * (d + 1) * sizeof(double);
+    cudaFuncSetAttribute(fit_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    count_launch(), fit_solve_kernel<<<BH, d, smem, st>>>(G, rhs, d, f.B, status);
+    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+}
+
+sparsepr_status run_apply(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
+                          const sparsepr_route_out& r, const float* O_sp, const float* probe_dense,
+                          const sparsepr_fit_out& f, float* O_out, void* ws, cudaStream_t st) {
+    (void)p;
+    int32_t* pslot = at<int32_t>(ws, pl.o_pslot);
+    cudaMemsetAsync(pslot, 0xff, (size_t)pl.BH * pl.N * sizeof(int32_t), st);
+    if (pl.Mp > 0)
+        count_launch(), probe_slot_kernel<<<(pl.BH * pl.Mp + 255) / 256, 256, 0, st>>>(r.probe_idx, part.pos_q, pl.BH, pl.N, pl.Mp,
+                                                                       pslot);
+    const int d = pl.d;
+    const size_t smem = (size_t)(d * d + 64 * (d + 4) + 3 * d) * sizeof(float);
+    const dim3 grid((pl.N + 63) / 64, pl.BH);
+    if (d == 128) {
+        cudaFuncSetAttribute(apply_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        count_launch(), apply_kernel<128><<<grid, 256, smem, st>>>(O_sp, f.B, f.mu_x, f.sigma, f.mu_r, pslot, probe_dense,
+                                                  part.perm_q, pl.N, pl.Mp, O_out);
+    } else {
+        cudaFuncSetAttribute(apply_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        count_launch(), apply_kernel<64><<<grid, 256, smem, st>>>(O_sp, f.B, f.mu_x, f.sigma, f.mu_r, pslot, probe_dense,
+                                                 part.perm_q, pl.N, pl.Mp, O_out);
+    }
+    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+}
+
+}  // namespace spr

@@ -1,0 +1,25 @@
+// Stage entry points shared by the C ABI (api.cu) and the stage files.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace spr {
+
+sparsepr_status run_partition(const sparsepr_params& p, const Plan& pl, const void* Q, const void* K,
+                              const void* V, const sparsepr_partition_out& out, void* ws, cudaStream_t st);
+sparsepr_status run_route(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
+                          const sparsepr_route_out& r, void* ws, cudaStream_t st);
+bool attention_uses_tc(const sparsepr_params& p);
+sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
+                              const sparsepr_route_out& r, float* O_sp, float* probe_dense,
+                              float* probe_sparse, void* ws, cudaStream_t st);
+sparsepr_status run_fit(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
+                        const sparsepr_route_out& r, const float* probe_sparse, const float* probe_dense,
+                        const sparsepr_fit_out& f, void* ws, cudaStream_t st);
+sparsepr_status run_apply(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
+                          const sparsepr_route_out& r, const float* O_sp, const float* probe_dense, const sparsepr_fit_out& f, float* O_out,
+                          void* ws, cudaStream_t st);
+
+}  // namespace spr

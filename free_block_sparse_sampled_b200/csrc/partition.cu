@@ -1,0 +1,782 @@
+// Response-coupled partitioning ("Partition the Support, Reconstruct the
+// Residual", §4.1, B.1, B.2, C.1).
+//
+//   M_K = Q_s^T Q_s / M_s over evenly spaced sampled queries
+//   F_K from an FP32 eigendecomposition (parallel cyclic Jacobi, one block/head)
+//   phi_K = K F_K, k-means with C_k requested centres -> paired K/V groups
+//   kbar, vbar, mu_K, M_Q = Ktilde^T Ktilde / (C_k' d), F_Q, phi_Q = RMSNorm(q F_Q)
+//   k-means with C_q requested centres -> query groups, qbar, c_a, d_i
+//
+// Every reduction that feeds an integer decision runs in a fixed order: the
+// k-means centre update sums members in the order of a stable counting sort,
+// never through floating-point atomics.
+#include "common.cuh"
+#include "internal.h"
+
+namespace spr {
+
+// ---------------------------------------------------------------- Gram kernels
+// M_K[bh] = (1/Ms) sum_t q_{s_t} q_{s_t}^T with s_t = floor(t N / Ms)  (paper §4.1, C.2).
+template <typename T>
+__global__ void __launch_bounds__(256) sampled_gram_kernel(const T* __restrict__ X, int N, int d,
+                                                           int Ms_eff, float* __restrict__ out) {
+    const int bh = blockIdx.z, i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    __shared__ float si[32][33], sj[32][33];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const T* Xh = X + (size_t)bh * N * d;
+    for (int t0 = 0; t0 < Ms_eff; t0 += 32) {
+        for (int r = ty; r < 32; r += 8) {
+            const int t = t0 + r;
+            float a = 0.f, b = 0.f;
+            if (t < Ms_eff) {
+                const long long row = (Ms_eff >= N) ? t : ((long long)t * N) / Ms_eff;
+                const T* xr = Xh + row * d;
+                a = ldf(xr + i0 + tx);
+                b = ldf(xr + j0 + tx);
+            }
+            si[r][tx] = a;
+            sj[r][tx] = b;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int r = 0; r < 32; ++r) {
+            const float bj = sj[r][tx];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u] = fmaf(si[r][ty + 8 * u], bj, acc[u]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        out[(size_t)bh * d * d + (size_t)(i0 + ty + 8 * u) * d + j0 + tx] = acc[u] / (float)Ms_eff;
+}
+
+// mu_K = unweighted mean of the C_k' nonempty K-group centroids (paper B.2).
+__global__ void centroid_mean_kernel(const float* __restrict__ cen, const int32_t* __restrict__ ng,
+                                     int Ck, int d, float* __restrict__ mu) {
+    const int bh = blockIdx.x, j = threadIdx.x;
+    const int C = ng[bh * 2 + 1];
+    float s = 0.f;
+    for (int b = 0; b < C; ++b) s += cen[((size_t)bh * Ck + b) * d + j];
+    mu[bh * d + j] = s / (float)C;
+}
+
+// M_Q[bh] = sum_b (kbar_b - mu_K)(kbar_b - mu_K)^T / (C_k' d)  (paper §4.1).
+__global__ void __launch_bounds__(256) centred_gram_kernel(const float* __restrict__ cen,
+                                                           const float* __restrict__ mu,
+                                                           const int32_t* __restrict__ ng, int Ck,
+                                                           int d, float* __restrict__ out) {
+    const int bh = blockIdx.z, i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int C = ng[bh * 2 + 1];
+    __shared__ float si[32][33], sj[32][33];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* base = cen + (size_t)bh * Ck * d;
+    const float mi = mu[bh * d + i0 + tx], mj = mu[bh * d + j0 + tx];
+    for (int t0 = 0; t0 < C; t0 += 32) {
+        for (int r = ty; r < 32; r += 8) {
+            const int t = t0 + r;
+            si[r][tx] = (t < C) ? base[(size_t)t * d + i0 + tx] - mi : 0.f;
+            sj[r][tx] = (t < C) ? base[(size_t)t * d + j0 + tx] - mj : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int r = 0; r < 32; ++r) {
+            const float bj = sj[r][tx];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u] = fmaf(si[r][ty + 8 * u], bj, acc[u]);
+        }
+        __syncthreads();
+    }
+    const float scale = 1.f / ((float)C * (float)d);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        out[(size_t)bh * d * d + (size_t)(i0 + ty + 8 * u) * d + j0 + tx] = acc[u] * scale;
+}
+
+// ---------------------------------------------------------------- eigen factor
+// Parallel cyclic Jacobi (round-robin pairing: d/2 disjoint rotations per
+// round, d-1 rounds per sweep) on one symmetric d x d matrix per block, then
+// F[:, c] = u_c sqrt(max(lambda_c, 0)) * scale for the r leading eigenpairs
+// (descending, ties to the lower index) and zero columns up to Rp.
+// For the query factor (ng != nullptr) r = max(1, min(r_req, d, C_k' - 1)).
+__global__ void __launch_bounds__(512) jacobi_factor_kernel(const float* __restrict__ Ain, int d,
+                                                            float* __restrict__ F, int Rp,
+                                                            int r_req, const int32_t* ng,
+                                                            float scale, int32_t* r_out,
+                                                            int max_sweeps) {
+    extern __shared__ float sm[];
+    const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const int ld = d + 1, half = d / 2;
+    float* A = sm;
+    float* V = A + d * ld;
+    float* cs = V + d * ld;
+    float* sn = cs + half;
+    int* pp = reinterpret_cast<int*>(sn + half);
+    int* qq = pp + half;
+    float* red = reinterpret_cast<float*>(qq + half);   // 64 floats
+    int* order = reinterpret_cast<int*>(red + 64);      // d ints
+
+    const float* Ah = Ain + (size_t)bh * d * d;
+    for (int e = tid; e < d * d; e += nt) {
+        const int i = e / d, j = e % d;
+        A[i * ld + j] = 0.5f * (Ah[i * d + j] + Ah[j * d + i]);
+        V[i * ld + j] = (i == j) ? 1.f : 0.f;
+    }
+    __syncthreads();
+
+    for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+        // convergence: off-diagonal energy vs total energy
+        float off = 0.f, tot = 0.f;
+        for (int e = tid; e < d * d; e += nt) {
+            const int i = e / d, j = e % d;
+            const float a = A[i * ld + j];
+            tot += a * a;
+            if (i != j) off += a * a;
+        }
+        off = warp_sum(off);
+        tot = warp_sum(tot);
+        if ((tid & 31) == 0) {
+            red[tid >> 5] = off;
+            red[32 + (tid >> 5)] = tot;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float o = 0.f, t = 0.f;
+            for (int w = 0; w < nt / 32; ++w) {
+                o += red[w];
+                t += red[32 + w];
+            }
+            red[0] = o;
+            red[32] = t;
+        }
+        __syncthreads();
+        const bool converged = !(red[0] > 1e-13f * red[32]);
+        __syncthreads();
+        if (converged) break;
+
+        for (int round = 0; round < d - 1; ++round) {
+            for (int k = tid; k < half; k += nt) {
+                int p, q;
+                if (k == 0) {
+                    p = round;
+                    q = d - 1;
+                } else {
+                    p = (round + k) % (d - 1);
+                    q = (round - k + (d - 1)) % (d - 1);
+                }
+                if (p > q) {
+                    const int t = p;
+                    p = q;
+                    q = t;
+                }
+                const float apq = A[p * ld + q], app = A[p * ld + p], aqq = A[q * ld + q];
+                float c = 1.f, s = 0.f;
+                if (apq != 0.f) {
+                    const float theta = (aqq - app) / (2.f * apq);
+                    const float t = copysignf(1.f, theta) / (fabsf(theta) + sqrtf(theta * theta + 1.f));
+                    c = 1.f / sqrtf(t * t + 1.f);
+                    s = t * c;
+                }
+                cs[k] = c;
+                sn[k] = s;
+                pp[k] = p;
+                qq[k] = q;
+            }
+            __syncthreads();
+            for (int e = tid; e < half * d; e += nt) {   // rows p, q of J^T A
+                const int k = e / d, j = e % d;
+                const int p = pp[k], q = qq[k];
+                const float c = cs[k], s = sn[k];
+                const float ap = A[p * ld + j], aq = A[q * ld + j];
+                A[p * ld + j] = c * ap - s * aq;
+                A[q * ld + j] = s * ap + c * aq;
+            }
+            __syncthreads();
+            for (int e = tid; e < half * d; e += nt) {   // columns p, q of (J^T A) J and V J
+                const int k = e / d, i = e % d;
+                const int p = pp[k], q = qq[k];
+                const float c = cs[k], s = sn[k];
+                const float ap = A[i * ld + p], aq = A[i * ld + q];
+                A[i * ld + p] = c * ap - s * aq;
+                A[i * ld + q] = s * ap + c * aq;
+                const float vp = V[i * ld + p], vq = V[i * ld + q];
+                V[i * ld + p] = c * vp - s * vq;
+                V[i * ld + q] = s * vp + c * vq;
+            }
+            __syncthreads();
+        }
+    }
+
+    // descending eigenvalue order, ties to the lower index
+    for (int i = tid; i < d; i += nt) {
+        const float li = A[i * ld + i];
+        int rank = 0;
+        for (int j = 0; j < d; ++j) {
+            const float lj = A[j * ld + j];
+            rank += (lj > li) || (lj == li && j < i);
+        }
+        order[rank] = i;
+    }
+    __syncthreads();
+    int r = r_req;
+    if (ng != nullptr) r = max(1, min(min(r_req, d), ng[bh * 2 + 1] - 1));
+    if (tid == 0 && r_out != nullptr) r_out[bh] = r;
+    float* Fh = F + (size_t)bh * d * Rp;
+    for (int e = tid; e < d * Rp; e += nt) {
+        const int i = e / Rp, c = e % Rp;
+        float v = 0.f;
+        if (c < r) {
+            const int col = order[c];
+            v = V[i * ld + col] * sqrtf(fmaxf(A[col * ld + col], 0.f)) * scale;
+        }
+        Fh[e] = v;
+    }
+}
+
+// ---------------------------------------------------------------- projections
+// phi[i] = x_i F (R columns); with RMS: divided by max(sqrt(|x_i F|^2 / r), eps)
+// (paper §4.1 phi_K, B.2 phi_Q).  One thread per row, F in shared memory.
+template <typename T, int R, bool RMS>
+__global__ void __launch_bounds__(128) project_kernel(const T* __restrict__ X,
+                                                      const float* __restrict__ F, int N, int d,
+                                                      const int32_t* __restrict__ r_eff, float eps,
+                                                      float* __restrict__ phi) {
+    extern __shared__ float Fs[];
+    const int bh = blockIdx.y;
+    for (int e = threadIdx.x; e < d * R; e += blockDim.x) Fs[e] = F[(size_t)bh * d * R + e];
+    __syncthreads();
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    const T* x = X + ((size_t)bh * N + i) * d;
+    float acc[R];
+#pragma unroll
+    for (int c = 0; c < R; ++c) acc[c] = 0.f;
+    for (int t0 = 0; t0 < d; t0 += 8) {
+        float v[8];
+        load8(x + t0, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float* Fr = Fs + (t0 + u) * R;
+#pragma unroll
+            for (int c = 0; c < R; ++c) acc[c] = fmaf(v[u], Fr[c], acc[c]);
+        }
+    }
+    if (RMS) {
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < R; ++c) ss = fmaf(acc[c], acc[c], ss);
+        const float den = fmaxf(sqrtf(ss / (float)r_eff[bh]), eps);
+#pragma unroll
+        for (int c = 0; c < R; ++c) acc[c] = acc[c] / den;
+    }
+    float4* out = reinterpret_cast<float4*>(phi + ((size_t)bh * N + i) * R);
+#pragma unroll
+    for (int c = 0; c < R; c += 4) out[c / 4] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+}
+
+// ---------------------------------------------------------------- k-means
+// Initial centres: rows drawn uniformly with replacement (paper C.1) by the
+// SplitMix64 stream of (seed, head, stage).  One warp per centre.
+template <int R>
+__global__ void kmeans_init_kernel(const float* __restrict__ phi, int N, int C, uint64_t seed,
+                                   int stage, float* __restrict__ cen, float* __restrict__ hn) {
+    const int bh = blockIdx.y, lane = threadIdx.x & 31;
+    const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (c >= C) return;
+    const int row = kmeans_init_row(seed, bh, stage, c, N);
+    const float* src = phi + ((size_t)bh * N + row) * R;
+    float* dst = cen + ((size_t)bh * C + c) * R;
+    float ss = 0.f;
+    for (int t = lane; t < R; t += 32) {
+        const float v = src[t];
+        dst[t] = v;
+        ss = fmaf(v, v, ss);
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) hn[(size_t)bh * C + c] = 0.5f * ss;
+}
+
+// Assignment: label = argmax_c (x.c - |c|^2/2), ties to the lowest c.  Labels
+// are updated in place; changed labels are counted per head.
+template <int R>
+__global__ void __launch_bounds__(128) kmeans_assign_kernel(
+    const float* __restrict__ phi, const float* __restrict__ cen, const float* __restrict__ hn,
+    int N, int C, int32_t* __restrict__ labels, int32_t* __restrict__ ctl, int first,
+    float* __restrict__ dbg_scores, int32_t* __restrict__ dbg_hist, int max_iter) {
+    constexpr int CH = 64;
+    __shared__ __align__(16) float cs[CH * R];
+    __shared__ float hs[CH];
+    const int bh = blockIdx.y;
+    int32_t* hc = ctl + bh * kCtlStride;
+    if (hc[kCtlDone]) return;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const bool valid = i < N;
+    float x[R];
+    if (valid) {
+        const float4* src = reinterpret_cast<const float4*>(phi + ((size_t)bh * N + i) * R);
+#pragma unroll
+        for (int t = 0; t < R; t += 4) {
+            const float4 v = src[t / 4];
+            x[t] = v.x; x[t + 1] = v.y; x[t + 2] = v.z; x[t + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int t = 0; t < R; ++t) x[t] = 0.f;
+    }
+    float best = -INFINITY;
+    int bi = 0;
+    const float* ch = cen + (size_t)bh * C * R;
+    for (int c0 = 0; c0 < C; c0 += CH) {
+        const int n = min(CH, C - c0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < n * R; e += blockDim.x) cs[e] = ch[(size_t)c0 * R + e];
+        for (int e = threadIdx.x; e < n; e += blockDim.x) hs[e] = hn[(size_t)bh * C + c0 + e];
+        __syncthreads();
+        for (int cc = 0; cc < n; ++cc) {
+            const float* cr = cs + cc * R;
+            float s = 0.f;
+#pragma unroll
+            for (int t = 0; t < R; ++t) s = fmaf(x[t], cr[t], s);
+            const float sc = s - hs[cc];
+            if (dbg_scores != nullptr && valid) dbg_scores[((size_t)bh * N + i) * C + c0 + cc] = sc;
+            if (sc > best) {
+                best = sc;
+                bi = c0 + cc;
+            }
+        }
+    }
+    int changed = 0;
+    if (valid) {
+        int32_t* lp = labels + (size_t)bh * N + i;
+        changed = (!first) && (*lp != bi);
+        *lp = bi;
+        if (dbg_hist != nullptr) dbg_hist[((size_t)bh * max_iter + hc[kCtlIters]) * N + i] = bi;
+    }
+    const unsigned ballot = __ballot_sync(0xffffffffu, changed);
+    if ((threadIdx.x & 31) == 0 && ballot) atomicAdd(&hc[kCtlChanged], __popc(ballot));
+}
+
+// After each assignment: count it, and stop the head once changed labels <= stop.
+__global__ void kmeans_check_kernel(int32_t* ctl, int BH, int stop, int first) {
+    const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (bh >= BH) return;
+    int32_t* hc = ctl + bh * kCtlStride;
+    if (hc[kCtlDone]) return;
+    hc[kCtlIters] += 1;
+    if (!first && hc[kCtlChanged] <= stop) hc[kCtlDone] = 1;
+    hc[kCtlChanged] = 0;
+}
+
+__global__ void kmeans_reset_kernel(int32_t* ctl, int BH, int save_slot) {
+    const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (bh >= BH) return;
+    int32_t* hc = ctl + bh * kCtlStride;
+    if (save_slot >= 0) hc[save_slot] = hc[kCtlIters];
+    hc[kCtlChanged] = 0;
+    hc[kCtlDone] = 0;
+    hc[kCtlIters] = 0;
+}
+
+// ---- stable counting sort of labels (group-major order, stable by index)
+__global__ void __launch_bounds__(1024) label_hist_kernel(const int32_t* __restrict__ labels, int N,
+                                                          int C, int n_tiles,
+                                                          int32_t* __restrict__ hist,
+                                                          const int32_t* __restrict__ ctl) {
+    const int bh = blockIdx.y, tile = blockIdx.x;
+    if (ctl != nullptr && ctl[bh * kCtlStride + kCtlDone]) return;
+    __shared__ int h[kMaxGroups];
+    for (int c = threadIdx.x; c < C; c += blockDim.x) h[c] = 0;
+    __syncthreads();
+    const int i = tile * kSortTile + threadIdx.x;
+    if (i < N) atomicAdd(&h[labels[(size_t)bh * N + i]], 1);
+    __syncthreads();
+    int32_t* dst = hist + ((size_t)bh * n_tiles + tile) * C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) dst[c] = h[c];
+}
+
+// Turns the per-tile counts into scatter bases and writes group offsets [C+1].
+__global__ void __launch_bounds__(1024) label_scan_kernel(int32_t* __restrict__ hist, int N, int C,
+                                                          int n_tiles, int32_t* __restrict__ offs,
+                                                          const int32_t* __restrict__ ctl) {
+    const int bh = blockIdx.x;
+    if (ctl != nullptr && ctl[bh * kCtlStride + kCtlDone]) return;
+    __shared__ int tot[kMaxGroups];
+    __shared__ int scratch[33];
+    int32_t* hh = hist + (size_t)bh * n_tiles * C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        int run = 0;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int v = hh[(size_t)t * C + c];
+            hh[(size_t)t * C + c] = run;
+            run += v;
+        }
+        tot[c] = run;
+    }
+    __syncthreads();
+    block_exclusive_scan(tot, C, scratch);
+    int32_t* oo = offs + (size_t)bh * (C + 1);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        const int base = tot[c];
+        oo[c] = base;
+        for (int t = 0; t < n_tiles; ++t) hh[(size_t)t * C + c] += base;
+    }
+    if (threadIdx.x == 0) oo[C] = N;
+}
+
+__global__ void __launch_bounds__(1024) label_scatter_kernel(const int32_t* __restrict__ labels, int N,
+                                                             int C, int n_tiles,
+                                                             const int32_t* __restrict__ hist,
+                                                             int32_t* __restrict__ sorted,
+                                                             const int32_t* __restrict__ ctl) {
+    const int bh = blockIdx.y, tile = blockIdx.x;
+    if (ctl != nullptr && ctl[bh * kCtlStride + kCtlDone]) return;
+    __shared__ int cnt[kMaxGroups];
+    const int32_t* base = hist + ((size_t)bh * n_tiles + tile) * C;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) cnt[c] = base[c];
+    __syncthreads();
+    const int i = tile * kSortTile + threadIdx.x;
+    const int lab = (i < N) ? labels[(size_t)bh * N + i] : -1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        if (warp == w) {
+            const unsigned m = __match_any_sync(0xffffffffu, lab);
+            const int leader = __ffs(m) - 1;
+            const int rank = __popc(m & ((1u << lane) - 1u));
+            int start = 0;
+            if (lane == leader && lab >= 0) {
+                start = cnt[lab];
+                cnt[lab] = start + __popc(m);
+            }
+            start = __shfl_sync(0xffffffffu, start, leader);
+            if (lab >= 0) sorted[(size_t)bh * N + start + rank] = i;
+        }
+        __syncthreads();
+    }
+}
+
+// Centre update: member mean in sorted (index) order; empty centres keep
+// their value.  One warp per centre.
+template <int R>
+__global__ void centre_update_kernel(const float* __restrict__ phi, const int32_t* __restrict__ sorted,
+                                     const int32_t* __restrict__ offs, int N, int C,
+                                     float* __restrict__ cen, float* __restrict__ hn,
+                                     const int32_t* __restrict__ ctl) {
+    const int bh = blockIdx.y, lane = threadIdx.x & 31;
+    if (ctl[bh * kCtlStride + kCtlDone]) return;
+    const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (c >= C) return;
+    const int s = offs[(size_t)bh * (C + 1) + c], e = offs[(size_t)bh * (C + 1) + c + 1];
+    if (e == s) return;
+    constexpr int PL = (R + 31) / 32;
+    float acc[PL];
+#pragma unroll
+    for (int u = 0; u < PL; ++u) acc[u] = 0.f;
+    const float* ph = phi + (size_t)bh * N * R;
+    const int32_t* so = sorted + (size_t)bh * N;
+    for (int p = s; p < e; ++p) {
+        const float* row = ph + (size_t)so[p] * R;
+#pragma unroll
+        for (int u = 0; u < PL; ++u) {
+            const int t = lane + 32 * u;
+            if (t < R) acc[u] += row[t];
+        }
+    }
+    const float inv_n = (float)(e - s);
+    float ss = 0.f;
+    float* dst = cen + ((size_t)bh * C + c) * R;
+#pragma unroll
+    for (int u = 0; u < PL; ++u) {
+        const int t = lane + 32 * u;
+        if (t < R) {
+            const float m = acc[u] / inv_n;
+            dst[t] = m;
+            ss = fmaf(m, m, ss);
+        }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) hn[(size_t)bh * C + c] = 0.5f * ss;
+}
+
+// ---------------------------------------------------------------- compaction
+// Nonempty groups renumbered in increasing order of centre index (paper §4.1:
+// C_k counts the nonempty groups).  Writes new ids, compacted offsets (tail
+// filled with N) and the count.
+__global__ void __launch_bounds__(1024) compact_groups_kernel(const int32_t* __restrict__ offs_raw,
+                                                              int C, int N,
+                                                              int32_t* __restrict__ new_id,
+                                                              int32_t* __restrict__ offs_out,
+                                                              int32_t* __restrict__ ng, int which) {
+    const int bh = blockIdx.x;
+    __shared__ int flag[kMaxGroups];
+    __shared__ int scratch[33];
+    const int32_t* o = offs_raw + (size_t)bh * (C + 1);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) flag[c] = (o[c + 1] - o[c]) > 0;
+    __syncthreads();
+    const int total = block_exclusive_scan(flag, C, scratch);
+    int32_t* oo = offs_out + (size_t)bh * (C + 1);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        const bool ne = (o[c + 1] - o[c]) > 0;
+        new_id[(size_t)bh * C + c] = ne ? flag[c] : -1;
+        if (ne) oo[flag[c]] = o[c];
+    }
+    for (int c = total + threadIdx.x; c <= C; c += blockDim.x) oo[c] = N;
+    if (threadIdx.x == 0) ng[bh * 2 + which] = total;
+}
+
+__global__ void relabel_kernel(const int32_t* __restrict__ raw, const int32_t* __restrict__ new_id,
+                               const int32_t* __restrict__ sorted, int BH, int N, int C,
+                               int32_t* __restrict__ label_out, int32_t* __restrict__ perm_out,
+                               int32_t* __restrict__ pos_out) {
+    const size_t total = (size_t)BH * N;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int bh = (int)(e / N);
+        label_out[e] = new_id[(size_t)bh * C + raw[e]];
+        const int src = sorted[e];
+        perm_out[e] = src;
+        if (pos_out != nullptr) pos_out[(size_t)bh * N + src] = (int)(e - (size_t)bh * N);
+    }
+}
+
+// Xp[r] = X[perm[r]] in 16-byte chunks (group-major gather, paper §4.3).
+__global__ void gather_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ perm,
+                                   int BH, int N, int chunks, uint4* __restrict__ Xp) {
+    const size_t total = (size_t)BH * N * chunks;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = e / chunks;
+        const int ch = (int)(e - row * chunks);
+        const size_t bh = row / N;
+        const size_t src = bh * N + perm[row];
+        Xp[e] = X[src * chunks + ch];
+    }
+}
+
+// Mean of the rows of each group in group-major storage (fixed row order).
+template <typename T>
+__global__ void group_mean_kernel(const T* __restrict__ Xp, const int32_t* __restrict__ offs,
+                                  const int32_t* __restrict__ ng, int which, int N, int C, int d,
+                                  float* __restrict__ out) {
+    const int bh = blockIdx.y, g = blockIdx.x, j = threadIdx.x;
+    if (g >= ng[bh * 2 + which]) return;
+    const int s = offs[(size_t)bh * (C + 1) + g], e = offs[(size_t)bh * (C + 1) + g + 1];
+    const T* base = Xp + (size_t)bh * N * d + j;
+    float acc = 0.f;
+    for (int r = s; r < e; ++r) acc += ldf(base + (size_t)r * d);
+    out[((size_t)bh * C + g) * d + j] = acc / (float)(e - s);
+}
+
+// c_a: mean of phi_Q over the members of query group a (members in index order).
+__global__ void group_mean_indirect_kernel(const float* __restrict__ phi,
+                                           const int32_t* __restrict__ perm,
+                                           const int32_t* __restrict__ offs,
+                                           const int32_t* __restrict__ ng, int N, int C, int R,
+                                           float* __restrict__ out) {
+    const int bh = blockIdx.y, g = blockIdx.x, j = threadIdx.x;
+    if (g >= ng[bh * 2 + 0] || j >= R) return;
+    const int s = offs[(size_t)bh * (C + 1) + g], e = offs[(size_t)bh * (C + 1) + g + 1];
+    const int32_t* pr = perm + (size_t)bh * N;
+    float acc = 0.f;
+    for (int r = s; r < e; ++r) acc += phi[((size_t)bh * N + pr[r]) * R + j];
+    out[((size_t)bh * C + g) * R + j] = acc / (float)(e - s);
+}
+
+// d_i = |phi_Q(q_i) - c_a|  (paper A.2), by original row.
+__global__ void query_dist_kernel(const float* __restrict__ phi, const float* __restrict__ ca,
+                                  const int32_t* __restrict__ qlab, int BH, int N, int C, int R,
+                                  float* __restrict__ dist) {
+    const size_t total = (size_t)BH * N;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int bh = (int)(e / N);
+        const float* x = phi + e * R;
+        const float* c = ca + ((size_t)bh * C + qlab[e]) * R;
+        float ss = 0.f;
+        for (int t = 0; t < R; ++t) {
+            const float df = x[t] - c[t];
+            ss = fmaf(df, df, ss);
+        }
+        dist[e] = sqrtf(ss);
+    }
+}
+
+__global__ void iters_out_kernel(const int32_t* __restrict__ ctl, int BH, int32_t* __restrict__ out) {
+    const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (bh >= BH) return;
+    out[bh * 2 + 0] = ctl[bh * kCtlStride + kCtlItersK];
+    out[bh * 2 + 1] = ctl[bh * kCtlStride + kCtlItersQ];
+}
+
+// ================================================================ host side
+namespace {
+
+inline int grid_for(size_t total, int threads) {
+    size_t g = (total + threads - 1) / threads;
+    return (int)(g > 148 * 64 ? 148 * 64 : (g == 0 ? 1 : g));
+}
+
+template <int R>
+void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float* phi, int C,
+                int stage, float* cen, float* hn, float* dbg_scores, int32_t* dbg_hist,
+                int save_slot, cudaStream_t st) {
+    int32_t* ctl = at<int32_t>(ws, pl.o_ctl);
+    int32_t* raw = at<int32_t>(ws, pl.o_raw);
+    int32_t* hist = at<int32_t>(ws, pl.o_hist);
+    int32_t* sorted = at<int32_t>(ws, pl.o_sorted);
+    int32_t* offs = at<int32_t>(ws, pl.o_offs);
+    const int BH = pl.BH, N = pl.N;
+    const int bgrid = (BH + 127) / 128;
+    count_launch(), kmeans_reset_kernel<<<bgrid, 128, 0, st>>>(ctl, BH, save_slot);
+    count_launch(), kmeans_init_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, N, C, p.seed, stage, cen, hn);
+    const dim3 agrid((N + 127) / 128, BH);
+    const dim3 tgrid(pl.n_sort_tiles, BH);
+    for (int it = 0; it < p.kmeans_iters; ++it) {
+        const int first = it == 0;
+        if (!first) {
+            count_launch(), label_hist_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, ctl);
+            count_launch(), label_scan_kernel<<<BH, 1024, 0, st>>>(hist, N, C, pl.n_sort_tiles, offs, ctl);
+            count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, sorted, ctl);
+            count_launch(), centre_update_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, sorted, offs, N, C, cen, hn, ctl);
+        }
+        const bool last = (it == p.kmeans_iters - 1);
+        (void)last;
+        count_launch(), kmeans_assign_kernel<R><<<agrid, 128, 0, st>>>(phi, cen, hn, N, C, raw, ctl, first,
+                                                       dbg_scores, dbg_hist, p.kmeans_iters);
+        count_launch(), kmeans_check_kernel<<<bgrid, 128, 0, st>>>(ctl, BH, pl.stop_changed, first);
+    }
+}
+
+void kmeans_dispatch(int R, const Plan& pl, const sparsepr_params& p, void* ws, const float* phi,
+                     int C, int stage, float* cen, float* hn, float* dbg_scores, int32_t* dbg_hist,
+                     int save_slot, cudaStream_t st) {
+    switch (R) {
+        case 16: kmeans_run<16>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
+        case 32: kmeans_run<32>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
+        case 48: kmeans_run<48>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
+        default: kmeans_run<64>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
+    }
+}
+
+template <typename T, bool RMS>
+void project_dispatch(int R, const T* X, const float* F, int BH, int N, int d, const int32_t* r_eff,
+                      float eps, float* phi, cudaStream_t st) {
+    const dim3 grid((N + 127) / 128, BH);
+    const size_t smem = (size_t)d * R * sizeof(float);
+    switch (R) {
+        case 16: count_launch(), project_kernel<T, 16, RMS><<<grid, 128, smem, st>>>(X, F, N, d, r_eff, eps, phi); break;
+        case 32: count_launch(), project_kernel<T, 32, RMS><<<grid, 128, smem, st>>>(X, F, N, d, r_eff, eps, phi); break;
+        case 48: count_launch(), project_kernel<T, 48, RMS><<<grid, 128, smem, st>>>(X, F, N, d, r_eff, eps, phi); break;
+        default: count_launch(), project_kernel<T, 64, RMS><<<grid, 128, smem, st>>>(X, F, N, d, r_eff, eps, phi); break;
+    }
+}
+
+// Final group sort of raw labels -> compaction -> labels/perm/pos outputs.
+void finalize_groups(const Plan& pl, void* ws, int C, int which, int32_t* label_out,
+                     int32_t* perm_out, int32_t* pos_out, int32_t* offs_out, int32_t* ng,
+                     cudaStream_t st) {
+    int32_t* raw = at<int32_t>(ws, pl.o_raw);
+    int32_t* hist = at<int32_t>(ws, pl.o_hist);
+    int32_t* sorted = at<int32_t>(ws, pl.o_sorted);
+    int32_t* offs = at<int32_t>(ws, pl.o_offs);
+    int32_t* newid = at<int32_t>(ws, pl.o_newid);
+    const int BH = pl.BH, N = pl.N;
+    const dim3 tgrid(pl.n_sort_tiles, BH);
+    count_launch(), label_hist_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, nullptr);
+    count_launch(), label_scan_kernel<<<BH, 1024, 0, st>>>(hist, N, C, pl.n_sort_tiles, offs, nullptr);
+    count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, sorted, nullptr);
+    count_launch(), compact_groups_kernel<<<BH, 1024, 0, st>>>(offs, C, N, newid, offs_out, ng, which);
+    count_launch(), relabel_kernel<<<grid_for((size_t)BH * N, 256), 256, 0, st>>>(raw, newid, sorted, BH, N, C,
+                                                                  label_out, perm_out, pos_out);
+}
+
+void gather(const void* X, const int32_t* perm, const Plan& pl, void* Xp, cudaStream_t st) {
+    const int chunks = pl.d * pl.esz / 16;
+    const size_t total = (size_t)pl.BH * pl.N * chunks;
+    count_launch(), gather_rows_kernel<<<grid_for(total, 256), 256, 0, st>>>(
+        static_cast<const uint4*>(X), perm, pl.BH, pl.N, chunks, static_cast<uint4*>(Xp));
+}
+
+template <typename T>
+sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const T* Q, const T* K,
+                                const T* V, const sparsepr_partition_out& out, void* ws,
+                                cudaStream_t st) {
+    const int BH = pl.BH, N = pl.N, d = pl.d;
+    float* mat = at<float>(ws, pl.o_mat);
+    float* FK = at<float>(ws, pl.o_FK);
+    float* FQ = at<float>(ws, pl.o_FQ);
+    int32_t* rq = at<int32_t>(ws, pl.o_rq);
+    float* phiK = at<float>(ws, pl.o_phiK);
+    float* phiQ = at<float>(ws, pl.o_phiQ);
+    float* cenK = at<float>(ws, pl.o_cenK);
+    float* hnK = at<float>(ws, pl.o_hnK);
+    float* cenQ = at<float>(ws, pl.o_cenQ);
+    float* hnQ = at<float>(ws, pl.o_hnQ);
+    float* muK = at<float>(ws, pl.o_muK);
+    int32_t* ctl = at<int32_t>(ws, pl.o_ctl);
+    const bool dbg = (p.flags & SPARSEPR_FLAG_DEBUG_EXPORT) != 0;
+
+    const size_t jac_smem = (size_t)(2 * d * (d + 1) + 2 * (d / 2) + 64) * sizeof(float) +
+                            (size_t)(2 * (d / 2) + d) * sizeof(int);
+    cudaFuncSetAttribute(jacobi_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)jac_smem);
+
+    // 1-2. key-response metric and factor (§4.1)
+    count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff, mat);
+    count_launch(), jacobi_factor_kernel<<<BH, 512, jac_smem, st>>>(mat, d, FK, pl.RKp, pl.rK_eff, nullptr,
+                                                    1.f / sqrtf((float)d), nullptr, 20);
+    project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, st);
+    // 3. paired K/V groups
+    kmeans_dispatch(pl.RKp, pl, p, ws, phiK, pl.Ck, 0, cenK, hnK, dbg ? out.debug_kv_scores : nullptr,
+                    dbg ? out.debug_kv_hist : nullptr, -1, st);
+    if (out.kv_centres) cudaMemcpyAsync(out.kv_centres, cenK, (size_t)BH * pl.Ck * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    finalize_groups(pl, ws, pl.Ck, 1, out.kv_label, out.perm_kv, nullptr, out.kv_offsets, out.n_groups, st);
+    gather(K, out.perm_kv, pl, out.Kp, st);
+    gather(V, out.perm_kv, pl, out.Vp, st);
+    // 4. centroids, query metric, factor, coordinates (§4.1, B.2)
+    count_launch(), group_mean_kernel<T><<<dim3(pl.Ck, BH), d, 0, st>>>(static_cast<const T*>(out.Kp), out.kv_offsets,
+                                                        out.n_groups, 1, N, pl.Ck, d, out.k_centroid);
+    count_launch(), group_mean_kernel<T><<<dim3(pl.Ck, BH), d, 0, st>>>(static_cast<const T*>(out.Vp), out.kv_offsets,
+                                                        out.n_groups, 1, N, pl.Ck, d, out.v_centroid);
+    count_launch(), centroid_mean_kernel<<<BH, d, 0, st>>>(out.k_centroid, out.n_groups, pl.Ck, d, muK);
+    count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
+                                                                          out.n_groups, pl.Ck, d, mat);
+    count_launch(), jacobi_factor_kernel<<<BH, 512, jac_smem, st>>>(mat, d, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 20);
+    project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, st);
+    // 5. query groups
+    kmeans_dispatch(pl.RQp, pl, p, ws, phiQ, pl.Cq, 1, cenQ, hnQ, dbg ? out.debug_q_scores : nullptr,
+                    dbg ? out.debug_q_hist : nullptr, kCtlItersK, st);
+    count_launch(), kmeans_reset_kernel<<<(BH + 127) / 128, 128, 0, st>>>(ctl, BH, kCtlItersQ);
+    if (out.q_centres) cudaMemcpyAsync(out.q_centres, cenQ, (size_t)BH * pl.Cq * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
+    finalize_groups(pl, ws, pl.Cq, 0, out.q_label, out.perm_q, out.pos_q, out.q_offsets, out.n_groups, st);
+    gather(Q, out.perm_q, pl, out.Qp, st);
+    count_launch(), group_mean_kernel<T><<<dim3(pl.Cq, BH), d, 0, st>>>(static_cast<const T*>(out.Qp), out.q_offsets,
+                                                        out.n_groups, 0, N, pl.Cq, d, out.q_centroid);
+    // c_a (phi_Q space) into the query-centre buffer, then d_i (A.2)
+    count_launch(), group_mean_indirect_kernel<<<dim3(pl.Cq, BH), 64, 0, st>>>(phiQ, out.perm_q, out.q_offsets,
+                                                              out.n_groups, N, pl.Cq, pl.RQp, cenQ);
+    count_launch(), query_dist_kernel<<<grid_for((size_t)BH * N, 256), 256, 0, st>>>(phiQ, cenQ, out.q_label, BH, N,
+                                                                     pl.Cq, pl.RQp, out.q_dist);
+    count_launch(), iters_out_kernel<<<(BH + 127) / 128, 128, 0, st>>>(ctl, BH, out.kmeans_iters_run);
+    if (out.F_K) cudaMemcpyAsync(out.F_K, FK, (size_t)BH * d * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    if (out.F_Q) cudaMemcpyAsync(out.F_Q, FQ, (size_t)BH * d * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
+    if (out.phi_K) cudaMemcpyAsync(out.phi_K, phiK, (size_t)BH * N * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    if (out.phi_Q) cudaMemcpyAsync(out.phi_Q, phiQ, (size_t)BH * N * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
+    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+}
+
+}  // namespace
+
+sparsepr_status run_partition(const sparsepr_params& p, const Plan& pl, const void* Q, const void* K,
+                              const void* V, const sparsepr_partition_out& out, void* ws,
+                              cudaStream_t st) {
+    if (p.dtype == SPARSEPR_BF16)
+        return partition_typed<__nv_bfloat16>(p, pl, static_cast<const __nv_bfloat16*>(Q),
+                                              static_cast<const __nv_bfloat16*>(K),
+                                              static_cast<const __nv_bfloat16*>(V), out, ws, st);
+    return partition_typed<float>(p, pl, static_cast<const float*>(Q), static_cast<const float*>(K),
+                                  static_cast<const float*>(V), out, ws, st);
+}
+
+}  // namespace spr

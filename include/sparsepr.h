@@ -1,0 +1,220 @@
+/*
+ * sparsepr.h -- C ABI of the B200 (sm_100a) SparsePR attention call.
+ *
+ * The operation is one attention call of "Partition the Support, Reconstruct
+ * the Residual: Training-Free Sparse Attention for Video Generation and World
+ * Models" (Taghavi, Langari, Pandey; arXiv 2608.18484v2), written "paper"
+ * below with the section or formula that defines each step:
+ *
+ *   partition  response-coupled partitioning           paper §4.1, B.1, B.2, C.1
+ *   route      value-error score + prefix budget rule   paper §4.3, B.3, A.2
+ *   attention  renormalised block-sparse attention       paper §3 Eq. (2), §4.3
+ *              and exact attention on the probe rows
+ *   probe_fit  weighted ridge on probe residuals         paper §4.2, A.3, D.3
+ *   apply      corrected output, original query order    paper §4.2 (O-hat)
+ *   call       all of the above, fused on one stream
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are caller-owned DEVICE pointers (e.g. from torch).  The library
+ *   allocates no device memory: every intermediate lives in one caller-owned
+ *   device workspace of sparsepr_workspace_size() bytes, 256-byte aligned.
+ * - Q, K, V are [B, H, N, d] row-major, contiguous, in p->dtype (bf16 or
+ *   fp32).  All float outputs are fp32.  Index outputs are int32 unless noted.
+ *   "BH" below is B*H; per-head slices are contiguous.
+ * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *   NULL = legacy default stream) unless documented otherwise.  Group counts
+ *   and list lengths stay on the device; no entry point synchronises except
+ *   sparsepr_call with a non-NULL stats pointer and
+ *   sparsepr_get_device_status.
+ * - Arguments are validated on the host before anything is launched; a
+ *   failed check returns SPARSEPR_INVALID_ARG / UNSUPPORTED /
+ *   WORKSPACE_TOO_SMALL and launches nothing.  A failed launch returns
+ *   SPARSEPR_CUDA_ERROR.  Failures found on the device (a bounded wait that
+ *   ran out, a non-positive Cholesky pivot) are recorded in a status word in
+ *   the workspace, read by sparsepr_get_device_status(); no kernel traps.
+ * - Outputs sized with C_q or C_k are sized for the REQUESTED counts; only the
+ *   first C_q' / C_k' (nonempty groups, reported in n_groups) entries are
+ *   meaningful.
+ */
+#ifndef SPARSEPR_H
+#define SPARSEPR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPARSEPR_OK = 0,
+    SPARSEPR_INVALID_ARG = 1,          /* bad shape, null pointer, value out of range */
+    SPARSEPR_UNSUPPORTED = 2,          /* valid but not built (e.g. d not in {64,128}) */
+    SPARSEPR_WORKSPACE_TOO_SMALL = 3,
+    SPARSEPR_CUDA_ERROR = 4,           /* a CUDA runtime call or launch failed */
+    SPARSEPR_TIMEOUT = 5,              /* device: a bounded wait gave up */
+    SPARSEPR_NUMERIC = 6               /* device: ridge Gram matrix not positive definite */
+} sparsepr_status;
+
+typedef enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 } sparsepr_dtype;
+
+/* flags */
+#define SPARSEPR_FLAG_DEBUG_EXPORT 1   /* fill the debug_* outputs of partition */
+#define SPARSEPR_FLAG_SIMT_ATTENTION 2 /* bf16: use the CUDA-core attention kernel */
+
+/* Problem statement (paper §3 / §4 notation).  All fields are read on the host. */
+typedef struct {
+    int32_t B, H, N, d;        /* batch, heads, tokens, head dim (d in {64,128}) */
+    int32_t T, Y, X;           /* token grid; N must equal T*Y*X (row-major t,y,x) */
+    int32_t dtype;             /* sparsepr_dtype of Q, K, V */
+    double density;            /* target executed-pair density incl. probes (§4.3) */
+    int32_t M;                 /* exact probe rows per head (§4.2); min(M,N) used */
+    int32_t Ms;                /* sampled queries for M_K (§4.1, C.2) */
+    double lambda;             /* ridge coefficient (§4.2), > 0 */
+    int32_t Cq, Ck;            /* requested query / K-V group counts, 1..2048 */
+    int32_t rK, rQ;            /* response ranks (§4.1, B.2), 1..64 */
+    int32_t kmeans_iters;      /* maximum k-means assignments, >= 1 (Table C.1) */
+    double kmeans_tol;         /* stop when changed labels <= floor(tol*N) */
+    uint64_t seed;             /* k-means initial-centre stream seed (C.1) */
+    int32_t block;             /* attention query tile rows: 64 or 128 */
+    float eps_rms;             /* RMSNorm floor in phi_Q (B.2) */
+    float eps_std;             /* variance floor in the standardisation (D.3) */
+    int32_t flags;             /* SPARSEPR_FLAG_* */
+} sparsepr_params;
+
+/* Outputs of sparsepr_partition (paper §4.1).  Required unless marked
+ * optional (NULL = not written).  Sizes: BH*N int32 for per-row arrays. */
+typedef struct {
+    void* Qp; void* Kp; void* Vp; /* [BH,N,d] p->dtype: rows in group-major order,
+                                     stable by original index (§4.3); V keeps its key's row */
+    int32_t* q_label;     /* [BH,N] query group of each ORIGINAL row (0..C_q'-1) */
+    int32_t* kv_label;    /* [BH,N] K/V group of each original key row */
+    int32_t* perm_q;      /* [BH,N] permuted row -> original row */
+    int32_t* perm_kv;     /* [BH,N] */
+    int32_t* pos_q;       /* [BH,N] original row -> permuted row */
+    int32_t* q_offsets;   /* [BH,Cq+1] first permuted row of each query group */
+    int32_t* kv_offsets;  /* [BH,Ck+1] */
+    int32_t* n_groups;    /* [BH,2] (C_q', C_k') nonempty group counts */
+    int32_t* kmeans_iters_run; /* [BH,2] assignments run (K/V, query) */
+    float* q_centroid;    /* [BH,Cq,d] qbar_a: mean of raw query rows (B.3) */
+    float* k_centroid;    /* [BH,Ck,d] kbar_b */
+    float* v_centroid;    /* [BH,Ck,d] vbar_b */
+    float* q_dist;        /* [BH,N] d_i = |phi_Q(q_i) - c_a| by original row (A.2) */
+    /* optional */
+    float* F_K;           /* [BH,d,rK] key factor (columns beyond r_K' zero) */
+    float* F_Q;           /* [BH,d,rQ] query factor (columns beyond r_Q' zero) */
+    float* phi_K;         /* [BH,N,RKp] key coordinates, RKp = rK rounded up to 16 */
+    float* phi_Q;         /* [BH,N,RQp] query coordinates (after RMSNorm) */
+    float* kv_centres;    /* [BH,Ck,RKp] k-means centres used by the last assignment */
+    float* q_centres;     /* [BH,Cq,RQp] */
+    /* optional, only with SPARSEPR_FLAG_DEBUG_EXPORT (small problems) */
+    float* debug_kv_scores;   /* [BH,N,Ck] fp32 scores of the last K/V assignment */
+    float* debug_q_scores;    /* [BH,N,Cq] */
+    int32_t* debug_kv_hist;   /* [BH,kmeans_iters,N] raw labels after each assignment */
+    int32_t* debug_q_hist;    /* [BH,kmeans_iters,N] */
+} sparsepr_partition_out;
+
+/* Outputs of sparsepr_route (paper §4.3, B.3, A.2). */
+typedef struct {
+    float* score;         /* [BH,Cq,Ck] s_ab (B.3), rows a<C_q', cols b<C_k' */
+    uint8_t* mask;        /* [BH,Cq,Ck] z_ab */
+    int32_t* sel_count;   /* [BH,Cq] number of selected K/V groups of group a */
+    int32_t* sel_groups;  /* [BH,Cq,Ck] selected K/V groups of a, ascending, first sel_count */
+    int64_t* pairs;       /* [BH,2] (P_route, P_exec = P_route + min(M,N)*N) */
+    int32_t* probe_idx;   /* [BH,M'] probe rows (original index), M' = min(M,N);
+                             ordered by group, then by (d_i, i) */
+    int32_t* probe_group; /* [BH,M'] query group of each probe */
+    float* probe_weight;  /* [BH,M'] w~_p (unit mean, A.3) */
+    int32_t* probe_alloc; /* [BH,Cq] m_a probes per query group */
+} sparsepr_route_out;
+
+/* Outputs of sparsepr_probe_fit (paper §4.2, A.3). */
+typedef struct {
+    float* B;             /* [BH,d,d] B_lambda (row i, column j) */
+    float* mu_x;          /* [BH,d] */
+    float* sigma;         /* [BH,d] sqrt(weighted var + eps_std) */
+    float* mu_r;          /* [BH,d] */
+} sparsepr_fit_out;
+
+/* Optional statistics of sparsepr_call. */
+typedef struct {
+    float ms_partition, ms_route, ms_attention, ms_fit, ms_apply, ms_total;
+    int64_t pairs_route;    /* summed over heads */
+    int64_t pairs_exec;     /* pairs_route + BH * min(M,N) * N */
+    int64_t pairs_visited;  /* query-key pairs the attention tiles computed (incl. masked) */
+    double rho_exec;        /* pairs_exec / (BH * N * N) */
+    int64_t launches;       /* kernels this call launched (memsets and copies not counted) */
+} sparsepr_stats;
+
+/* Status text for a sparsepr_status value (static string). */
+const char* sparsepr_status_string(int32_t status);
+
+/* Host-side validation of *p; returns SPARSEPR_OK or the first failed check. */
+sparsepr_status sparsepr_validate(const sparsepr_params* p);
+
+/* Bytes of device workspace every entry point below needs for *p (0 if *p is
+ * invalid).  The same workspace may be reused by successive calls on one
+ * stream; calls on different streams need different workspaces. */
+size_t sparsepr_workspace_size(const sparsepr_params* p);
+
+/* §4.1: sampled-query key metric M_K, FP32 eigen-factor F_K, K/V k-means in
+ * phi_K; centroids, M_Q, F_Q, phi_Q = RMSNorm(q F_Q), query k-means;
+ * compaction to nonempty groups, group-major permutation and gather of
+ * Q, K, V, q-bar/k-bar/v-bar and d_i.  Q, K, V: [BH,N,d] device, p->dtype. */
+sparsepr_status sparsepr_partition(const sparsepr_params* p, const void* Q, const void* K,
+                                   const void* V, const sparsepr_partition_out* part,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* §4.3, B.3, A.2: routing scores, per-query-group prefix selection at the key
+ * budget beta = (density - M/N) N, executed-pair counts, stratified probe
+ * selection and coverage weights.  Reads the partition outputs. */
+sparsepr_status sparsepr_route(const sparsepr_params* p, const sparsepr_partition_out* part,
+                               const sparsepr_route_out* route, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Eq. (2) over the selected cells for every permuted query row, plus exact
+ * dense attention for the probe rows.
+ *   O_sp:         [BH,N,d] fp32, PERMUTED query order (row r = part->perm_q[r])
+ *   probe_dense:  [BH,M',d] fp32, O^dense of each probe (route->probe_idx order)
+ *   probe_sparse: [BH,M',d] fp32, O^sp of each probe */
+sparsepr_status sparsepr_attention(const sparsepr_params* p, const sparsepr_partition_out* part,
+                                   const sparsepr_route_out* route, float* O_sp,
+                                   float* probe_dense, float* probe_sparse, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* §4.2 / A.3: coverage weights w_p = |G_a|/m_a (group sizes from
+ * part->q_offsets, m_a from route->probe_alloc), weighted standardisation,
+ * centring and the ridge solve B = (Xbar^T W Xbar + lambda I)^-1 Xbar^T W Rbar
+ * on R = probe_dense - probe_sparse (Cholesky, fp64 internally).  A
+ * non-positive pivot records SPARSEPR_NUMERIC in the device status word and
+ * leaves B = 0. */
+sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const sparsepr_partition_out* part,
+                                   const sparsepr_route_out* route, const float* probe_sparse,
+                                   const float* probe_dense, const sparsepr_fit_out* fit,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* §4.2: O_out[b,h,i] = O^dense for probe rows, O^sp + mu_R + ((O^sp - mu_X)/sigma) B
+ * otherwise, written in ORIGINAL query order.  O_out: [BH,N,d] fp32. */
+sparsepr_status sparsepr_apply(const sparsepr_params* p, const sparsepr_partition_out* part,
+                               const sparsepr_route_out* route, const float* O_sp,
+                               const float* probe_dense, const sparsepr_fit_out* fit,
+                               float* O_out, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* The whole call on one stream: partition -> route -> attention -> fit ->
+ * apply.  O_out: [BH,N,d] fp32 original order.  With stats != NULL the call
+ * records per-stage CUDA events, synchronises the stream and fills *stats. */
+sparsepr_status sparsepr_call(const sparsepr_params* p, const void* Q, const void* K,
+                              const void* V, float* O_out, sparsepr_stats* stats,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads (synchronously on `stream`) and clears the device status word of
+ * `workspace`: *out = SPARSEPR_OK or the first device-side failure. */
+sparsepr_status sparsepr_get_device_status(void* workspace, void* stream, int32_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSEPR_H */
