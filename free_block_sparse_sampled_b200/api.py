@@ -67,11 +67,11 @@ class SparsePRConfig:
     @property
     def RKp(self) -> int:
         r = min(self.rK, self.d, min(self.Ms, self.N))
-        return (r + 15) // 16 * 16
+        return max(32, (r + 15) // 16 * 16)
 
     @property
     def RQp(self) -> int:
-        return (min(self.rQ, self.d) + 15) // 16 * 16
+        return max(32, (min(self.rQ, self.d) + 15) // 16 * 16)
 
     def c_params(self) -> A.Params:
         return A.Params(self.B, self.H, self.N, self.d, self.T, self.Y, self.X,

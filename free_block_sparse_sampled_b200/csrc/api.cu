@@ -28,8 +28,9 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     int rk = p.rK < p.d ? p.rK : p.d;
     rk = rk < pl.Ms_eff ? rk : pl.Ms_eff;
     pl.rK_eff = rk;
-    pl.RKp = round_up(rk, 16);
-    pl.RQp = round_up(p.rQ < p.d ? p.rQ : p.d, 16);
+    // coordinate rows: a multiple of 16 floats and at least one 128-byte TMA chunk
+    pl.RKp = round_up(rk, 16) < 32 ? 32 : round_up(rk, 16);
+    pl.RQp = round_up(p.rQ < p.d ? p.rQ : p.d, 16) < 32 ? 32 : round_up(p.rQ < p.d ? p.rQ : p.d, 16);
     pl.Mp = p.M < p.N ? p.M : p.N;
     pl.esz = p.dtype == SPARSEPR_BF16 ? 2 : 4;
     pl.n_sort_tiles = (p.N + kSortTile - 1) / kSortTile;
@@ -76,6 +77,9 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_fstat = bump(c, BH * 3 * d * 8);
     pl.o_G = bump(c, BH * d * d * 8);
     pl.o_rhs = bump(c, BH * d * d * 8);
+    pl.o_vh = bump(c, p.dtype == SPARSEPR_BF16 ? BH * N * d * 2 : 256);
+    pl.o_vmax = bump(c, BH * 4);
+    pl.o_vscale = bump(c, BH * 4);
     // outputs owned by the workspace (fused call)
     pl.o_Qp = bump(c, BH * N * d * es);
     pl.o_Kp = bump(c, BH * N * d * es);

@@ -16,6 +16,9 @@
 //
 // fp32 inputs (or the SIMT flag): CUDA-core kernel with the same work items.
 #include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
@@ -226,10 +229,11 @@ __global__ void __launch_bounds__(256) attention_simt_kernel(
 
 // ---------------------------------------------------------------- tcgen05 kernel
 namespace tc {
-constexpr int BM = 128, BN = 128, NS = 2;
+constexpr int BM = 128, BN = 128, NS = 2, RING = 4, NBOX = 5;   // boxes of 8 << k rows, k < NBOX
 constexpr uint32_t kSpin = 1u << 20;   // polls of mbarrier.try_wait before giving up
 enum { B_Q = 0, B_KF = 1, B_KE = B_KF + NS, B_VF = B_KE + NS, B_VE = B_VF + NS, B_SF = B_VE + NS,
-       B_SE = B_SF + 2, B_PF = B_SE + 2, B_OD = B_PF + 1, B_DR = B_OD + 1, N_BAR = B_DR + 1 };
+       B_SE = B_SF + 2, B_PF = B_SE + 2, B_OD = B_PF + 1, B_DR = B_OD + 1, B_MF = B_DR + 1,
+       B_ME = B_MF + RING, N_BAR = B_ME + RING };
 
 template <int D>
 struct Layout {
@@ -241,20 +245,56 @@ struct Layout {
     static constexpr int oV = oK + NS * KB;
     static constexpr int oP = oV + NS * KB;
     static constexpr int oBar = oP + PB;
-    static constexpr int oMisc = oBar + N_BAR * 8;
+    static constexpr int oMeta = oBar + N_BAR * 8;  // RING x 16 valid-row counts
+    static constexpr int oMisc = oMeta + RING * 16;
     static constexpr int bytes = oMisc + 64;
     static constexpr int smem = bytes + 1024;      // slack for 1024-byte alignment
 };
+
+// Tensor maps: K (bf16) and V (fp16) rows in boxes of 8, 16, 32, 64, 128 rows x
+// 64 channels; Q and probe-Q in boxes of 128 rows.  All 128-byte swizzled.
+struct Maps {
+    CUtensorMap k[NBOX];
+    CUtensorMap v[NBOX];
+    CUtensorMap q;
+    CUtensorMap qp;
+};
+
+// Loads the 16 slots of one 128-row stage: runs of slots with consecutive
+// rows go out as the fewest power-of-two boxes; padding slots read rows past
+// the end of the tensor, which TMA fills with zeros.
+template <int D>
+__device__ __forceinline__ void load_slots(uint32_t dst, const CUtensorMap* maps, uint32_t bar, const int (&rows)[16],
+                                           int oob) {
+    int u = 0;
+    while (u < 16) {
+        int L = 1;
+        if (rows[u] != oob) {
+            while (u + L < 16 && rows[u + L] == rows[u] + 8 * L) ++L;
+        } else {
+            while (u + L < 16 && rows[u + L] == oob) ++L;
+        }
+        int s = u, rem = L;
+        while (rem > 0) {
+            int k = 31 - __clz(rem);
+            if (k > NBOX - 1) k = NBOX - 1;
+            for (int hh = 0; hh < D / 64; ++hh)
+                sm100::tma_load_2d(dst + hh * BN * 128 + s * 1024, &maps[k], bar, hh * 64, rows[s]);
+            s += 1 << k;
+            rem -= 1 << k;
+        }
+        u += L;
+    }
+}
 }  // namespace tc
 
 template <int D>
 __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
-    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQP,
-    const int4* __restrict__ items, const int32_t* __restrict__ counter, int n_probe_items, int N,
-    int Mp, int Cq, int Ck, const int32_t* __restrict__ kv_off, const int32_t* __restrict__ sel_count,
-    const int32_t* __restrict__ sel_groups, float* __restrict__ O_sp, float* __restrict__ probe_dense,
-    DevStatus* status, unsigned long long* __restrict__ visited, float scale_log2) {
+    const __grid_constant__ tc::Maps maps, const int4* __restrict__ items, const int32_t* __restrict__ counter,
+    int n_probe_items, int N, int Mp, int Cq, int Ck, int total_rows, const int32_t* __restrict__ kv_off,
+    const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_groups, const float* __restrict__ vscale,
+    float* __restrict__ O_sp, float* __restrict__ probe_dense, DevStatus* status,
+    unsigned long long* __restrict__ visited, float scale_log2) {
     using namespace tc;
     using namespace sm100;
     using L = Layout<D>;
@@ -270,6 +310,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
     const uint32_t s_base = smem_u32(sm);
     const uint32_t sQ = s_base + L::oQ, sK = s_base + L::oK, sV = s_base + L::oV, sP = s_base + L::oP;
     auto bar = [&](int i) -> uint32_t { return s_base + L::oBar + 8 * i; };
+    uint8_t* meta = sm + L::oMeta;
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::oMisc);   // [0] tmem, [1] abort, [2] n_tiles
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
@@ -288,6 +329,10 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
         mbar_init(bar(B_PF), 128);
         mbar_init(bar(B_OD), 1);
         mbar_init(bar(B_DR), 1);
+        for (int s = 0; s < RING; ++s) {
+            mbar_init(bar(B_MF + s), 1);
+            mbar_init(bar(B_ME + s), 128);
+        }
         fence_barrier_init();
         misc[1] = 0;
     }
@@ -324,36 +369,37 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
     if (warp == 4) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const CUtensorMap* tq = (it.a < 0) ? &tmQP : &tmQ;
+            const CUtensorMap* tq = (it.a < 0) ? &maps.qp : &maps.q;
             prefetch_tmap(tq);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
             const int qrow = (it.a < 0) ? it.bh * Mp + it.row0 : it.bh * N + it.row0;
             mbar_arrive_expect_tx(bar(B_Q), L::QB);
-            for (int u = 0; u < 16; ++u)
-                for (int hh = 0; hh < D / 64; ++hh)
-                    tma_load_2d(sQ + hh * BM * 128 + u * 1024, tq, bar(B_Q), hh * 64, qrow + 8 * u);
+            for (int hh = 0; hh < D / 64; ++hh) tma_load_2d(sQ + hh * BM * 128, tq, bar(B_Q), hh * 64, qrow);
             SlotCursor cur(it, sel_groups, sel_count, kv_off, Cq, Ck, N);
-            int pad_row = -1, issued_k = 0, issued_v = 0;
+            int issued_k = 0, issued_v = 0;
             for (int j = 0; j < n_tiles; ++j) {
-                const int stage = j % NS, use = j / NS;
+                const int stage = j % NS, use = j / NS, ring = j % RING;
+                int rows[16];
+                uint32_t vw[4] = {0u, 0u, 0u, 0u};
+                for (int u = 0; u < 16; ++u) {
+                    int row, v;
+                    cur.next(row, v);
+                    rows[u] = row >= 0 ? it.bh * N + row : total_rows;
+                    vw[u >> 2] |= (uint32_t)v << (8 * (u & 3));
+                }
+                if (j >= RING && !mbar_wait(bar(B_ME + ring), ((j / RING) - 1) & 1, abort_flag, kSpin)) {
+                    record_status(status, SPARSEPR_TIMEOUT, 40);
+                    *abort_flag = 1;
+                    break;
+                }
+                *reinterpret_cast<uint4*>(meta + ring * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+                mbar_arrive(bar(B_MF + ring));
                 if (j >= NS && !mbar_wait(bar(B_KE + stage), (use - 1) & 1, abort_flag, kSpin)) {
                     record_status(status, SPARSEPR_TIMEOUT, 41);
                     *abort_flag = 1;
                     break;
                 }
-                int rows[16];
-                for (int u = 0; u < 16; ++u) {
-                    int row, v;
-                    cur.next(row, v);
-                    if (pad_row < 0) pad_row = row;
-                    rows[u] = row >= 0 ? row : pad_row;
-                }
                 mbar_arrive_expect_tx(bar(B_KF + stage), L::KB);
-                for (int u = 0; u < 16; ++u)
-                    for (int hh = 0; hh < D / 64; ++hh)
-                        tma_load_2d(sK + stage * L::KB + hh * BN * 128 + u * 1024, &tmK, bar(B_KF + stage),
-                                    hh * 64, it.bh * N + rows[u]);
+                load_slots<D>(sK + stage * L::KB, maps.k, bar(B_KF + stage), rows, total_rows);
                 issued_k = j + 1;
                 if (j >= NS && !mbar_wait(bar(B_VE + stage), (use - 1) & 1, abort_flag, kSpin)) {
                     record_status(status, SPARSEPR_TIMEOUT, 42);
@@ -361,10 +407,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                     break;
                 }
                 mbar_arrive_expect_tx(bar(B_VF + stage), L::KB);
-                for (int u = 0; u < 16; ++u)
-                    for (int hh = 0; hh < D / 64; ++hh)
-                        tma_load_2d(sV + stage * L::KB + hh * BN * 128 + u * 1024, &tmV, bar(B_VF + stage),
-                                    hh * 64, it.bh * N + rows[u]);
+                load_slots<D>(sV + stage * L::KB, maps.v, bar(B_VF + stage), rows, total_rows);
                 issued_v = j + 1;
             }
             // every copy this CTA issued lands before the CTA can exit (abort or not)
@@ -378,8 +421,8 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            constexpr uint32_t idesc_qk = idesc_f32acc(128, 128, kFmtBF16, false);
+            constexpr uint32_t idesc_pv = idesc_f32acc(128, D, kFmtF16, true);
             bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
             auto issue_pv = [&](int t) -> bool {
                 const int stage = t % NS;
@@ -390,7 +433,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t a = smem_desc(sP + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
                     const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
-                    mma_bf16_ss(tO, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_f16_ss(tO, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(B_OD));
                 mma_commit(bar(B_VE + stage));
@@ -406,7 +449,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t a = smem_desc(sQ + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
                     const uint64_t b = smem_desc(sK + stage * L::KB + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
-                    mma_bf16_ss(tS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_f16_ss(tS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(B_SF + sb));
                 mma_commit(bar(B_KE + stage));
@@ -429,9 +472,8 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         uint8_t* prow = sm + L::oP + r * 128;
-        SlotCursor cur(it, sel_groups, sel_count, kv_off, Cq, Ck, N);
         for (int j = 0; j < n_tiles; ++j) {
-            const int sb = j & 1;
+            const int sb = j & 1, ring = j % RING;
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + sb), (j / 2) & 1, abort_flag, kSpin));
             if (!ok) break;
             tc_fence_after();
@@ -446,11 +488,15 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(B_SE + sb));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_MF + ring), (j / RING) & 1, abort_flag, kSpin));
+            if (!ok) break;
+            const uint4 vw = *reinterpret_cast<const uint4*>(meta + ring * 16);
+            mbar_arrive(bar(B_ME + ring));
+            const uint32_t vwa[4] = {vw.x, vw.y, vw.z, vw.w};
             float mx = -INFINITY;
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                int row_unused, v;
-                cur.next(row_unused, v);
+                const int v = (int)((vwa[u >> 2] >> (8 * (u & 3))) & 0xffu);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float x = (i < v) ? s[u * 8 + i] * scale_log2 : -INFINITY;
@@ -467,7 +513,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 tc_fence_after();
             }
             if (__any_sync(0xffffffffu, need)) {
-                const float alpha = need ? exp2f(m_ref - m_new) : 1.f;
+                const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
                 if (need) {
                     m_ref = m_new;
                     l *= alpha;
@@ -483,15 +529,15 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 }
                 tmem_wait_st();
             }
-            // P = exp2(s - m_ref) as bf16 into the swizzled K-major P tile
+            // P = exp2(s - m_ref) as fp16 (<= 2^8) into the swizzled K-major P tile
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 uint32_t w[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const __nv_bfloat162 pr = __floats2bfloat162_rn(exp2f(s[u * 8 + 2 * i] - m_ref),
-                                                                    exp2f(s[u * 8 + 2 * i + 1] - m_ref));
-                    const float2 back = __bfloat1622float2(pr);
+                    const __half2 pr = __floats2half2_rn(ex2_approx(s[u * 8 + 2 * i] - m_ref),
+                                                         ex2_approx(s[u * 8 + 2 * i + 1] - m_ref));
+                    const float2 back = __half22float2(pr);
                     l += back.x + back.y;
                     w[i] = *reinterpret_cast<const uint32_t*>(&pr);
                 }
@@ -509,7 +555,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 tc_fence_after();
                 float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + it.row0 + r) * D
                                         : O_sp + ((size_t)it.bh * N + it.row0 + r) * D;
-                const float inv = 1.f / l;
+                const float inv = vscale[it.bh] / l;
 #pragma unroll
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     float v[32];
@@ -538,6 +584,50 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
     }
 }
 
+// ---------------------------------------------------------------- V for the tensor-core kernel
+// The P V product runs in fp16 (P <= 2^8 keeps 11 mantissa bits).  V is
+// copied to fp16 with an exact per-head power-of-two scale that keeps
+// |v| <= 2^14; the output is multiplied back by that power of two.
+__global__ void vmax_kernel(const __nv_bfloat16* __restrict__ V, size_t per_head, unsigned* __restrict__ vmax) {
+    const int bh = blockIdx.y;
+    const __nv_bfloat16* v = V + (size_t)bh * per_head;
+    float m = 0.f;
+    for (size_t e = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; e < per_head;
+         e += (size_t)gridDim.x * blockDim.x * 8) {
+        float x[8];
+        load8(v + e, x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+    }
+    m = warp_max(m);
+    if ((threadIdx.x & 31) == 0) atomicMax(&vmax[bh], __float_as_uint(m));
+}
+
+__global__ void vconvert_kernel(const __nv_bfloat16* __restrict__ V, size_t per_head, const unsigned* __restrict__ vmax,
+                                __half* __restrict__ VH, float* __restrict__ vscale) {
+    const int bh = blockIdx.y;
+    const float mx = __uint_as_float(vmax[bh]);
+    int k = 0;
+    if (mx > 16384.f && isfinite(mx)) {
+        int e;
+        frexpf(mx, &e);
+        k = e - 14;
+    }
+    const float s = ldexpf(1.f, -k);
+    if (blockIdx.x == 0 && threadIdx.x == 0) vscale[bh] = ldexpf(1.f, k);
+    const __nv_bfloat16* v = V + (size_t)bh * per_head;
+    __half* h = VH + (size_t)bh * per_head;
+    for (size_t e = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; e < per_head;
+         e += (size_t)gridDim.x * blockDim.x * 8) {
+        float x[8];
+        load8(v + e, x);
+        __half2 o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = __floats2half2_rn(x[2 * i] * s, x[2 * i + 1] * s);
+        *reinterpret_cast<uint4*>(h + e) = *reinterpret_cast<const uint4*>(o);
+    }
+}
+
 // ================================================================ host side
 namespace {
 
@@ -557,17 +647,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, d] bf16 row-major, boxes of 8 rows x 64 channels, 128-byte swizzle.
-bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+// [rows, d] row-major 16-bit elements, boxes of box_rows rows x 64 channels, 128-byte swizzle.
+bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows, bool fp16) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr || rows == 0) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    const cuuint32_t box[2] = {64, 8};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     const cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 inline int grid_for(size_t total, int threads) {
@@ -607,27 +697,40 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
     const int grid = pl.n_probe_items + pl.n_items_max;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)d);
     if (attention_uses_tc(p)) {
-        CUtensorMap mQ, mK, mV, mQP;
-        bool ok = make_rows_map(&mQ, part.Qp, (uint64_t)BH * N, d) && make_rows_map(&mK, part.Kp, (uint64_t)BH * N, d) &&
-                  make_rows_map(&mV, part.Vp, (uint64_t)BH * N, d);
-        if (!ok) return SPARSEPR_CUDA_ERROR;
-        if (Mp > 0) {
-            if (!make_rows_map(&mQP, qprobe, (uint64_t)BH * Mp, d)) return SPARSEPR_CUDA_ERROR;
-        } else {
-            mQP = mQ;
+        __half* VH = at<__half>(ws, pl.o_vh);
+        unsigned* vmax = at<unsigned>(ws, pl.o_vmax);
+        float* vscale = at<float>(ws, pl.o_vscale);
+        const size_t per_head = (size_t)N * d;
+        cudaMemsetAsync(vmax, 0, (size_t)BH * sizeof(unsigned), st);
+        const dim3 vgrid((unsigned)std::min<size_t>((per_head / 8 + 255) / 256, 148), BH);
+        count_launch(), vmax_kernel<<<vgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(part.Vp), per_head, vmax);
+        count_launch(), vconvert_kernel<<<vgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(part.Vp), per_head,
+                                                              vmax, VH, vscale);
+        tc::Maps maps;
+        const uint64_t rows = (uint64_t)BH * N;
+        bool ok = true;
+        for (int k = 0; k < tc::NBOX; ++k) {
+            ok = ok && make_rows_map(&maps.k[k], part.Kp, rows, d, 8 << k, false);
+            ok = ok && make_rows_map(&maps.v[k], VH, rows, d, 8 << k, true);
         }
+        ok = ok && make_rows_map(&maps.q, part.Qp, rows, d, 128, false);
+        if (Mp > 0) ok = ok && make_rows_map(&maps.qp, qprobe, (uint64_t)BH * Mp, d, 128, false);
+        else maps.qp = maps.q;
+        if (!ok) return SPARSEPR_CUDA_ERROR;
         if (d == 128) {
             auto k = attention_tc_kernel<128>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<128>::smem);
-            count_launch(), k<<<grid, 192, tc::Layout<128>::smem, st>>>(mQ, mK, mV, mQP, items, counter, pl.n_probe_items, N, Mp,
-                                                       pl.Cq, pl.Ck, part.kv_offsets, r.sel_count, r.sel_groups,
-                                                       O_sp, probe_dense, status, visited, scale_log2);
+            count_launch(), k<<<grid, 192, tc::Layout<128>::smem, st>>>(maps, items, counter, pl.n_probe_items, N, Mp,
+                                                                       pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
+                                                                       r.sel_count, r.sel_groups, vscale, O_sp,
+                                                                       probe_dense, status, visited, scale_log2);
         } else {
             auto k = attention_tc_kernel<64>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<64>::smem);
-            count_launch(), k<<<grid, 192, tc::Layout<64>::smem, st>>>(mQ, mK, mV, mQP, items, counter, pl.n_probe_items, N, Mp,
-                                                      pl.Cq, pl.Ck, part.kv_offsets, r.sel_count, r.sel_groups,
-                                                      O_sp, probe_dense, status, visited, scale_log2);
+            count_launch(), k<<<grid, 192, tc::Layout<64>::smem, st>>>(maps, items, counter, pl.n_probe_items, N, Mp,
+                                                                      pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
+                                                                      r.sel_count, r.sel_groups, vscale, O_sp,
+                                                                      probe_dense, status, visited, scale_log2);
         }
     } else {
         const int threads = 2 * pl.BM;

@@ -66,6 +66,13 @@ __device__ __forceinline__ float warp_max(float x) {
     return x;
 }
 
+// Round to TF32 (10 explicit mantissa bits), nearest even.
+__device__ __forceinline__ float tf32_round(float x) {
+    uint32_t r;
+    asm("cvt.rn.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
 // Order-preserving map of a float to uint32 (ascending floats -> ascending keys).
 __device__ __forceinline__ uint32_t float_order_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -100,7 +107,7 @@ struct Plan {
     // internal buffers (byte offsets into the workspace)
     size_t o_status, o_ctl, o_mat, o_FK, o_FQ, o_rq, o_phiK, o_phiQ, o_cenK, o_hnK, o_cenQ, o_hnQ,
         o_raw, o_hist, o_sorted, o_offs, o_newid, o_muK, o_t1, o_t2, o_mloc, o_pslot, o_palloc,
-        o_poff, o_psum, o_qprobe, o_work, o_fstat, o_G, o_rhs;
+        o_poff, o_psum, o_qprobe, o_work, o_fstat, o_G, o_rhs, o_vh, o_vmax, o_vscale;
     // outputs owned by the workspace for sparsepr_call
     size_t o_Qp, o_Kp, o_Vp, o_qlab, o_kvlab, o_permq, o_permk, o_posq, o_qoff, o_kvoff, o_ng, o_its,
         o_qcen, o_kcen, o_vcen, o_qdist, o_score, o_mask, o_selc, o_selg, o_pairs, o_pidx, o_pgrp,

@@ -1,0 +1,255 @@
+// k-means assignment on the tensor cores ("Partition the Support, Reconstruct
+// the Residual", §4.1, C.1): label = argmax_c (x.c - |c|^2/2), ties to the
+// lowest c, for 128 points per block against every centre.
+//
+// Coordinates and centres are stored TF32-rounded (round to nearest even),
+// so the tcgen05 kind::tf32 products are exact and the scores carry only fp32
+// accumulation error.  Centres stream through shared memory in blocks of up
+// to 256 (TMA, 128-byte swizzle, two stages); the scores of a block land in
+// TMEM (two buffers) and eight epilogue warps (two per TMEM lane quadrant,
+// each owning half of the columns) take the running argmax while the next
+// block multiplies.  All waits are bounded.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace spr {
+namespace kmtc {
+constexpr int BP = 128;                 // points per block (TMEM lanes)
+constexpr int NBMAX = 256;              // centres per MMA block
+constexpr uint32_t kSpin = 1u << 20;
+enum { B_A = 0, B_BF = 1, B_BE = 3, B_DF = 5, B_DE = 7, B_DR = 9, N_BAR = 10 };
+constexpr int oA = 0;                                   // 2 chunks x 128 rows x 128 B
+constexpr int oB = oA + 2 * BP * 128;                   // 2 stages x 2 chunks x 256 rows x 128 B
+constexpr int oBar = oB + 2 * 2 * NBMAX * 128;
+constexpr int oRed = oBar + N_BAR * 8;                  // 128 x (score, index) of the upper half
+constexpr int oMisc = oRed + BP * 8;
+constexpr int kSmem = oMisc + 64 + 1024;
+
+struct Maps {
+    CUtensorMap pts;       // [BH*N, R] fp32, box 32 x 128
+    CUtensorMap cen;       // [BH*C, R] fp32, box 32 x NB
+};
+}  // namespace kmtc
+
+__global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
+    const __grid_constant__ kmtc::Maps maps, const float* __restrict__ hn, int N, int C, int R, int NB, int nblk,
+    int32_t* __restrict__ labels, int32_t* __restrict__ ctl, int first, float* __restrict__ dbg_scores,
+    int32_t* __restrict__ dbg_hist, int max_iter, DevStatus* status) {
+    using namespace kmtc;
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int bh = blockIdx.y, p0 = blockIdx.x * BP;
+    int32_t* hc = ctl + bh * kCtlStride;
+    if (hc[kCtlDone]) return;
+    if (*reinterpret_cast<volatile const int32_t*>(&status->code) != 0) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t s_base = smem_u32(sm);
+    auto bar = [&](int i) -> uint32_t { return s_base + oBar + 8 * i; };
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + oMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    const int nchunk = (R + 31) / 32;           // 32 fp32 per 128-byte row chunk
+    const int ksteps = R / 8;                   // kind::tf32 K = 8 per instruction
+
+    if (tid == 0) {
+        mbar_init(bar(B_A), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_BF + s), 1);
+            mbar_init(bar(B_BE + s), 1);
+            mbar_init(bar(B_DF + s), 1);
+            mbar_init(bar(B_DE + s), 256);
+        }
+        mbar_init(bar(B_DR), 1);
+        fence_barrier_init();
+        misc[1] = 0;
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(misc), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (warp == 8) {
+        if (lane == 0) {   // TMA producer
+            prefetch_tmap(&maps.pts);
+            prefetch_tmap(&maps.cen);
+            mbar_arrive_expect_tx(bar(B_A), nchunk * BP * 128);
+            for (int ch = 0; ch < nchunk; ++ch)
+                tma_load_2d(s_base + oA + ch * BP * 128, &maps.pts, bar(B_A), ch * 32, bh * N + p0);
+            int issued = 0;
+            for (int blk = 0; blk < nblk; ++blk) {
+                const int stage = blk & 1;
+                if (blk >= 2 && !mbar_wait(bar(B_BE + stage), ((blk >> 1) - 1) & 1, abort_flag, kSpin)) {
+                    record_status(status, SPARSEPR_TIMEOUT, 20);
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(bar(B_BF + stage), nchunk * NB * 128);
+                for (int ch = 0; ch < nchunk; ++ch)
+                    tma_load_2d(s_base + oB + (stage * 2 + ch) * NBMAX * 128, &maps.cen, bar(B_BF + stage), ch * 32,
+                                bh * C + blk * NB);
+                issued = blk + 1;
+            }
+            mbar_wait(bar(B_A), 0, nullptr, kSpin);
+            for (int t = max(0, issued - 2); t < issued; ++t)
+                mbar_wait(bar(B_BF + (t & 1)), (t >> 1) & 1, nullptr, kSpin);
+        }
+    } else if (warp == 9) {
+        if (lane == 0) {   // MMA issuer
+            const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NB >> 3) << 17) |
+                                   ((uint32_t)(BP >> 4) << 24);   // F32 <- TF32 x TF32, K-major both
+            bool ok = mbar_wait(bar(B_A), 0, abort_flag, kSpin);
+            for (int blk = 0; ok && blk < nblk; ++blk) {
+                const int stage = blk & 1;
+                if (!mbar_wait(bar(B_BF + stage), (blk >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                if (blk >= 2 && !mbar_wait(bar(B_DE + stage), ((blk >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                tc_fence_after();
+                for (int kk = 0; kk < ksteps; ++kk) {
+                    const uint64_t a = smem_desc(s_base + oA + (kk / 4) * BP * 128 + (kk % 4) * 32, 16, 1024);
+                    const uint64_t b = smem_desc(s_base + oB + (stage * 2 + kk / 4) * NBMAX * 128 + (kk % 4) * 32, 16, 1024);
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem + stage * NB),
+                        "l"(a), "l"(b), "r"(idesc), "r"(kk > 0 ? 1u : 0u)
+                        : "memory");
+                }
+                mma_commit(bar(B_DF + stage));
+                mma_commit(bar(B_BE + stage));
+            }
+            if (!ok) {
+                record_status(status, SPARSEPR_TIMEOUT, 21);
+                *abort_flag = 1;
+            }
+            mma_commit(bar(B_DR));
+            mbar_wait(bar(B_DR), 0, nullptr, kSpin);
+        }
+    } else {
+        // epilogue: warps 0-3 take the lower half of each centre block, 4-7 the upper half
+        const int half = warp >> 2, row = (warp & 3) * 32 + lane;
+        const int p = p0 + row;
+        const bool valid = p < N;
+        const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const int hw = NB / 2;
+        float best = -INFINITY;
+        int bi = 0x7fffffff;
+        bool ok = true;
+        for (int blk = 0; blk < nblk; ++blk) {
+            const int db = blk & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + db), (blk >> 1) & 1, abort_flag, kSpin));
+            if (!ok) break;
+            tc_fence_after();
+            for (int c0 = 0; c0 < hw; c0 += 32) {
+                float v[32];
+                tmem_ld32(t_row + db * NB + half * hw + c0, v);
+                tmem_wait_ld();
+                const int cb = blk * NB + half * hw + c0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int c = cb + i;
+                    if (c < C) {
+                        const float sc = v[i] - __ldg(hn + (size_t)bh * C + c);
+                        if (dbg_scores != nullptr && valid) dbg_scores[((size_t)bh * N + p) * C + c] = sc;
+                        if (sc > best) {
+                            best = sc;
+                            bi = c;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_DE + db));
+        }
+        float* red_s = reinterpret_cast<float*>(sm + oRed);
+        int* red_i = reinterpret_cast<int*>(sm + oRed + BP * 4);
+        if (half == 1) {
+            red_s[row] = best;
+            red_i[row] = bi;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (half == 0) {
+            const float b1 = red_s[row];
+            const int i1 = red_i[row];
+            if (b1 > best || (b1 == best && i1 < bi)) {
+                best = b1;
+                bi = i1;
+            }
+            if (bi == 0x7fffffff) bi = 0;
+            int changed = 0;
+            if (valid && ok) {
+                int32_t* lp = labels + (size_t)bh * N + p;
+                changed = (!first) && (*lp != bi);
+                *lp = bi;
+                if (dbg_hist != nullptr) dbg_hist[((size_t)bh * max_iter + hc[kCtlIters]) * N + p] = bi;
+            }
+            const unsigned ballot = __ballot_sync(0xffffffffu, changed);
+            if (lane == 0 && ballot) atomicAdd(&hc[kCtlChanged], __popc(ballot));
+        }
+        if (!ok) {
+            record_status(status, SPARSEPR_TIMEOUT, 22);
+            *abort_flag = 1;
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ================================================================ host side
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn_km() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+bool make_f32_map(CUtensorMap* m, const void* base, uint64_t rows, int R, int box_rows) {
+    EncodeTiledFn fn = encode_fn_km();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)R, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)R * 4};
+    const cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+void kmeans_centre_blocks(int C, int& NB, int& nblk) {
+    nblk = (C + kmtc::NBMAX - 1) / kmtc::NBMAX;
+    NB = round_up((C + nblk - 1) / nblk, 64);
+    if (NB > kmtc::NBMAX) NB = kmtc::NBMAX;
+}
+
+bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, int BH, int N, int C, int R,
+                             int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
+                             int max_iter, DevStatus* status, cudaStream_t st) {
+    int NB, nblk;
+    kmeans_centre_blocks(C, NB, nblk);
+    kmtc::Maps maps;
+    if (!make_f32_map(&maps.pts, phi, (uint64_t)BH * N, R, kmtc::BP)) return false;
+    if (!make_f32_map(&maps.cen, cen, (uint64_t)BH * C, R, NB)) return false;
+    cudaFuncSetAttribute(kmeans_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
+    count_launch(), kmeans_assign_tc_kernel<<<dim3((N + kmtc::BP - 1) / kmtc::BP, BH), 320, kmtc::kSmem, st>>>(
+        maps, hn, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
+    return true;
+}
+
+}  // namespace spr

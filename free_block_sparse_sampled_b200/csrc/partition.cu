@@ -271,9 +271,12 @@ __global__ void __launch_bounds__(128) project_kernel(const T* __restrict__ X,
 #pragma unroll
         for (int c = 0; c < R; ++c) acc[c] = acc[c] / den;
     }
+    // k-means runs on TF32 coordinates (exact products on the tensor cores)
     float4* out = reinterpret_cast<float4*>(phi + ((size_t)bh * N + i) * R);
 #pragma unroll
-    for (int c = 0; c < R; c += 4) out[c / 4] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+    for (int c = 0; c < R; c += 4)
+        out[c / 4] = make_float4(tf32_round(acc[c]), tf32_round(acc[c + 1]), tf32_round(acc[c + 2]),
+                                 tf32_round(acc[c + 3]));
 }
 
 // ---------------------------------------------------------------- k-means
@@ -456,8 +459,8 @@ __global__ void __launch_bounds__(1024) label_scatter_kernel(const int32_t* __re
     }
 }
 
-// Centre update: member mean in sorted (index) order; empty centres keep
-// their value.  One warp per centre.
+// Centre update: member mean in sorted (index) order, rounded to TF32; empty
+// centres keep their value.  One warp per centre.
 template <int R>
 __global__ void centre_update_kernel(const float* __restrict__ phi, const int32_t* __restrict__ sorted,
                                      const int32_t* __restrict__ offs, int N, int C,
@@ -483,14 +486,14 @@ __global__ void centre_update_kernel(const float* __restrict__ phi, const int32_
             if (t < R) acc[u] += row[t];
         }
     }
-    const float inv_n = (float)(e - s);
+    const float count = (float)(e - s);
     float ss = 0.f;
     float* dst = cen + ((size_t)bh * C + c) * R;
 #pragma unroll
     for (int u = 0; u < PL; ++u) {
         const int t = lane + 32 * u;
         if (t < R) {
-            const float m = acc[u] / inv_n;
+            const float m = tf32_round(acc[u] / count);
             dst[t] = m;
             ss = fmaf(m, m, ss);
         }
@@ -640,10 +643,10 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
             count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, sorted, ctl);
             count_launch(), centre_update_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, sorted, offs, N, C, cen, hn, ctl);
         }
-        const bool last = (it == p.kmeans_iters - 1);
-        (void)last;
-        count_launch(), kmeans_assign_kernel<R><<<agrid, 128, 0, st>>>(phi, cen, hn, N, C, raw, ctl, first,
-                                                       dbg_scores, dbg_hist, p.kmeans_iters);
+        if (!launch_kmeans_assign_tc(phi, cen, hn, BH, N, C, R, raw, ctl, first, dbg_scores, dbg_hist,
+                                     p.kmeans_iters, at<DevStatus>(ws, pl.o_status), st))
+            count_launch(), kmeans_assign_kernel<R><<<agrid, 128, 0, st>>>(phi, cen, hn, N, C, raw, ctl, first,
+                                                                          dbg_scores, dbg_hist, p.kmeans_iters);
         count_launch(), kmeans_check_kernel<<<bgrid, 128, 0, st>>>(ctl, BH, pl.stop_changed, first);
     }
 }

@@ -132,18 +132,27 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
     return desc;
 }
 
-// Instruction descriptor for kind::f16 with BF16 A/B and FP32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+// Instruction descriptor for kind::f16 with FP32 accumulation; A and B share
+// one format: 0 = F16, 1 = BF16.
+constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t ab_format, bool b_mn_major) {
     return (1u << 4)                       // D format: F32
-           | (1u << 7)                     // A format: BF16
-           | (1u << 10)                    // B format: BF16
+           | (ab_format << 7)              // A format
+           | (ab_format << 10)             // B format
            | ((b_mn_major ? 1u : 0u) << 16)
            | ((uint32_t)(N >> 3) << 17)
            | ((uint32_t)(M >> 4) << 24);
 }
 
+// Hardware base-2 exponential (MUFU); exp2(-inf) = +0.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // D[tmem] (+)= A[smem] * B[smem]
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"

@@ -19,6 +19,9 @@ path and the oracle read bit-identical values.
 
 from __future__ import annotations
 
+import concurrent.futures
+import os
+
 import numpy as np
 
 from .workloads import Workload
@@ -29,9 +32,10 @@ _PERIODS = 2.0 * 32.0 ** (np.arange(8) / 7.0)
 def bf16_round(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); returns float32."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    u = x.view(np.uint32)
+    # finite inputs: the sum stays below 2^32
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32)
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -106,9 +110,15 @@ def generate_inputs(w: Workload, heads=None, bits: bool = False):
     dt = np.uint16 if use_bits else np.float32
     out = [np.zeros((w.B, w.H, w.N, w.d), dtype=dt) for _ in range(3)]
     todo = heads if heads is not None else [(b, h) for b in range(w.B) for h in range(w.H)]
-    for b, h in todo:
+
+    def fill(bh):
+        b, h = bh
         for dst, src in zip(out, generate_head(w, b, h)):
             dst[b, h] = bf16_bits(src) if use_bits else src
+
+    # heads draw from independent streams, so threads do not change the values
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, todo))
     return tuple(out)
 
 
