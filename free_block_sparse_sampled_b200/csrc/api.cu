@@ -80,6 +80,10 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_vh = bump(c, p.dtype == SPARSEPR_BF16 ? BH * N * d * 2 : 256);
     pl.o_vmax = bump(c, BH * 4);
     pl.o_vscale = bump(c, BH * 4);
+    pl.o_qsplit = bump(c, BH * 3 * (size_t)round_up(p.Cq, 128) * d * 2);
+    pl.o_uw = bump(c, BH * N * 8);
+    pl.o_lbar = bump(c, BH * Cq * Ck * 4);
+    pl.o_vv = bump(c, BH * Ck * 4);
     // outputs owned by the workspace (fused call)
     pl.o_Qp = bump(c, BH * N * d * es);
     pl.o_Kp = bump(c, BH * N * d * es);

@@ -232,21 +232,22 @@ namespace tc {
 constexpr int BM = 128, BN = 128, NS = 2, RING = 4, NBOX = 5;   // boxes of 8 << k rows, k < NBOX
 constexpr uint32_t kSpin = 1u << 20;   // polls of mbarrier.try_wait before giving up
 enum { B_Q = 0, B_KF = 1, B_KE = B_KF + NS, B_VF = B_KE + NS, B_VE = B_VF + NS, B_SF = B_VE + NS,
-       B_SE = B_SF + 2, B_PF = B_SE + 2, B_OD = B_PF + 1, B_DR = B_OD + 1, B_MF = B_DR + 1,
+       B_SE = B_SF + 2, B_PF = B_SE + 2, B_OD = B_PF + 2, B_DR = B_OD + 2, B_MF = B_DR + 1,
        B_ME = B_MF + RING, N_BAR = B_ME + RING };
 
 template <int D>
 struct Layout {
     static constexpr int QB = BM * D * 2;          // Q tile bytes
     static constexpr int KB = BN * D * 2;          // one K (or V) stage
-    static constexpr int PB = BM * BN * 2;         // P tile
+    static constexpr int PB = BM * BN * 2;         // one P tile (two buffers)
     static constexpr int oQ = 0;
     static constexpr int oK = oQ + QB;
     static constexpr int oV = oK + NS * KB;
     static constexpr int oP = oV + NS * KB;
-    static constexpr int oBar = oP + PB;
+    static constexpr int oBar = oP + 2 * PB;
     static constexpr int oMeta = oBar + N_BAR * 8;  // RING x 16 valid-row counts
-    static constexpr int oMisc = oMeta + RING * 16;
+    static constexpr int oRun = oMeta + RING * 16;  // 16 x (first row, slot count) of the tile being loaded
+    static constexpr int oMisc = oRun + 16 * 8;
     static constexpr int bytes = oMisc + 64;
     static constexpr int smem = bytes + 1024;      // slack for 1024-byte alignment
 };
@@ -326,8 +327,10 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
             mbar_init(bar(B_SF + s), 1);
             mbar_init(bar(B_SE + s), 128);
         }
-        mbar_init(bar(B_PF), 128);
-        mbar_init(bar(B_OD), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_PF + s), 128);
+            mbar_init(bar(B_OD + s), 1);
+        }
         mbar_init(bar(B_DR), 1);
         for (int s = 0; s < RING; ++s) {
             mbar_init(bar(B_MF + s), 1);
@@ -367,50 +370,121 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
     const int n_tiles = (int)misc[2];
 
     if (warp == 4) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (whole warp)
+        // A window of 32 selected K/V groups is held one per lane; a warp
+        // prefix sum of their 8-row slot counts places every group in the
+        // item's slot sequence.  For each 128-key tile the lanes whose group
+        // overlaps it record one run (first row, slot count) and the valid
+        // row count of each slot; runs are then issued by their own lanes as
+        // the fewest power-of-two boxes.
+        const CUtensorMap* tq = (it.a < 0) ? &maps.qp : &maps.q;
         if (lane == 0) {
-            const CUtensorMap* tq = (it.a < 0) ? &maps.qp : &maps.q;
             prefetch_tmap(tq);
+            for (int k = 0; k < NBOX; ++k) {
+                prefetch_tmap(&maps.k[k]);
+                prefetch_tmap(&maps.v[k]);
+            }
             const int qrow = (it.a < 0) ? it.bh * Mp + it.row0 : it.bh * N + it.row0;
             mbar_arrive_expect_tx(bar(B_Q), L::QB);
             for (int hh = 0; hh < D / 64; ++hh) tma_load_2d(sQ + hh * BM * 128, tq, bar(B_Q), hh * 64, qrow);
-            SlotCursor cur(it, sel_groups, sel_count, kv_off, Cq, Ck, N);
-            int issued_k = 0, issued_v = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int stage = j % NS, use = j / NS, ring = j % RING;
-                int rows[16];
-                uint32_t vw[4] = {0u, 0u, 0u, 0u};
-                for (int u = 0; u < 16; ++u) {
-                    int row, v;
-                    cur.next(row, v);
-                    rows[u] = row >= 0 ? it.bh * N + row : total_rows;
-                    vw[u >> 2] |= (uint32_t)v << (8 * (u & 3));
+        }
+        const bool probe = it.a < 0;
+        const int32_t* sg = sel_groups + ((size_t)it.bh * Cq + (probe ? 0 : it.a)) * Ck;
+        const int32_t* ko = kv_off + (size_t)it.bh * (Ck + 1);
+        const int n_groups = probe ? 1 : sel_count[(size_t)it.bh * Cq + it.a];
+        int2* runs = reinterpret_cast<int2*>(sm + L::oRun);
+        int gbase = 0, w_begin = 0, w_end = 0, my_rs = 0, my_len = 0, my_sb = 0, my_se = 0;
+        auto load_window = [&]() {
+            const int g = gbase + lane;
+            my_rs = 0;
+            my_len = 0;
+            if (g < n_groups) {
+                if (probe) {
+                    my_len = N;
+                } else {
+                    const int b = sg[g];
+                    my_rs = ko[b];
+                    my_len = ko[b + 1] - my_rs;
                 }
-                if (j >= RING && !mbar_wait(bar(B_ME + ring), ((j / RING) - 1) & 1, abort_flag, kSpin)) {
-                    record_status(status, SPARSEPR_TIMEOUT, 40);
-                    *abort_flag = 1;
-                    break;
-                }
-                *reinterpret_cast<uint4*>(meta + ring * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
-                mbar_arrive(bar(B_MF + ring));
-                if (j >= NS && !mbar_wait(bar(B_KE + stage), (use - 1) & 1, abort_flag, kSpin)) {
-                    record_status(status, SPARSEPR_TIMEOUT, 41);
-                    *abort_flag = 1;
-                    break;
-                }
-                mbar_arrive_expect_tx(bar(B_KF + stage), L::KB);
-                load_slots<D>(sK + stage * L::KB, maps.k, bar(B_KF + stage), rows, total_rows);
-                issued_k = j + 1;
-                if (j >= NS && !mbar_wait(bar(B_VE + stage), (use - 1) & 1, abort_flag, kSpin)) {
-                    record_status(status, SPARSEPR_TIMEOUT, 42);
-                    *abort_flag = 1;
-                    break;
-                }
-                mbar_arrive_expect_tx(bar(B_VF + stage), L::KB);
-                load_slots<D>(sV + stage * L::KB, maps.v, bar(B_VF + stage), rows, total_rows);
-                issued_v = j + 1;
             }
-            // every copy this CTA issued lands before the CTA can exit (abort or not)
+            const int ns = (my_len + 7) >> 3;
+            int incl = ns;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            my_sb = w_begin + incl - ns;
+            my_se = w_begin + incl;
+            w_end = w_begin + __shfl_sync(0xffffffffu, incl, 31);
+        };
+        load_window();
+        int issued_k = 0, issued_v = 0;
+        auto lane0_wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
+            int ok = 1;
+            if (lane == 0 && !mbar_wait(b, parity, abort_flag, kSpin)) {
+                record_status(status, SPARSEPR_TIMEOUT, where);
+                *abort_flag = 1;
+                ok = 0;
+            }
+            return __shfl_sync(0xffffffffu, ok, 0) != 0;
+        };
+        auto issue = [&](uint32_t dst, const CUtensorMap* mp, uint32_t b) {
+            if (lane < 16) {
+                const int2 rn = runs[lane];   // (first global row, slots) of a run starting at slot lane
+                int done = 0;
+                while (done < rn.y) {
+                    int k = 31 - __clz(rn.y - done);
+                    if (k > NBOX - 1) k = NBOX - 1;
+                    const int y = (rn.x == total_rows) ? total_rows : rn.x + 8 * done;
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        tma_load_2d(dst + hh * BN * 128 + (lane + done) * 1024, &mp[k], b, hh * 64, y);
+                    done += 1 << k;
+                }
+            }
+        };
+        for (int j = 0; j < n_tiles; ++j) {
+            const int stage = j % NS, use = j / NS, ring = j % RING;
+            const int T0 = 16 * j;
+            if (j >= RING && !lane0_wait(bar(B_ME + ring), ((j / RING) - 1) & 1, 40)) break;
+            uint8_t* vm = meta + ring * 16;
+            if (lane < 16) {
+                vm[lane] = 0;
+                runs[lane] = make_int2(0, 0);
+            }
+            __syncwarp();
+            while (true) {
+                const int lo = max(my_sb, T0), hi = min(my_se, T0 + 16);
+                if (lo < hi) {
+                    const int o = lo - my_sb;
+                    runs[lo - T0] = make_int2(it.bh * N + my_rs + 8 * o, hi - lo);
+                    for (int t = lo; t < hi; ++t) vm[t - T0] = (uint8_t)min(8, my_len - 8 * (t - my_sb));
+                }
+                if (w_end >= T0 + 16 || gbase + 32 >= n_groups) break;
+                gbase += 32;
+                w_begin = w_end;
+                load_window();
+            }
+            if (lane == 0 && w_end < T0 + 16) {   // past the last group: zero-filled padding slots
+                const int ps = max(w_end, T0);
+                runs[ps - T0] = make_int2(total_rows, T0 + 16 - ps);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_MF + ring));
+            if (j >= NS && !lane0_wait(bar(B_KE + stage), (use - 1) & 1, 41)) break;
+            if (lane == 0) mbar_arrive_expect_tx(bar(B_KF + stage), L::KB);
+            __syncwarp();
+            issue(sK + stage * L::KB, maps.k, bar(B_KF + stage));
+            issued_k = j + 1;
+            if (j >= NS && !lane0_wait(bar(B_VE + stage), (use - 1) & 1, 42)) break;
+            if (lane == 0) mbar_arrive_expect_tx(bar(B_VF + stage), L::KB);
+            __syncwarp();
+            issue(sV + stage * L::KB, maps.v, bar(B_VF + stage));
+            issued_v = j + 1;
+            __syncwarp();
+        }
+        // every copy this CTA issued lands before the CTA can exit (abort or not)
+        if (lane == 0) {
             mbar_wait(bar(B_Q), 0, nullptr, kSpin);
             for (int t = max(0, issued_k - NS); t < issued_k; ++t)
                 mbar_wait(bar(B_KF + t % NS), (t / NS) & 1, nullptr, kSpin);
@@ -425,17 +499,17 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
             constexpr uint32_t idesc_pv = idesc_f32acc(128, D, kFmtF16, true);
             bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
             auto issue_pv = [&](int t) -> bool {
-                const int stage = t % NS;
-                if (!mbar_wait(bar(B_PF), t & 1, abort_flag, kSpin)) return false;
+                const int stage = t % NS, pb = t & 1;
+                if (!mbar_wait(bar(B_PF + pb), (t >> 1) & 1, abort_flag, kSpin)) return false;
                 if (!mbar_wait(bar(B_VF + stage), (t / NS) & 1, abort_flag, kSpin)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t a = smem_desc(sP + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
+                    const uint64_t a = smem_desc(sP + pb * L::PB + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
                     const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
                     mma_f16_ss(tO, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(bar(B_OD));
+                mma_commit(bar(B_OD + pb));
                 mma_commit(bar(B_VE + stage));
                 return true;
             };
@@ -471,9 +545,9 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
         const int r = tid;   // 0..127
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        uint8_t* prow = sm + L::oP + r * 128;
         for (int j = 0; j < n_tiles; ++j) {
             const int sb = j & 1, ring = j % RING;
+            uint8_t* prow = sm + L::oP + sb * L::PB + r * 128;
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + sb), (j / 2) & 1, abort_flag, kSpin));
             if (!ok) break;
             tc_fence_after();
@@ -493,26 +567,40 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
             const uint4 vw = *reinterpret_cast<const uint4*>(meta + ring * 16);
             mbar_arrive(bar(B_ME + ring));
             const uint32_t vwa[4] = {vw.x, vw.y, vw.z, vw.w};
-            float mx = -INFINITY;
+            // mask the rows past the end of a group in partially used slots
+            // (slot counts are the same for every row: uniform branches)
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int v = (int)((vwa[u >> 2] >> (8 * (u & 3))) & 0xffu);
+                if (v < 8) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float x = (i < v) ? s[u * 8 + i] * scale_log2 : -INFINITY;
-                    s[u * 8 + i] = x;
-                    mx = fmaxf(mx, x);
+                    for (int i = 0; i < 8; ++i)
+                        if (i >= v) s[u * 8 + i] = -INFINITY;
                 }
             }
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 128; c += 4) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mx4[q] = fmaxf(mx4[q], s[c + q]);
+            }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
             const float m_new = fmaxf(m_ref, mx);
             const bool need = (j > 0) && (m_new > m_ref + 8.f);
             if (j == 0) m_ref = m_new;
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD), (j - 1) & 1, abort_flag, kSpin));
+            // P buffer sb was last read by PV(j-2); O is rescaled only once PV(j-1) is done
+            if (j >= 2) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + sb), ((j - 2) >> 1) & 1, abort_flag, kSpin));
                 if (!ok) break;
                 tc_fence_after();
             }
-            if (__any_sync(0xffffffffu, need)) {
+            const bool any_need = __any_sync(0xffffffffu, need);
+            if (any_need) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + (sb ^ 1)), ((j - 1) >> 1) & 1, abort_flag, kSpin));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            if (any_need) {
                 const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
                 if (need) {
                     m_ref = m_new;
@@ -529,28 +617,32 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 }
                 tmem_wait_st();
             }
-            // P = exp2(s - m_ref) as fp16 (<= 2^8) into the swizzled K-major P tile
+            // P = exp2(s * scale - m_ref) as fp16 (<= 2^8) into the swizzled K-major P tile
+            const float neg_m = -m_ref;
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 uint32_t w[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const __half2 pr = __floats2half2_rn(ex2_approx(s[u * 8 + 2 * i] - m_ref),
-                                                         ex2_approx(s[u * 8 + 2 * i + 1] - m_ref));
-                    const float2 back = __half22float2(pr);
-                    l += back.x + back.y;
+                    const float p0 = ex2_approx(fmaf(s[u * 8 + 2 * i], scale_log2, neg_m));
+                    const float p1 = ex2_approx(fmaf(s[u * 8 + 2 * i + 1], scale_log2, neg_m));
+                    l4[i] += p0 + p1;
+                    const __half2 pr = __floats2half2_rn(p0, p1);
                     w[i] = *reinterpret_cast<const uint32_t*>(&pr);
                 }
                 const int chunk = u >> 3, unit = u & 7;
                 uint4* dst = reinterpret_cast<uint4*>(prow + chunk * (BM * 128) + ((unit ^ (r & 7)) << 4));
                 *dst = make_uint4(w[0], w[1], w[2], w[3]);
             }
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar(B_PF));
+            mbar_arrive(bar(B_PF + sb));
         }
         if (ok && n_tiles > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD), (n_tiles - 1) & 1, abort_flag, kSpin));
+            const int t = n_tiles - 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + (t & 1)), (t >> 1) & 1, abort_flag, kSpin));
             if (ok) {
                 tc_fence_after();
                 float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + it.row0 + r) * D

@@ -107,7 +107,7 @@ struct Plan {
     // internal buffers (byte offsets into the workspace)
     size_t o_status, o_ctl, o_mat, o_FK, o_FQ, o_rq, o_phiK, o_phiQ, o_cenK, o_hnK, o_cenQ, o_hnQ,
         o_raw, o_hist, o_sorted, o_offs, o_newid, o_muK, o_t1, o_t2, o_mloc, o_pslot, o_palloc,
-        o_poff, o_psum, o_qprobe, o_work, o_fstat, o_G, o_rhs, o_vh, o_vmax, o_vscale;
+        o_poff, o_psum, o_qprobe, o_work, o_fstat, o_G, o_rhs, o_vh, o_vmax, o_vscale, o_qsplit, o_uw, o_lbar, o_vv;
     // outputs owned by the workspace for sparsepr_call
     size_t o_Qp, o_Kp, o_Vp, o_qlab, o_kvlab, o_permq, o_permk, o_posq, o_qoff, o_kvoff, o_ng, o_its,
         o_qcen, o_kcen, o_vcen, o_qdist, o_score, o_mask, o_selc, o_selg, o_pairs, o_pidx, o_pgrp,
@@ -128,6 +128,17 @@ inline long long& launch_counter() {
     return n;
 }
 inline void count_launch() { ++launch_counter(); }
+
+// Streaming multiprocessors of the current device (cached per host thread).
+inline int sm_count() {
+    static thread_local int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    }
+    return n;
+}
 
 template <typename T>
 __host__ __device__ inline T* at(void* ws, size_t off) {

@@ -12,6 +12,10 @@ sparsepr_status run_partition(const sparsepr_params& p, const Plan& pl, const vo
 sparsepr_status run_route(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
                           const sparsepr_route_out& r, void* ws, cudaStream_t st);
 bool attention_uses_tc(const sparsepr_params& p);
+bool route_uses_tc(const sparsepr_params& p);
+// Tensor-core routing-score segment sums; false if its tensor maps could not be built.
+bool launch_route_tc(const Plan& pl, const sparsepr_partition_out& part, void* ws, float* t1, float* t2, float* ml,
+                     cudaStream_t st);
 // Tensor-core k-means assignment; false if its tensor maps could not be built.
 bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, int BH, int N, int C, int R,
                              int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,

@@ -17,15 +17,16 @@
 
 namespace spr {
 namespace kmtc {
-constexpr int BP = 128;                 // points per block (TMEM lanes)
+constexpr int BP = 128;                 // points per item (TMEM lanes)
 constexpr int NBMAX = 256;              // centres per MMA block
 constexpr uint32_t kSpin = 1u << 20;
-enum { B_A = 0, B_BF = 1, B_BE = 3, B_DF = 5, B_DE = 7, B_DR = 9, N_BAR = 10 };
-constexpr int oA = 0;                                   // 2 chunks x 128 rows x 128 B
-constexpr int oB = oA + 2 * BP * 128;                   // 2 stages x 2 chunks x 256 rows x 128 B
+enum { B_AF = 0, B_AE = 2, B_BF = 4, B_BE = 6, B_DF = 8, B_DE = 10, B_DR = 12, N_BAR = 13 };
+constexpr int oA = 0;                                   // 2 buffers x 2 chunks x 128 rows x 128 B
+constexpr int oB = oA + 2 * 2 * BP * 128;               // 2 stages x 2 chunks x 256 rows x 128 B
 constexpr int oBar = oB + 2 * 2 * NBMAX * 128;
 constexpr int oRed = oBar + N_BAR * 8;                  // 128 x (score, index) of the upper half
-constexpr int oMisc = oRed + BP * 8;
+constexpr int oHn = oRed + BP * 8;                      // 2 x 256 half-norms of the centre block
+constexpr int oMisc = oHn + 2 * NBMAX * 4;
 constexpr int kSmem = oMisc + 64 + 1024;
 
 struct Maps {
@@ -34,18 +35,20 @@ struct Maps {
 };
 }  // namespace kmtc
 
+// Persistent: block k handles items k, k + grid, ... where an item is 128
+// points of one head; heads whose k-means has stopped are skipped by every role.
+template <bool DBG>
 __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
-    const __grid_constant__ kmtc::Maps maps, const float* __restrict__ hn, int N, int C, int R, int NB, int nblk,
-    int32_t* __restrict__ labels, int32_t* __restrict__ ctl, int first, float* __restrict__ dbg_scores,
+    const __grid_constant__ kmtc::Maps maps, const float* __restrict__ hn, int BH, int N, int C, int R, int NB,
+    int nblk, int32_t* __restrict__ labels, int32_t* __restrict__ ctl, int first, float* __restrict__ dbg_scores,
     int32_t* __restrict__ dbg_hist, int max_iter, DevStatus* status) {
     using namespace kmtc;
     using namespace sm100;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int bh = blockIdx.y, p0 = blockIdx.x * BP;
-    int32_t* hc = ctl + bh * kCtlStride;
-    if (hc[kCtlDone]) return;
     if (*reinterpret_cast<volatile const int32_t*>(&status->code) != 0) return;
+    const int tiles_per_head = (N + BP - 1) / BP;
+    const int n_items = BH * tiles_per_head;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_u32(sm);
     auto bar = [&](int i) -> uint32_t { return s_base + oBar + 8 * i; };
@@ -53,10 +56,12 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     const int nchunk = (R + 31) / 32;           // 32 fp32 per 128-byte row chunk
     const int ksteps = R / 8;                   // kind::tf32 K = 8 per instruction
+    auto item_live = [&](int w) -> bool { return ctl[(w / tiles_per_head) * kCtlStride + kCtlDone] == 0; };
 
     if (tid == 0) {
-        mbar_init(bar(B_A), 1);
         for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_AF + s), 1);
+            mbar_init(bar(B_AE + s), 1);
             mbar_init(bar(B_BF + s), 1);
             mbar_init(bar(B_BE + s), 1);
             mbar_init(bar(B_DF + s), 1);
@@ -79,48 +84,61 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         if (lane == 0) {   // TMA producer
             prefetch_tmap(&maps.pts);
             prefetch_tmap(&maps.cen);
-            mbar_arrive_expect_tx(bar(B_A), nchunk * BP * 128);
-            for (int ch = 0; ch < nchunk; ++ch)
-                tma_load_2d(s_base + oA + ch * BP * 128, &maps.pts, bar(B_A), ch * 32, bh * N + p0);
-            int issued = 0;
-            for (int blk = 0; blk < nblk; ++blk) {
-                const int stage = blk & 1;
-                if (blk >= 2 && !mbar_wait(bar(B_BE + stage), ((blk >> 1) - 1) & 1, abort_flag, kSpin)) {
-                    record_status(status, SPARSEPR_TIMEOUT, 20);
-                    *abort_flag = 1;
-                    break;
-                }
-                mbar_arrive_expect_tx(bar(B_BF + stage), nchunk * NB * 128);
+            int li = 0, gb = 0;           // local item count, global centre-block count
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+                if (!item_live(w)) continue;
+                const int bh = w / tiles_per_head, p0 = (w % tiles_per_head) * BP, ab = li & 1;
+                if (li >= 2 && !mbar_wait(bar(B_AE + ab), ((li >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                mbar_arrive_expect_tx(bar(B_AF + ab), nchunk * BP * 128);
                 for (int ch = 0; ch < nchunk; ++ch)
-                    tma_load_2d(s_base + oB + (stage * 2 + ch) * NBMAX * 128, &maps.cen, bar(B_BF + stage), ch * 32,
-                                bh * C + blk * NB);
-                issued = blk + 1;
+                    tma_load_2d(s_base + oA + (ab * 2 + ch) * BP * 128, &maps.pts, bar(B_AF + ab), ch * 32, bh * N + p0);
+                for (int blk = 0; blk < nblk; ++blk, ++gb) {
+                    const int stage = gb & 1;
+                    if (gb >= 2 && !mbar_wait(bar(B_BE + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar(B_BF + stage), nchunk * NB * 128);
+                    for (int ch = 0; ch < nchunk; ++ch)
+                        tma_load_2d(s_base + oB + (stage * 2 + ch) * NBMAX * 128, &maps.cen, bar(B_BF + stage),
+                                    ch * 32, bh * C + blk * NB);
+                }
+                ++li;
             }
-            mbar_wait(bar(B_A), 0, nullptr, kSpin);
-            for (int t = max(0, issued - 2); t < issued; ++t)
-                mbar_wait(bar(B_BF + (t & 1)), (t >> 1) & 1, nullptr, kSpin);
+            if (!ok) {
+                record_status(status, SPARSEPR_TIMEOUT, 20);
+                *abort_flag = 1;
+            }
+            for (int t = max(0, li - 2); t < li; ++t) mbar_wait(bar(B_AF + (t & 1)), (t >> 1) & 1, nullptr, kSpin);
+            for (int t = max(0, gb - 2); t < gb; ++t) mbar_wait(bar(B_BF + (t & 1)), (t >> 1) & 1, nullptr, kSpin);
         }
     } else if (warp == 9) {
         if (lane == 0) {   // MMA issuer
             const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NB >> 3) << 17) |
                                    ((uint32_t)(BP >> 4) << 24);   // F32 <- TF32 x TF32, K-major both
-            bool ok = mbar_wait(bar(B_A), 0, abort_flag, kSpin);
-            for (int blk = 0; ok && blk < nblk; ++blk) {
-                const int stage = blk & 1;
-                if (!mbar_wait(bar(B_BF + stage), (blk >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
-                if (blk >= 2 && !mbar_wait(bar(B_DE + stage), ((blk >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
-                tc_fence_after();
-                for (int kk = 0; kk < ksteps; ++kk) {
-                    const uint64_t a = smem_desc(s_base + oA + (kk / 4) * BP * 128 + (kk % 4) * 32, 16, 1024);
-                    const uint64_t b = smem_desc(s_base + oB + (stage * 2 + kk / 4) * NBMAX * 128 + (kk % 4) * 32, 16, 1024);
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem + stage * NB),
-                        "l"(a), "l"(b), "r"(idesc), "r"(kk > 0 ? 1u : 0u)
-                        : "memory");
+            int li = 0, gb = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+                if (!item_live(w)) continue;
+                const int ab = li & 1;
+                if (!mbar_wait(bar(B_AF + ab), (li >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                for (int blk = 0; blk < nblk; ++blk, ++gb) {
+                    const int stage = gb & 1;
+                    if (!mbar_wait(bar(B_BF + stage), (gb >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    if (gb >= 2 && !mbar_wait(bar(B_DE + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kk = 0; kk < ksteps; ++kk) {
+                        const uint64_t a = smem_desc(s_base + oA + (ab * 2 + kk / 4) * BP * 128 + (kk % 4) * 32, 16, 1024);
+                        const uint64_t b = smem_desc(s_base + oB + (stage * 2 + kk / 4) * NBMAX * 128 + (kk % 4) * 32, 16, 1024);
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem + stage * NB),
+                            "l"(a), "l"(b), "r"(idesc), "r"(kk > 0 ? 1u : 0u)
+                            : "memory");
+                    }
+                    mma_commit(bar(B_DF + stage));
+                    mma_commit(bar(B_BE + stage));
                 }
-                mma_commit(bar(B_DF + stage));
-                mma_commit(bar(B_BE + stage));
+                mma_commit(bar(B_AE + ab));
+                ++li;
             }
             if (!ok) {
                 record_status(status, SPARSEPR_TIMEOUT, 21);
@@ -132,63 +150,78 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
     } else {
         // epilogue: warps 0-3 take the lower half of each centre block, 4-7 the upper half
         const int half = warp >> 2, row = (warp & 3) * 32 + lane;
-        const int p = p0 + row;
-        const bool valid = p < N;
         const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const int hw = NB / 2;
-        float best = -INFINITY;
-        int bi = 0x7fffffff;
+        float* red_s = reinterpret_cast<float*>(sm + oRed);
+        int* red_i = reinterpret_cast<int*>(sm + oRed + BP * 4);
+        float* hns = reinterpret_cast<float*>(sm + oHn);
+        int gb = 0;
         bool ok = true;
-        for (int blk = 0; blk < nblk; ++blk) {
-            const int db = blk & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + db), (blk >> 1) & 1, abort_flag, kSpin));
-            if (!ok) break;
-            tc_fence_after();
-            for (int c0 = 0; c0 < hw; c0 += 32) {
-                float v[32];
-                tmem_ld32(t_row + db * NB + half * hw + c0, v);
-                tmem_wait_ld();
-                const int cb = blk * NB + half * hw + c0;
+        for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+            if (!item_live(w)) continue;
+            const int bh = w / tiles_per_head, p = (w % tiles_per_head) * BP + row;
+            const bool valid = p < N;
+            int32_t* hc = ctl + bh * kCtlStride;
+            float best = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int blk = 0; blk < nblk; ++blk, ++gb) {
+                const int db = gb & 1;
+                // half-norms of this centre block (columns past C never win)
+                float* hb = hns + db * NBMAX;
+                for (int c = tid; c < NB; c += 256) {
+                    const int cg = blk * NB + c;
+                    hb[c] = (cg < C) ? hn[(size_t)bh * C + cg] : INFINITY;
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + db), (gb >> 1) & 1, abort_flag, kSpin));
+                if (!ok) break;
+                tc_fence_after();
+                for (int c0 = 0; c0 < hw; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(t_row + db * NB + half * hw + c0, v);
+                    tmem_wait_ld();
+                    const int cb = blk * NB + half * hw + c0;
+                    const float* hr = hb + half * hw + c0;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c = cb + i;
-                    if (c < C) {
-                        const float sc = v[i] - __ldg(hn + (size_t)bh * C + c);
-                        if (dbg_scores != nullptr && valid) dbg_scores[((size_t)bh * N + p) * C + c] = sc;
+                    for (int i = 0; i < 32; ++i) {
+                        const float sc = v[i] - hr[i];
+                        if (DBG) {
+                            if (valid && cb + i < C) dbg_scores[((size_t)bh * N + p) * C + cb + i] = sc;
+                        }
                         if (sc > best) {
                             best = sc;
-                            bi = c;
+                            bi = cb + i;
                         }
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(bar(B_DE + db));
             }
-            tc_fence_before();
-            mbar_arrive(bar(B_DE + db));
-        }
-        float* red_s = reinterpret_cast<float*>(sm + oRed);
-        int* red_i = reinterpret_cast<int*>(sm + oRed + BP * 4);
-        if (half == 1) {
-            red_s[row] = best;
-            red_i[row] = bi;
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (half == 0) {
-            const float b1 = red_s[row];
-            const int i1 = red_i[row];
-            if (b1 > best || (b1 == best && i1 < bi)) {
-                best = b1;
-                bi = i1;
+            if (!ok) break;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (half == 1) {
+                red_s[row] = best;
+                red_i[row] = bi;
             }
-            if (bi == 0x7fffffff) bi = 0;
-            int changed = 0;
-            if (valid && ok) {
-                int32_t* lp = labels + (size_t)bh * N + p;
-                changed = (!first) && (*lp != bi);
-                *lp = bi;
-                if (dbg_hist != nullptr) dbg_hist[((size_t)bh * max_iter + hc[kCtlIters]) * N + p] = bi;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (half == 0) {
+                const float b1 = red_s[row];
+                const int i1 = red_i[row];
+                if (b1 > best || (b1 == best && i1 < bi)) {
+                    best = b1;
+                    bi = i1;
+                }
+                if (bi == 0x7fffffff) bi = 0;
+                int changed = 0;
+                if (valid) {
+                    int32_t* lp = labels + (size_t)bh * N + p;
+                    changed = (!first) && (*lp != bi);
+                    *lp = bi;
+                    if (dbg_hist != nullptr) dbg_hist[((size_t)bh * max_iter + hc[kCtlIters]) * N + p] = bi;
+                }
+                const unsigned ballot = __ballot_sync(0xffffffffu, changed);
+                if (lane == 0 && ballot) atomicAdd(&hc[kCtlChanged], __popc(ballot));
             }
-            const unsigned ballot = __ballot_sync(0xffffffffu, changed);
-            if (lane == 0 && ballot) atomicAdd(&hc[kCtlChanged], __popc(ballot));
         }
         if (!ok) {
             record_status(status, SPARSEPR_TIMEOUT, 22);
@@ -246,9 +279,17 @@ bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn
     kmtc::Maps maps;
     if (!make_f32_map(&maps.pts, phi, (uint64_t)BH * N, R, kmtc::BP)) return false;
     if (!make_f32_map(&maps.cen, cen, (uint64_t)BH * C, R, NB)) return false;
-    cudaFuncSetAttribute(kmeans_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
-    count_launch(), kmeans_assign_tc_kernel<<<dim3((N + kmtc::BP - 1) / kmtc::BP, BH), 320, kmtc::kSmem, st>>>(
-        maps, hn, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
+    const int items = BH * ((N + kmtc::BP - 1) / kmtc::BP);
+    const int grid = items < sm_count() ? items : sm_count();
+    if (dbg_scores != nullptr) {
+        cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
+        count_launch(), kmeans_assign_tc_kernel<true><<<grid, 320, kmtc::kSmem, st>>>(
+            maps, hn, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
+    } else {
+        cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
+        count_launch(), kmeans_assign_tc_kernel<false><<<grid, 320, kmtc::kSmem, st>>>(
+            maps, hn, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
+    }
     return true;
 }
 

@@ -101,7 +101,8 @@ __global__ void __launch_bounds__(256) centred_gram_kernel(const float* __restri
 // F[:, c] = u_c sqrt(max(lambda_c, 0)) * scale for the r leading eigenpairs
 // (descending, ties to the lower index) and zero columns up to Rp.
 // For the query factor (ng != nullptr) r = max(1, min(r_req, d, C_k' - 1)).
-__global__ void __launch_bounds__(512) jacobi_factor_kernel(const float* __restrict__ Ain, int d,
+template <int d>
+__global__ void __launch_bounds__(512) jacobi_factor_kernel(const float* __restrict__ Ain,
                                                             float* __restrict__ F, int Rp,
                                                             int r_req, const int32_t* ng,
                                                             float scale, int32_t* r_out,
@@ -126,8 +127,10 @@ __global__ void __launch_bounds__(512) jacobi_factor_kernel(const float* __restr
     }
     __syncthreads();
 
+    float off_prev = INFINITY;
     for (int sweep = 0; sweep < max_sweeps; ++sweep) {
-        // convergence: off-diagonal energy vs total energy
+        // convergence: off-diagonal energy vs total energy; stop once it is at
+        // fp32 rounding level or a sweep no longer halves it
         float off = 0.f, tot = 0.f;
         for (int e = tid; e < d * d; e += nt) {
             const int i = e / d, j = e % d;
@@ -152,7 +155,9 @@ __global__ void __launch_bounds__(512) jacobi_factor_kernel(const float* __restr
             red[32] = t;
         }
         __syncthreads();
-        const bool converged = !(red[0] > 1e-13f * red[32]);
+        const float off_now = red[0];
+        const bool converged = !(off_now > 1e-11f * red[32]) || (sweep >= 3 && off_now > 0.5f * off_prev);
+        off_prev = off_now;
         __syncthreads();
         if (converged) break;
 
@@ -722,13 +727,13 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
 
     const size_t jac_smem = (size_t)(2 * d * (d + 1) + 2 * (d / 2) + 64) * sizeof(float) +
                             (size_t)(2 * (d / 2) + d) * sizeof(int);
-    cudaFuncSetAttribute(jacobi_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)jac_smem);
+    auto jacobi = (d == 128) ? jacobi_factor_kernel<128> : jacobi_factor_kernel<64>;
+    cudaFuncSetAttribute(jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jac_smem);
 
     // 1-2. key-response metric and factor (§4.1)
     count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff, mat);
-    count_launch(), jacobi_factor_kernel<<<BH, 512, jac_smem, st>>>(mat, d, FK, pl.RKp, pl.rK_eff, nullptr,
-                                                    1.f / sqrtf((float)d), nullptr, 20);
+    count_launch(), jacobi<<<BH, 512, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d),
+                                                      nullptr, 16);
     project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, st);
     // 3. paired K/V groups
     kmeans_dispatch(pl.RKp, pl, p, ws, phiK, pl.Ck, 0, cenK, hnK, dbg ? out.debug_kv_scores : nullptr,
@@ -745,7 +750,7 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), centroid_mean_kernel<<<BH, d, 0, st>>>(out.k_centroid, out.n_groups, pl.Ck, d, muK);
     count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
                                                                           out.n_groups, pl.Ck, d, mat);
-    count_launch(), jacobi_factor_kernel<<<BH, 512, jac_smem, st>>>(mat, d, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 20);
+    count_launch(), jacobi<<<BH, 512, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16);
     project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, st);
     // 5. query groups
     kmeans_dispatch(pl.RQp, pl, p, ws, phiQ, pl.Cq, 1, cenQ, hnQ, dbg ? out.debug_q_scores : nullptr,

@@ -106,9 +106,55 @@ __global__ void __launch_bounds__(256) route_partial_kernel(
     }
 }
 
+// lbar[a][b] = qbar_a kbar_b^T / sqrt(d) for every pair of nonempty groups (32x32 tiles).
+__global__ void __launch_bounds__(256) centroid_logits_kernel(const float* __restrict__ qbar,
+                                                              const float* __restrict__ kbar,
+                                                              const int32_t* __restrict__ ng, int Cq, int Ck, int d,
+                                                              float* __restrict__ lbar) {
+    const int bh = blockIdx.z, a0 = blockIdx.y * 32, b0 = blockIdx.x * 32;
+    const int Cqp = ng[bh * 2 + 0], Ckp = ng[bh * 2 + 1];
+    if (a0 >= Cqp || b0 >= Ckp) return;
+    const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
+    __shared__ float sa[32][33], sb[32][33];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int t0 = 0; t0 < d; t0 += 32) {
+        for (int r = ty; r < 32; r += 8) {
+            sa[r][tx] = (a0 + r < Cqp) ? qbar[((size_t)bh * Cq + a0 + r) * d + t0 + tx] : 0.f;
+            sb[r][tx] = (b0 + r < Ckp) ? kbar[((size_t)bh * Ck + b0 + r) * d + t0 + tx] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int t = 0; t < 32; ++t) {
+            const float bv = sb[tx][t];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u] = fmaf(sa[ty + 8 * u][t], bv, acc[u]);
+        }
+        __syncthreads();
+    }
+    const float inv = 1.f / sqrtf((float)d);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int a = a0 + ty + 8 * u, b = b0 + tx;
+        if (a < Cqp && b < Ckp) lbar[((size_t)bh * Cq + a) * Ck + b] = acc[u] * inv;
+    }
+}
+
+// |vbar_b|^2, one warp per K/V group.
+__global__ void centroid_sqnorm_kernel(const float* __restrict__ vbar, const int32_t* __restrict__ ng, int Ck, int d,
+                                       float* __restrict__ vv) {
+    const int bh = blockIdx.y, lane = threadIdx.x & 31;
+    const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (b >= ng[bh * 2 + 1]) return;
+    const float* v = vbar + ((size_t)bh * Ck + b) * d;
+    float acc = 0.f;
+    for (int t = lane; t < d; t += 32) acc = fmaf(v[t], v[t], acc);
+    acc = warp_sum(acc);
+    if (lane == 0) vv[(size_t)bh * Ck + b] = acc;
+}
+
 // Scores, ranking and the prefix rule for one query group per block.
 __global__ void __launch_bounds__(1024) route_select_kernel(
-    const float* __restrict__ qbar, const float* __restrict__ kbar, const float* __restrict__ vbar,
+    const float* __restrict__ lbar_in, const float* __restrict__ vv_in,
     const float* __restrict__ t1o, const float* __restrict__ t2o, const float* __restrict__ mloc,
     const int32_t* __restrict__ q_off, const int32_t* __restrict__ kv_off,
     const int32_t* __restrict__ ng, int Cq, int Ck, int d, long long beta,
@@ -117,24 +163,18 @@ __global__ void __launch_bounds__(1024) route_select_kernel(
     __shared__ unsigned long long keys[kMaxGroups];
     __shared__ float lb[kMaxGroups];
     __shared__ int sz[kMaxGroups];
-    __shared__ float qv[128];
     __shared__ float red[32];
     __shared__ int scratch[33];
     __shared__ int cut;
     const int a = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int Cqp = ng[bh * 2 + 0], Ckp = ng[bh * 2 + 1];
     if (a >= Cqp) return;
-    for (int t = tid; t < d; t += blockDim.x) qv[t] = qbar[((size_t)bh * Cq + a) * d + t];
     if (tid == 0) cut = Ckp - 1;
     __syncthreads();
-    const float inv_sqrt_d = 1.f / sqrtf((float)d);
     const size_t row = ((size_t)bh * Cq + a) * Ck;
     float mx = -INFINITY;
     for (int b = tid; b < Ckp; b += blockDim.x) {
-        const float* kb = kbar + ((size_t)bh * Ck + b) * d;
-        float l = 0.f;
-        for (int t = 0; t < d; ++t) l = fmaf(qv[t], kb[t], l);
-        l *= inv_sqrt_d;
+        const float l = lbar_in[row + b];
         lb[b] = l;
         mx = fmaxf(mx, fmaxf(l, mloc[row + b]));
     }
@@ -150,9 +190,7 @@ __global__ void __launch_bounds__(1024) route_select_kernel(
     const float m_a = red[0];
     const int32_t* ko = kv_off + (size_t)bh * (Ck + 1);
     for (int b = tid; b < Ckp; b += blockDim.x) {
-        const float* vb = vbar + ((size_t)bh * Ck + b) * d;
-        float vv = 0.f;
-        for (int t = 0; t < d; ++t) vv = fmaf(vb[t], vb[t], vv);
+        const float vv = vv_in[(size_t)bh * Ck + b];
         const int nb = ko[b + 1] - ko[b];
         const float inv_nb = 1.f / (float)nb;
         const float ea = expf(lb[b] - m_a);
@@ -347,10 +385,19 @@ sparsepr_status run_route(const sparsepr_params& p, const Plan& pl, const sparse
     const int BH = pl.BH;
     cudaMemsetAsync(r.pairs, 0, (size_t)BH * 2 * sizeof(int64_t), st);
     cudaMemsetAsync(r.sel_count, 0, (size_t)BH * pl.Cq * sizeof(int32_t), st);
-    if (p.dtype == SPARSEPR_BF16) route_partial<__nv_bfloat16>(pl, part, t1, t2, ml, st);
-    else route_partial<float>(pl, part, t1, t2, ml, st);
+    if (route_uses_tc(p)) {
+        if (!launch_route_tc(pl, part, ws, t1, t2, ml, st)) return SPARSEPR_CUDA_ERROR;
+    } else {
+        route_partial<float>(pl, part, t1, t2, ml, st);
+    }
+    float* lbar = at<float>(ws, pl.o_lbar);
+    float* vv = at<float>(ws, pl.o_vv);
+    count_launch(), centroid_logits_kernel<<<dim3((pl.Ck + 31) / 32, (pl.Cq + 31) / 32, BH), dim3(32, 8), 0, st>>>(
+        part.q_centroid, part.k_centroid, part.n_groups, pl.Cq, pl.Ck, pl.d, lbar);
+    count_launch(), centroid_sqnorm_kernel<<<dim3((pl.Ck + 7) / 8, BH), 256, 0, st>>>(part.v_centroid, part.n_groups,
+                                                                                      pl.Ck, pl.d, vv);
     count_launch(), route_select_kernel<<<dim3(pl.Cq, BH), 1024, 0, st>>>(
-        part.q_centroid, part.k_centroid, part.v_centroid, t1, t2, ml, part.q_offsets,
+        lbar, vv, t1, t2, ml, part.q_offsets,
         part.kv_offsets, part.n_groups, pl.Cq, pl.Ck, pl.d, (long long)pl.beta, r.score, r.mask,
         r.sel_count, r.sel_groups, reinterpret_cast<unsigned long long*>(r.pairs));
     count_launch(), probe_alloc_kernel<<<BH, 1024, 0, st>>>(part.q_offsets, part.n_groups, pl.Cq, pl.N, pl.Mp, alloc, poff, psum,
