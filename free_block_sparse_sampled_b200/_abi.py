@@ -16,7 +16,7 @@ FLAG_SIMT_ATTENTION = 2
 
 EXPORTED = ["sparsepr_status_string", "sparsepr_validate", "sparsepr_workspace_size",
             "sparsepr_partition", "sparsepr_route", "sparsepr_attention", "sparsepr_probe_fit",
-            "sparsepr_apply", "sparsepr_call", "sparsepr_get_device_status"]
+            "sparsepr_apply", "sparsepr_call", "sparsepr_last_error_string", "sparsepr_get_device_status"]
 
 P = ctypes.c_void_p
 
@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         L.sparsepr_call.restype = ctypes.c_int32
         L.sparsepr_call.argtypes = [ctypes.POINTER(Params), P, P, P, P, ctypes.POINTER(Stats), P,
                                     ctypes.c_size_t, P]
+        L.sparsepr_last_error_string.restype = ctypes.c_char_p
+        L.sparsepr_last_error_string.argtypes = []
         L.sparsepr_get_device_status.restype = ctypes.c_int32
         L.sparsepr_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         _LIB = L
@@ -107,7 +109,10 @@ def lib() -> ctypes.CDLL:
 
 class SparsePRError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        msg = f"{fn} failed: {STATUS_NAMES.get(status, status)}"
+        if status == 4 and _LIB is not None:
+            msg += f" ({_LIB.sparsepr_last_error_string().decode()})"
+        super().__init__(msg)
         self.status = status
 
 

@@ -326,7 +326,7 @@ sparsepr_status sparsepr_call(const sparsepr_params* p, const void* Q, const voi
     if ((s = run_apply(q, pl, part, route, O_sp, pdense, fit, O_out, ws, st)) != SPARSEPR_OK) return s;
     if (stats) {
         cudaEventRecord(ev[5], st);
-        if (cudaEventSynchronize(ev[5]) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
+        if (cuda_status(cudaEventSynchronize(ev[5])) != SPARSEPR_OK) return SPARSEPR_CUDA_ERROR;
         float ms[5];
         for (int i = 0; i < 5; ++i) cudaEventElapsedTime(&ms[i], ev[i], ev[i + 1]);
         stats->ms_partition = ms[0];
@@ -353,16 +353,19 @@ sparsepr_status sparsepr_call(const sparsepr_params* p, const void* Q, const voi
         stats->rho_exec = (double)exec_sum / ((double)pl.BH * (double)pl.N * (double)pl.N);
         stats->launches = launch_counter() - launches0;
     }
-    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+    return cuda_status(cudaGetLastError());
 }
+
+const char* sparsepr_last_error_string(void) { return last_error_buffer(); }
 
 sparsepr_status sparsepr_get_device_status(void* ws, void* stream, int32_t* out) {
     if (ws == nullptr || out == nullptr) return SPARSEPR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     int32_t v = 0;
-    if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
-    if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
+    sparsepr_status s = cuda_status(cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, st));
+    if (s == SPARSEPR_OK) s = cuda_status(cudaStreamSynchronize(st));
+    if (s == SPARSEPR_OK) s = cuda_status(cudaMemsetAsync(ws, 0, 256, st));
+    if (s != SPARSEPR_OK) return s;
     *out = v;
     return SPARSEPR_OK;
 }

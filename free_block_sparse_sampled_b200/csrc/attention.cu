@@ -27,8 +27,11 @@
 namespace spr {
 
 // ---------------------------------------------------------------- work items
+// Items never cross a query group.  pair == 0: one tile of BM rows per item
+// (w = rows).  pair == 1: two consecutive 128-row tiles per item
+// (w = rows of tile 0 | rows of tile 1 << 16).
 __global__ void __launch_bounds__(1024) build_work_kernel(const int32_t* __restrict__ q_off,
-                                                          const int32_t* __restrict__ ng, int Cq, int BM,
+                                                          const int32_t* __restrict__ ng, int Cq, int BM, int pair,
                                                           int4* __restrict__ items,
                                                           int32_t* __restrict__ counter) {
     __shared__ int cnt[kMaxGroups];
@@ -37,16 +40,20 @@ __global__ void __launch_bounds__(1024) build_work_kernel(const int32_t* __restr
     const int bh = blockIdx.x;
     const int Cqp = ng[bh * 2 + 0];
     const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
-    for (int a = threadIdx.x; a < Cqp; a += blockDim.x) cnt[a] = (qo[a + 1] - qo[a] + BM - 1) / BM;
+    const int span = pair ? 2 * BM : BM;
+    for (int a = threadIdx.x; a < Cqp; a += blockDim.x) cnt[a] = (qo[a + 1] - qo[a] + span - 1) / span;
     __syncthreads();
     const int total = block_exclusive_scan(cnt, Cqp, scratch);
     if (threadIdx.x == 0) base = atomicAdd(counter, total);
     __syncthreads();
     for (int a = threadIdx.x; a < Cqp; a += blockDim.x) {
         const int s = qo[a], size = qo[a + 1] - qo[a];
-        const int n = (size + BM - 1) / BM;
-        for (int t = 0; t < n; ++t)
-            items[base + cnt[a] + t] = make_int4(bh, a, s + t * BM, min(BM, size - t * BM));
+        const int n = (size + span - 1) / span;
+        for (int t = 0; t < n; ++t) {
+            const int rest = size - t * span;
+            const int w = pair ? (min(BM, rest) | (max(0, min(BM, rest - BM)) << 16)) : min(BM, rest);
+            items[base + cnt[a] + t] = make_int4(bh, a, s + t * span, w);
+        }
     }
 }
 
@@ -228,28 +235,41 @@ __global__ void __launch_bounds__(256) attention_simt_kernel(
 }
 
 // ---------------------------------------------------------------- tcgen05 kernel
+// One block handles up to two 128-row query tiles of the same query group
+// (or two tiles of probe rows) against the same key sequence.
+//   warps 0-3 / 4-7: online softmax of Q tile 0 / 1 (one TMEM lane per row)
+//   warp 8: TMA producer (whole warp), warp 9: MMA issuer
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).  P_t
+// (fp16, two per column) overwrites the first 64 columns of S_t and feeds
+// O_t += P_t V as a TMEM-operand MMA.  The MMA thread issues PV_t(j-1)
+// before S_t(j), so the commit that publishes S_t(j) also certifies that O_t
+// is quiescent for the softmax's lazy rescale.
 namespace tc {
 constexpr int BM = 128, BN = 128, NS = 2, RING = 4, NBOX = 5;   // boxes of 8 << k rows, k < NBOX
 constexpr uint32_t kSpin = 1u << 20;   // polls of mbarrier.try_wait before giving up
+#ifndef SPR_SOFT_EVERY
+#define SPR_SOFT_EVERY 0
+#endif
+constexpr int kSoftEvery = SPR_SOFT_EVERY;   // every n-th exponential pair on the FMA pipe (0: none)
 enum { B_Q = 0, B_KF = 1, B_KE = B_KF + NS, B_VF = B_KE + NS, B_VE = B_VF + NS, B_SF = B_VE + NS,
-       B_SE = B_SF + 2, B_PF = B_SE + 2, B_OD = B_PF + 2, B_DR = B_OD + 2, B_MF = B_DR + 1,
-       B_ME = B_MF + RING, N_BAR = B_ME + RING };
+       B_PF = B_SF + 2, B_OF = B_PF + 2, B_DR = B_OF + 1, B_MF = B_DR + 1, B_ME = B_MF + RING,
+       N_BAR = B_ME + RING };
 
 template <int D>
 struct Layout {
-    static constexpr int QB = BM * D * 2;          // Q tile bytes
+    static constexpr int QB = BM * D * 2;          // one Q tile
     static constexpr int KB = BN * D * 2;          // one K (or V) stage
-    static constexpr int PB = BM * BN * 2;         // one P tile (two buffers)
-    static constexpr int oQ = 0;
-    static constexpr int oK = oQ + QB;
+    static constexpr int oQ = 0;                   // two Q tiles
+    static constexpr int oK = oQ + 2 * QB;
     static constexpr int oV = oK + NS * KB;
-    static constexpr int oP = oV + NS * KB;
-    static constexpr int oBar = oP + 2 * PB;
-    static constexpr int oMeta = oBar + N_BAR * 8;  // RING x 16 valid-row counts
+    static constexpr int oBar = oV + NS * KB;
+    static constexpr int oMeta = (oBar + N_BAR * 8 + 15) / 16 * 16;   // RING x 16 valid-row counts (read as uint4)
     static constexpr int oRun = oMeta + RING * 16;  // 16 x (first row, slot count) of the tile being loaded
     static constexpr int oMisc = oRun + 16 * 8;
     static constexpr int bytes = oMisc + 64;
     static constexpr int smem = bytes + 1024;      // slack for 1024-byte alignment
+    static_assert(oK % 1024 == 0 && oV % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+    static_assert(oMeta % 16 == 0 && oRun % 8 == 0, "vector accesses need aligned offsets");
 };
 
 // Tensor maps: K (bf16) and V (fp16) rows in boxes of 8, 16, 32, 64, 128 rows x
@@ -260,37 +280,36 @@ struct Maps {
     CUtensorMap q;
     CUtensorMap qp;
 };
-
-// Loads the 16 slots of one 128-row stage: runs of slots with consecutive
-// rows go out as the fewest power-of-two boxes; padding slots read rows past
-// the end of the tensor, which TMA fills with zeros.
-template <int D>
-__device__ __forceinline__ void load_slots(uint32_t dst, const CUtensorMap* maps, uint32_t bar, const int (&rows)[16],
-                                           int oob) {
-    int u = 0;
-    while (u < 16) {
-        int L = 1;
-        if (rows[u] != oob) {
-            while (u + L < 16 && rows[u + L] == rows[u] + 8 * L) ++L;
-        } else {
-            while (u + L < 16 && rows[u + L] == oob) ++L;
-        }
-        int s = u, rem = L;
-        while (rem > 0) {
-            int k = 31 - __clz(rem);
-            if (k > NBOX - 1) k = NBOX - 1;
-            for (int hh = 0; hh < D / 64; ++hh)
-                sm100::tma_load_2d(dst + hh * BN * 128 + s * 1024, &maps[k], bar, hh * 64, rows[s]);
-            s += 1 << k;
-            rem -= 1 << k;
-        }
-        u += L;
-    }
-}
 }  // namespace tc
 
+struct Item2 {
+    int bh, a, row0, n0, n1;
+};
+
+__device__ __forceinline__ bool decode_item2(int item, const int4* items, const int32_t* counter, int n_probe_items,
+                                             int Mp, Item2& it) {
+    if (item < n_probe_items) {
+        const int per = (Mp + 255) / 256;
+        it.bh = item / per;
+        it.a = -1;
+        it.row0 = (item % per) * 256;
+        it.n0 = min(128, Mp - it.row0);
+        it.n1 = max(0, min(128, Mp - it.row0 - 128));
+        return true;
+    }
+    const int k = item - n_probe_items;
+    if (k >= *counter) return false;
+    const int4 w = items[k];
+    it.bh = w.x;
+    it.a = w.y;
+    it.row0 = w.z;
+    it.n0 = w.w & 0xffff;
+    it.n1 = w.w >> 16;
+    return true;
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1) attention_tc_kernel(
+__global__ void __launch_bounds__(320, 1) attention_tc_kernel(
     const __grid_constant__ tc::Maps maps, const int4* __restrict__ items, const int32_t* __restrict__ counter,
     int n_probe_items, int N, int Mp, int Cq, int Ck, int total_rows, const int32_t* __restrict__ kv_off,
     const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_groups, const float* __restrict__ vscale,
@@ -302,14 +321,15 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-    Item it;
-    if (!decode_item(blockIdx.x, items, counter, n_probe_items, BM, Mp, it)) return;
+    Item2 it;
+    if (!decode_item2(blockIdx.x, items, counter, n_probe_items, Mp, it)) return;
     // once any block has given up, the rest of the launch returns at once
     if (*reinterpret_cast<volatile const int32_t*>(&status->code) != 0) return;
+    const int nq = it.n1 > 0 ? 2 : 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_u32(sm);
-    const uint32_t sQ = s_base + L::oQ, sK = s_base + L::oK, sV = s_base + L::oV, sP = s_base + L::oP;
+    const uint32_t sQ = s_base + L::oQ, sK = s_base + L::oK, sV = s_base + L::oV;
     auto bar = [&](int i) -> uint32_t { return s_base + L::oBar + 8 * i; };
     uint8_t* meta = sm + L::oMeta;
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::oMisc);   // [0] tmem, [1] abort, [2] n_tiles
@@ -325,16 +345,13 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(B_SF + s), 1);
-            mbar_init(bar(B_SE + s), 128);
-        }
-        for (int s = 0; s < 2; ++s) {
             mbar_init(bar(B_PF + s), 128);
-            mbar_init(bar(B_OD + s), 1);
         }
+        mbar_init(bar(B_OF), 1);
         mbar_init(bar(B_DR), 1);
         for (int s = 0; s < RING; ++s) {
             mbar_init(bar(B_MF + s), 1);
-            mbar_init(bar(B_ME + s), 128);
+            mbar_init(bar(B_ME + s), 128 * nq);
         }
         fence_barrier_init();
         misc[1] = 0;
@@ -356,10 +373,10 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
         for (int o = 16; o > 0; o >>= 1) slots += __shfl_xor_sync(0xffffffffu, slots, o);
         if (lane == 0) {
             misc[2] = (uint32_t)((slots + 15) / 16);
-            atomicAdd(visited, (unsigned long long)((slots + 15) / 16) * (unsigned long long)(BM * BN));
+            atomicAdd(visited, (unsigned long long)((slots + 15) / 16) * (unsigned long long)(BM * BN * nq));
         }
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(smem_u32(misc), 512);
         tmem_relinquish();
     }
@@ -369,7 +386,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
     const uint32_t tmem = misc[0];
     const int n_tiles = (int)misc[2];
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------ TMA producer (whole warp)
         // A window of 32 selected K/V groups is held one per lane; a warp
         // prefix sum of their 8-row slot counts places every group in the
@@ -385,8 +402,10 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 prefetch_tmap(&maps.v[k]);
             }
             const int qrow = (it.a < 0) ? it.bh * Mp + it.row0 : it.bh * N + it.row0;
-            mbar_arrive_expect_tx(bar(B_Q), L::QB);
-            for (int hh = 0; hh < D / 64; ++hh) tma_load_2d(sQ + hh * BM * 128, tq, bar(B_Q), hh * 64, qrow);
+            mbar_arrive_expect_tx(bar(B_Q), nq * L::QB);
+            for (int t = 0; t < nq; ++t)
+                for (int hh = 0; hh < D / 64; ++hh)
+                    tma_load_2d(sQ + t * L::QB + hh * BM * 128, tq, bar(B_Q), hh * 64, qrow + t * BM);
         }
         const bool probe = it.a < 0;
         const int32_t* sg = sel_groups + ((size_t)it.bh * Cq + (probe ? 0 : it.a)) * Ck;
@@ -491,45 +510,57 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
             for (int t = max(0, issued_v - NS); t < issued_v; ++t)
                 mbar_wait(bar(B_VF + t % NS), (t / NS) & 1, nullptr, kSpin);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
             constexpr uint32_t idesc_qk = idesc_f32acc(128, 128, kFmtBF16, false);
             constexpr uint32_t idesc_pv = idesc_f32acc(128, D, kFmtF16, true);
-            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
-            auto issue_pv = [&](int t) -> bool {
-                const int stage = t % NS, pb = t & 1;
-                if (!mbar_wait(bar(B_PF + pb), (t >> 1) & 1, abort_flag, kSpin)) return false;
-                if (!mbar_wait(bar(B_VF + stage), (t / NS) & 1, abort_flag, kSpin)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t a = smem_desc(sP + pb * L::PB + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
-                    const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
-                    mma_f16_ss(tO, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(B_OD + pb));
-                mma_commit(bar(B_VE + stage));
-                return true;
-            };
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int stage = j % NS, sb = j & 1;
-                if (!mbar_wait(bar(B_KF + stage), (j / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
-                if (j >= 2 && !mbar_wait(bar(B_SE + sb), ((j - 2) / 2) & 1, abort_flag, kSpin)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t tS = sb ? tS1 : tS0;
-#pragma unroll
+            auto issue_s = [&](int t, int stage) {
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t a = smem_desc(sQ + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
+                    const uint64_t a = smem_desc(sQ + t * L::QB + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
                     const uint64_t b = smem_desc(sK + stage * L::KB + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
-                    mma_f16_ss(tS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_f16_ss(tmem + 128 * t, a, b, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar(B_SF + sb));
+            };
+            auto issue_pv = [&](int t, int jj) {
+                const int stage = jj % NS;
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
+                    mma_f16_ts(tmem + 256 + D * t, tmem + 128 * t + kk * 8, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int stage = j % NS;
+                if (!mbar_wait(bar(B_KF + stage), (j / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
+                if (j >= 1 && !mbar_wait(bar(B_VF + (j - 1) % NS), ((j - 1) / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
+                for (int t = 0; t < nq; ++t) {
+                    if (j >= 1) {
+                        if (!mbar_wait(bar(B_PF + t), (j - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(t, j - 1);
+                    }
+                    tc_fence_after();
+                    issue_s(t, stage);
+                    mma_commit(bar(B_SF + t));
+                }
+                if (!ok) break;
                 mma_commit(bar(B_KE + stage));
-                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+                if (j >= 1) mma_commit(bar(B_VE + (j - 1) % NS));
             }
-            if (ok && n_tiles > 0) ok = issue_pv(n_tiles - 1);
+            if (ok && n_tiles > 0) {
+                const int jl = n_tiles - 1;
+                if (!mbar_wait(bar(B_VF + jl % NS), (jl / NS) & 1, abort_flag, kSpin)) ok = false;
+                for (int t = 0; ok && t < nq; ++t) {
+                    if (!mbar_wait(bar(B_PF + t), jl & 1, abort_flag, kSpin)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(t, jl);
+                }
+                if (ok) {
+                    mma_commit(bar(B_VE + jl % NS));
+                    mma_commit(bar(B_OF));
+                }
+            }
             if (!ok) {
                 record_status(status, SPARSEPR_TIMEOUT, 43);
                 *abort_flag = 1;
@@ -538,69 +569,56 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
             mma_commit(bar(B_DR));
             mbar_wait(bar(B_DR), 0, nullptr, kSpin);
         }
-    } else {
-        // ------------------------------------------------ softmax warpgroup (rows = TMEM lanes)
-        const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-        const uint32_t tO = t_row + 256;
-        const int r = tid;   // 0..127
+    } else if (warp < 4 * nq) {
+        // ------------------------------------------------ softmax of Q tile t (rows = TMEM lanes)
+        const int t = warp >> 2, r = tid - 128 * t;
+        const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t tS = t_row + 128 * t, tO = t_row + 256 + D * t;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
+        auto mask_chunk = [&](float (&v)[32], const uint32_t (&vwa)[4], int c4) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int u = c4 * 4 + q;
+                const int cnt = (int)((vwa[u >> 2] >> (8 * (u & 3))) & 0xffu);
+                if (cnt < 8) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if (i >= cnt) v[q * 8 + i] = -INFINITY;
+                }
+            }
+        };
         for (int j = 0; j < n_tiles; ++j) {
-            const int sb = j & 1, ring = j % RING;
-            uint8_t* prow = sm + L::oP + sb * L::PB + r * 128;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + sb), (j / 2) & 1, abort_flag, kSpin));
+            const int ring = j % RING;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + t), j & 1, abort_flag, kSpin));
             if (!ok) break;
             tc_fence_after();
-            float s[128];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                float v[32];
-                tmem_ld32(t_row + sb * 128 + c4 * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) s[c4 * 32 + i] = v[i];
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(B_SE + sb));
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_MF + ring), (j / RING) & 1, abort_flag, kSpin));
             if (!ok) break;
             const uint4 vw = *reinterpret_cast<const uint4*>(meta + ring * 16);
             mbar_arrive(bar(B_ME + ring));
             const uint32_t vwa[4] = {vw.x, vw.y, vw.z, vw.w};
-            // mask the rows past the end of a group in partially used slots
-            // (slot counts are the same for every row: uniform branches)
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int v = (int)((vwa[u >> 2] >> (8 * (u & 3))) & 0xffu);
-                if (v < 8) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if (i >= v) s[u * 8 + i] = -INFINITY;
-                }
-            }
+            // row maximum over the 128 keys, read as two 64-column halves
+            // (ten warps share four register-file partitions: keep the live set small)
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 128; c += 4) {
+            for (int hf = 0; hf < 2; ++hf) {
+                float sv[2][32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) mx4[q] = fmaxf(mx4[q], s[c + q]);
+                for (int q = 0; q < 2; ++q) tmem_ld32(tS + (2 * hf + q) * 32, sv[q]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    mask_chunk(sv[q], vwa, 2 * hf + q);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], sv[q][i]);
+                }
             }
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
             const float m_new = fmaxf(m_ref, mx);
             const bool need = (j > 0) && (m_new > m_ref + 8.f);
             if (j == 0) m_ref = m_new;
-            // P buffer sb was last read by PV(j-2); O is rescaled only once PV(j-1) is done
-            if (j >= 2) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + sb), ((j - 2) >> 1) & 1, abort_flag, kSpin));
-                if (!ok) break;
-                tc_fence_after();
-            }
-            const bool any_need = __any_sync(0xffffffffu, need);
-            if (any_need) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + (sb ^ 1)), ((j - 1) >> 1) & 1, abort_flag, kSpin));
-                if (!ok) break;
-                tc_fence_after();
-            }
-            if (any_need) {
+            if (__any_sync(0xffffffffu, need)) {   // O_t is quiescent: PV_t(j-1) completed before S_t(j)
                 const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
                 if (need) {
                     m_ref = m_new;
@@ -617,43 +635,55 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
                 }
                 tmem_wait_st();
             }
-            // P = exp2(s * scale - m_ref) as fp16 (<= 2^8) into the swizzled K-major P tile
+            // P = exp2(s * scale - m_ref) as fp16 (<= 2^8), two per column over S's first 64
+            // columns; one pair in four takes the FMA-pipe exponential to offload the MUFU.
+            // P half hf lands in columns [32 hf, 32 hf + 32), already read in both halves.
             const float neg_m = -m_ref;
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                uint32_t w[4];
+            for (int hf = 0; hf < 2; ++hf) {
+                float sv[2][32];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float p0 = ex2_approx(fmaf(s[u * 8 + 2 * i], scale_log2, neg_m));
-                    const float p1 = ex2_approx(fmaf(s[u * 8 + 2 * i + 1], scale_log2, neg_m));
-                    l4[i] += p0 + p1;
-                    const __half2 pr = __floats2half2_rn(p0, p1);
-                    w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+                for (int q = 0; q < 2; ++q) tmem_ld32(tS + (2 * hf + q) * 32, sv[q]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    mask_chunk(sv[q], vwa, 2 * hf + q);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float x0 = fmaf(sv[q][2 * i], scale_log2, neg_m);
+                        const float x1 = fmaf(sv[q][2 * i + 1], scale_log2, neg_m);
+                        const bool soft = kSoftEvery > 0 && (i % kSoftEvery) == kSoftEvery - 1;
+                        const float p0 = soft ? exp2_poly(x0) : ex2_approx(x0);
+                        const float p1 = soft ? exp2_poly(x1) : ex2_approx(x1);
+                        l4[i & 3] += p0 + p1;
+                        const __half2 pr = __floats2half2_rn(p0, p1);
+                        w[i] = *reinterpret_cast<const uint32_t*>(&pr);
+                    }
+                    tmem_st16(tS + (2 * hf + q) * 16, w);
                 }
-                const int chunk = u >> 3, unit = u & 7;
-                uint4* dst = reinterpret_cast<uint4*>(prow + chunk * (BM * 128) + ((unit ^ (r & 7)) << 4));
-                *dst = make_uint4(w[0], w[1], w[2], w[3]);
             }
             l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_PF + sb));
+            mbar_arrive(bar(B_PF + t));
         }
         if (ok && n_tiles > 0) {
-            const int t = n_tiles - 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OD + (t & 1)), (t >> 1) & 1, abort_flag, kSpin));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF), 0, abort_flag, kSpin));
             if (ok) {
                 tc_fence_after();
-                float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + it.row0 + r) * D
-                                        : O_sp + ((size_t)it.bh * N + it.row0 + r) * D;
+                const int nrows = t == 0 ? it.n0 : it.n1;
+                const int row = it.row0 + BM * t + r;
+                float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + row) * D
+                                        : O_sp + ((size_t)it.bh * N + row) * D;
                 const float inv = vscale[it.bh] / l;
 #pragma unroll
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     float v[32];
                     tmem_ld32(tO + c4 * 32, v);
                     tmem_wait_ld();
-                    if (r < it.nrows) {
+                    if (r < nrows) {
                         float4* o4 = reinterpret_cast<float4*>(out + c4 * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
@@ -670,7 +700,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(
         tc_fence_before();
     }
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -713,7 +743,7 @@ __global__ void vconvert_kernel(const __nv_bfloat16* __restrict__ V, size_t per_
          e += (size_t)gridDim.x * blockDim.x * 8) {
         float x[8];
         load8(v + e, x);
-        __half2 o[4];
+        __align__(16) __half2 o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) o[i] = __floats2half2_rn(x[2 * i] * s, x[2 * i + 1] * s);
         *reinterpret_cast<uint4*>(h + e) = *reinterpret_cast<const uint4*>(o);
@@ -774,7 +804,9 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
     DevStatus* status = at<DevStatus>(ws, pl.o_status);
     unsigned long long* visited = at<unsigned long long>(ws, pl.o_work + 8);
     cudaMemsetAsync(counter, 0, 16, st);
-    count_launch(), build_work_kernel<<<BH, 1024, 0, st>>>(part.q_offsets, part.n_groups, pl.Cq, pl.BM, items, counter);
+    const bool tcore = attention_uses_tc(p);
+    count_launch(), build_work_kernel<<<BH, 1024, 0, st>>>(part.q_offsets, part.n_groups, pl.Cq, pl.BM, tcore ? 1 : 0,
+                                                           items, counter);
     if (Mp > 0) {
         const int chunks = d * pl.esz / 16;
         if (p.dtype == SPARSEPR_BF16)
@@ -788,7 +820,9 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
     }
     const int grid = pl.n_probe_items + pl.n_items_max;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)d);
-    if (attention_uses_tc(p)) {
+    if (tcore) {
+        const int n_probe2 = Mp > 0 ? BH * ((Mp + 255) / 256) : 0;
+        const int grid2 = n_probe2 + pl.n_items_max;
         __half* VH = at<__half>(ws, pl.o_vh);
         unsigned* vmax = at<unsigned>(ws, pl.o_vmax);
         float* vscale = at<float>(ws, pl.o_vscale);
@@ -812,14 +846,14 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
         if (d == 128) {
             auto k = attention_tc_kernel<128>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<128>::smem);
-            count_launch(), k<<<grid, 192, tc::Layout<128>::smem, st>>>(maps, items, counter, pl.n_probe_items, N, Mp,
+            count_launch(), k<<<grid2, 320, tc::Layout<128>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
                                                                        pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
                                                                        r.sel_count, r.sel_groups, vscale, O_sp,
                                                                        probe_dense, status, visited, scale_log2);
         } else {
             auto k = attention_tc_kernel<64>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<64>::smem);
-            count_launch(), k<<<grid, 192, tc::Layout<64>::smem, st>>>(maps, items, counter, pl.n_probe_items, N, Mp,
+            count_launch(), k<<<grid2, 320, tc::Layout<64>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
                                                                       pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
                                                                       r.sel_count, r.sel_groups, vscale, O_sp,
                                                                       probe_dense, status, visited, scale_log2);
@@ -843,7 +877,7 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
         count_launch(), gather_probe_rows_kernel<float><<<grid_for((size_t)BH * Mp * chunks, 256), 256, 0, st>>>(
             O_sp, r.probe_idx, part.pos_q, BH, N, Mp, d, probe_sparse);
     }
-    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+    return cuda_status(cudaGetLastError());
 }
 
 }  // namespace spr

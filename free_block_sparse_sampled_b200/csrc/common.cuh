@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 
 #include "sparsepr.h"
 
@@ -121,6 +122,19 @@ constexpr int kCtlChanged = 0, kCtlDone = 1, kCtlIters = 2, kCtlItersK = 3, kCtl
               kCtlWork = 8;
 
 bool make_plan(const sparsepr_params& p, Plan& pl);
+
+// Last CUDA error seen by this host thread (name and message), for
+// sparsepr_last_error_string().
+inline char* last_error_buffer() {
+    static thread_local char buf[256] = "no error";
+    return buf;
+}
+// Records err (if any) and maps it to a status.
+inline sparsepr_status cuda_status(cudaError_t err) {
+    if (err == cudaSuccess) return SPARSEPR_OK;
+    snprintf(last_error_buffer(), 256, "%s: %s", cudaGetErrorName(err), cudaGetErrorString(err));
+    return SPARSEPR_CUDA_ERROR;
+}
 
 // Kernels launched by this host thread since the counter was last reset.
 inline long long& launch_counter() {

@@ -261,7 +261,7 @@ sparsepr_status run_fit(const sparsepr_params& p, const Plan& pl, const sparsepr
         cudaMemsetAsync(f.mu_x, 0, (size_t)BH * d * 4, st);
         cudaMemsetAsync(f.mu_r, 0, (size_t)BH * d * 4, st);
         count_launch(), fill_kernel<<<(BH * d + 255) / 256, 256, 0, st>>>(f.sigma, BH * d, 1.f);
-        return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+        return cuda_status(cudaGetLastError());
     }
     count_launch(), fit_stats_kernel<<<BH, d, 0, st>>>(probe_sparse, probe_dense, r.probe_group, alloc, part.q_offsets,
                                        part.n_groups, psum, pl.Cq, Mp, d, p.eps_std, fstat, f.mu_x, f.sigma,
@@ -271,7 +271,7 @@ sparsepr_status run_fit(const sparsepr_params& p, const Plan& pl, const sparsepr
     const size_t smem = (size_t)d * (d + 1) * sizeof(double);
     cudaFuncSetAttribute(fit_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     count_launch(), fit_solve_kernel<<<BH, d, smem, st>>>(G, rhs, d, f.B, status);
-    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+    return cuda_status(cudaGetLastError());
 }
 
 sparsepr_status run_apply(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
@@ -295,7 +295,7 @@ sparsepr_status run_apply(const sparsepr_params& p, const Plan& pl, const sparse
         count_launch(), apply_kernel<64><<<grid, 256, smem, st>>>(O_sp, f.B, f.mu_x, f.sigma, f.mu_r, pslot, probe_dense,
                                                  part.perm_q, pl.N, pl.Mp, O_out);
     }
-    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+    return cuda_status(cudaGetLastError());
 }
 
 }  // namespace spr

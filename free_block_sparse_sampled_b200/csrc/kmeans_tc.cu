@@ -162,8 +162,9 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
             const int bh = w / tiles_per_head, p = (w % tiles_per_head) * BP + row;
             const bool valid = p < N;
             int32_t* hc = ctl + bh * kCtlStride;
-            float best = -INFINITY;
-            int bi = 0x7fffffff;
+            // four independent argmax chains (columns c = 4k + q), merged lowest index first
+            float best4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            int bi4[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
             for (int blk = 0; blk < nblk; ++blk, ++gb) {
                 const int db = gb & 1;
                 // half-norms of this centre block (columns past C never win)
@@ -188,15 +189,23 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                         if (DBG) {
                             if (valid && cb + i < C) dbg_scores[((size_t)bh * N + p) * C + cb + i] = sc;
                         }
-                        if (sc > best) {
-                            best = sc;
-                            bi = cb + i;
+                        if (sc > best4[i & 3]) {
+                            best4[i & 3] = sc;
+                            bi4[i & 3] = cb + i;
                         }
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(bar(B_DE + db));
             }
+            float best = best4[0];
+            int bi = bi4[0];
+#pragma unroll
+            for (int q = 1; q < 4; ++q)
+                if (best4[q] > best || (best4[q] == best && bi4[q] < bi)) {
+                    best = best4[q];
+                    bi = bi4[q];
+                }
             if (!ok) break;
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (half == 1) {

@@ -478,19 +478,36 @@ __global__ void centre_update_kernel(const float* __restrict__ phi, const int32_
     const int s = offs[(size_t)bh * (C + 1) + c], e = offs[(size_t)bh * (C + 1) + c + 1];
     if (e == s) return;
     constexpr int PL = (R + 31) / 32;
-    float acc[PL];
+    constexpr int U = 8;   // member rows in flight per lane; partial sums combined in a fixed order
+    float acc[U][PL];
 #pragma unroll
-    for (int u = 0; u < PL; ++u) acc[u] = 0.f;
+    for (int k = 0; k < U; ++k)
+#pragma unroll
+        for (int u = 0; u < PL; ++u) acc[k][u] = 0.f;
     const float* ph = phi + (size_t)bh * N * R;
     const int32_t* so = sorted + (size_t)bh * N;
-    for (int p = s; p < e; ++p) {
-        const float* row = ph + (size_t)so[p] * R;
+    for (int p0 = s; p0 < e; p0 += 32) {
+        const int my = (p0 + lane < e) ? so[p0 + lane] : -1;   // 32 member indices per load
+        const int n = min(32, e - p0);
+        for (int q0 = 0; q0 < n; q0 += U) {
 #pragma unroll
-        for (int u = 0; u < PL; ++u) {
-            const int t = lane + 32 * u;
-            if (t < R) acc[u] += row[t];
+            for (int k = 0; k < U; ++k) {
+                const int row = __shfl_sync(0xffffffffu, my, (q0 + k) & 31);
+                if (q0 + k < n) {
+                    const float* rp = ph + (size_t)row * R;
+#pragma unroll
+                    for (int u = 0; u < PL; ++u) {
+                        const int t = lane + 32 * u;
+                        if (t < R) acc[k][u] += rp[t];
+                    }
+                }
+            }
         }
     }
+#pragma unroll
+    for (int u = 0; u < PL; ++u)
+        acc[0][u] = ((acc[0][u] + acc[1][u]) + (acc[2][u] + acc[3][u])) +
+                    ((acc[4][u] + acc[5][u]) + (acc[6][u] + acc[7][u]));
     const float count = (float)(e - s);
     float ss = 0.f;
     float* dst = cen + ((size_t)bh * C + c) * R;
@@ -498,7 +515,7 @@ __global__ void centre_update_kernel(const float* __restrict__ phi, const int32_
     for (int u = 0; u < PL; ++u) {
         const int t = lane + 32 * u;
         if (t < R) {
-            const float m = tf32_round(acc[u] / count);
+            const float m = tf32_round(acc[0][u] / count);
             dst[t] = m;
             ss = fmaf(m, m, ss);
         }
@@ -771,7 +788,7 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     if (out.F_Q) cudaMemcpyAsync(out.F_Q, FQ, (size_t)BH * d * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
     if (out.phi_K) cudaMemcpyAsync(out.phi_K, phiK, (size_t)BH * N * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
     if (out.phi_Q) cudaMemcpyAsync(out.phi_Q, phiQ, (size_t)BH * N * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
-    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+    return cuda_status(cudaGetLastError());
 }
 
 }  // namespace

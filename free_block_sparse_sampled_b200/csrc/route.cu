@@ -406,7 +406,7 @@ sparsepr_status run_route(const sparsepr_params& p, const Plan& pl, const sparse
         count_launch(), probe_select_kernel<<<dim3(pl.Cq, BH), 256, 0, st>>>(
             part.q_offsets, part.perm_q, part.q_dist, part.n_groups, alloc, poff, psum,
             pl.Cq, pl.N, pl.Mp, r.probe_idx, r.probe_group, r.probe_weight);
-    return cudaGetLastError() == cudaSuccess ? SPARSEPR_OK : SPARSEPR_CUDA_ERROR;
+    return cuda_status(cudaGetLastError());
 }
 
 }  // namespace spr

@@ -115,6 +115,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
         : "memory");
 }
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -144,6 +153,20 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t ab_fo
            | ((uint32_t)(M >> 4) << 24);
 }
 
+// 2^x on the FMA pipe, for x <= 127: Cody-Waite range reduction x = n + f with
+// n = floor(x) (exact for base 2), then 2^f on [0,1) from a cubic fitted here by
+// least squares on Chebyshev nodes (relative error below 7.5e-5, under the
+// fp16 rounding of the attention weights), and 2^n added to the exponent bits.
+// Results below 2^-126 flush to zero.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -127.f);
+    const float n = floorf(x);
+    const float f = x - n;
+    const float p = fmaf(fmaf(fmaf(0.07802443f, f, 0.22606729f), f, 0.69583350f), f, 0.99992520f);
+    const int ni = __float2int_rn(n);
+    return ni < -126 ? 0.f : __int_as_float(__float_as_int(p) + ni * (1 << 23));
+}
+
 // Hardware base-2 exponential (MUFU); exp2(-inf) = +0.
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
@@ -158,6 +181,16 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]  (A: M rows in TMEM lanes, 16-bit K packed two per column)
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 

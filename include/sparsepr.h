@@ -209,6 +209,10 @@ sparsepr_status sparsepr_call(const sparsepr_params* p, const void* Q, const voi
                               const void* V, float* O_out, sparsepr_stats* stats,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Name and message of the last CUDA error any entry point met on this host
+ * thread ("no error" if none); valid until the next failing call. */
+const char* sparsepr_last_error_string(void);
+
 /* Reads (synchronously on `stream`) and clears the device status word of
  * `workspace`: *out = SPARSEPR_OK or the first device-side failure. */
 sparsepr_status sparsepr_get_device_status(void* workspace, void* stream, int32_t* out);
