@@ -16,7 +16,11 @@ FLAG_SIMT_ATTENTION = 2
 
 EXPORTED = ["sparsepr_status_string", "sparsepr_validate", "sparsepr_workspace_size",
             "sparsepr_partition", "sparsepr_route", "sparsepr_attention", "sparsepr_probe_fit",
-            "sparsepr_apply", "sparsepr_call", "sparsepr_last_error_string", "sparsepr_get_device_status"]
+            "sparsepr_apply", "sparsepr_call", "sparsepr_last_error_string", "sparsepr_get_device_status",
+            "sparsepr_probe_fit_static"]
+
+# size of the static scratch array behind sparsepr_probe_fit_static
+FIT_STATIC_SCRATCH_BYTES = 8 << 20
 
 P = ctypes.c_void_p
 
@@ -103,6 +107,9 @@ def lib() -> ctypes.CDLL:
         L.sparsepr_last_error_string.argtypes = []
         L.sparsepr_get_device_status.restype = ctypes.c_int32
         L.sparsepr_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+        L.sparsepr_probe_fit_static.restype = ctypes.c_int32
+        L.sparsepr_probe_fit_static.argtypes = [ctypes.POINTER(Params), ctypes.POINTER(PartitionOut),
+                                                ctypes.POINTER(RouteOut), P, P, ctypes.POINTER(FitOut), P, P]
         _LIB = L
     return _LIB
 

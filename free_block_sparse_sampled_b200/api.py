@@ -202,6 +202,22 @@ def probe_fit(cfg: SparsePRConfig, part, rt, probe_sparse, probe_dense, ws: torc
     return f
 
 
+def probe_fit_static(cfg: SparsePRConfig, part, rt, probe_sparse, probe_dense, fit: Dict[str, torch.Tensor],
+                     device_status: Optional[torch.Tensor] = None) -> Dict[str, torch.Tensor]:
+    """sparsepr_probe_fit_static: the probe fit with no workspace, for callers
+    that cannot allocate device memory where they fit.  ``fit`` holds the
+    caller's preallocated outputs (B, mu_x, sigma, mu_r); ``device_status`` an
+    optional device int32 that receives the fit's status."""
+    s = A.FitOut(*[_p(fit[n]) for n in A.FIT_FIELDS])
+    p = cfg.c_params()
+    A.check("sparsepr_probe_fit_static", A.lib().sparsepr_probe_fit_static(
+        ctypes.byref(p), ctypes.byref(part["_struct"]), ctypes.byref(rt["_struct"]), _p(probe_sparse),
+        _p(probe_dense), ctypes.byref(s), _p(device_status), _stream()))
+    out = dict(fit)
+    out["_struct"] = s
+    return out
+
+
 def apply(cfg: SparsePRConfig, part, rt, O_sp, probe_dense, fit, ws: torch.Tensor) -> torch.Tensor:
     out = torch.empty(cfg.B, cfg.H, cfg.N, cfg.d, dtype=torch.float32, device=ws.device)
     p = cfg.c_params()

@@ -194,6 +194,41 @@ sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const sparsepr_part
                                    const float* probe_dense, const sparsepr_fit_out* fit,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size in bytes of the static scratch array behind sparsepr_probe_fit_static
+ * (8 MiB).  A call needs
+ *   256 + r(4 BH) + r(24 BH d) + 2 r(8 BH d^2) bytes,  r(x) = x rounded up to 256,
+ * which allows up to 31 heads (B*H) at d = 128 and 125 heads at d = 64. */
+#define SPARSEPR_FIT_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* sparsepr_probe_fit without a workspace.  The paper has no counterpart: it
+ * exists for callers that hold the partition and routing results but cannot
+ * allocate device memory where they run the fit -- a host framework whose
+ * caching allocator has taken all free HBM, or a loop that must not take the
+ * device-wide synchronisation of cudaMalloc/cudaFree.
+ *
+ * Same kernels, arguments and outputs as sparsepr_probe_fit, except that the
+ * fit's scratch (fp64 weighted statistics, Gram matrices and right-hand
+ * sides) lives in one static device array of SPARSEPR_FIT_STATIC_SCRATCH_BYTES
+ * that every GPU loading the library holds until the process exits.  The
+ * function allocates nothing and calls no allocating routine.
+ *   device_status: optional caller-owned DEVICE int32 that receives
+ *                  SPARSEPR_OK, or SPARSEPR_NUMERIC after a non-positive
+ *                  Cholesky pivot (B is then 0), in stream order.
+ * Errors: a call whose scratch exceeds the array returns SPARSEPR_UNSUPPORTED
+ * before anything is launched; sparsepr_last_error_string() then gives the
+ * bytes needed and the limit.  Other checks as sparsepr_probe_fit.
+ * The first call on a device looks up the array's device address (which can
+ * load the module); make that first call before any stream capture.
+ * Every call on a device shares the array and finds the previous call's
+ * contents there; each call clears the status word it needs zeroed, and the
+ * rest is fully rewritten before it is read.  Calls whose work overlaps on
+ * the GPU (different streams, or host threads without ordering) race on the
+ * array and give undefined results. */
+sparsepr_status sparsepr_probe_fit_static(const sparsepr_params* p, const sparsepr_partition_out* part,
+                                          const sparsepr_route_out* route, const float* probe_sparse,
+                                          const float* probe_dense, const sparsepr_fit_out* fit,
+                                          int32_t* device_status, void* stream);
+
 /* §4.2: O_out[b,h,i] = O^dense for probe rows, O^sp + mu_R + ((O^sp - mu_X)/sigma) B
  * otherwise, written in ORIGINAL query order.  O_out: [BH,N,d] fp32. */
 sparsepr_status sparsepr_apply(const sparsepr_params* p, const sparsepr_partition_out* part,
