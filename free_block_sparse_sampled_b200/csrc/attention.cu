@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(256) attention_simt_kernel(
 // One block handles up to two 128-row query tiles of the same query group
 // (or two tiles of probe rows) against the same key sequence.
 //   warps 0-3 / 4-7: online softmax of Q tile 0 / 1 (one TMEM lane per row)
-//   warp 8: TMA producer (whole warp), warp 9: MMA issuer
+//   warp 8: TMA producer (whole warp), warp 9: MMA issuer, warps 10-11 idle
 // TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).  P_t
 // (fp16, two per column) overwrites the first 64 columns of S_t and feeds
 // O_t += P_t V as a TMEM-operand MMA.  The MMA thread issues PV_t(j-1)
@@ -246,11 +246,19 @@ __global__ void __launch_bounds__(256) attention_simt_kernel(
 // is quiescent for the softmax's lazy rescale.
 namespace tc {
 constexpr int BM = 128, BN = 128, NS = 2, RING = 4, NBOX = 5;   // boxes of 8 << k rows, k < NBOX
+constexpr int kThreads = 384;   // 3 warpgroups: softmax tile 0, softmax tile 1, producer + MMA
+constexpr int kLaunchRegs = 168, kRegsSoftmax = 224, kRegsOther = 56;
+// what the softmax warpgroups take, the third gives back: per block and per
+// SM sub-partition (which holds one warp of each warpgroup)
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kLaunchRegs, "register split");
+static_assert(2 * kRegsSoftmax + kRegsOther == 3 * kLaunchRegs, "register split per sub-partition");
 constexpr uint32_t kSpin = 1u << 20;   // polls of mbarrier.try_wait before giving up
-#ifndef SPR_SOFT_EVERY
-#define SPR_SOFT_EVERY 0
+#ifndef SPR_SOFT_PAIRS
+#define SPR_SOFT_PAIRS 2
 #endif
-constexpr int kSoftEvery = SPR_SOFT_EVERY;   // every n-th exponential pair on the FMA pipe (0: none)
+// exponential pairs, of every 16, computed on the FMA pipe instead of the MUFU
+constexpr int kSoftPairs = SPR_SOFT_PAIRS;
+static_assert(kSoftPairs >= 0 && kSoftPairs <= 16, "soft pairs per 16");
 enum { B_Q = 0, B_KF = 1, B_KE = B_KF + NS, B_VF = B_KE + NS, B_VE = B_VF + NS, B_SF = B_VE + NS,
        B_PF = B_SF + 2, B_OF = B_PF + 2, B_DR = B_OF + 1, B_MF = B_DR + 1, B_ME = B_MF + RING,
        N_BAR = B_ME + RING };
@@ -309,7 +317,7 @@ __device__ __forceinline__ bool decode_item2(int item, const int4* items, const 
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) attention_tc_kernel(
+__global__ void __launch_bounds__(384, 1) attention_tc_kernel(
     const __grid_constant__ tc::Maps maps, const int4* __restrict__ items, const int32_t* __restrict__ counter,
     int n_probe_items, int N, int Mp, int Cq, int Ck, int total_rows, const int32_t* __restrict__ kv_off,
     const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_groups, const float* __restrict__ vscale,
@@ -386,318 +394,324 @@ __global__ void __launch_bounds__(320, 1) attention_tc_kernel(
     const uint32_t tmem = misc[0];
     const int n_tiles = (int)misc[2];
 
-    if (warp == 8) {
-        // ------------------------------------------------ TMA producer (whole warp)
-        // A window of 32 selected K/V groups is held one per lane; a warp
-        // prefix sum of their 8-row slot counts places every group in the
-        // item's slot sequence.  For each 128-key tile the lanes whose group
-        // overlaps it record one run (first row, slot count) and the valid
-        // row count of each slot; runs are then issued by their own lanes as
-        // the fewest power-of-two boxes.
-        const CUtensorMap* tq = (it.a < 0) ? &maps.qp : &maps.q;
-        if (lane == 0) {
-            prefetch_tmap(tq);
-            for (int k = 0; k < NBOX; ++k) {
-                prefetch_tmap(&maps.k[k]);
-                prefetch_tmap(&maps.v[k]);
-            }
-            const int qrow = (it.a < 0) ? it.bh * Mp + it.row0 : it.bh * N + it.row0;
-            mbar_arrive_expect_tx(bar(B_Q), nq * L::QB);
-            for (int t = 0; t < nq; ++t)
-                for (int hh = 0; hh < D / 64; ++hh)
-                    tma_load_2d(sQ + t * L::QB + hh * BM * 128, tq, bar(B_Q), hh * 64, qrow + t * BM);
-        }
-        const bool probe = it.a < 0;
-        const int32_t* sg = sel_groups + ((size_t)it.bh * Cq + (probe ? 0 : it.a)) * Ck;
-        const int32_t* ko = kv_off + (size_t)it.bh * (Ck + 1);
-        const int n_groups = probe ? 1 : sel_count[(size_t)it.bh * Cq + it.a];
-        int2* runs = reinterpret_cast<int2*>(sm + L::oRun);
-        int gbase = 0, w_begin = 0, w_end = 0, my_rs = 0, my_len = 0, my_sb = 0, my_se = 0;
-        auto load_window = [&]() {
-            const int g = gbase + lane;
-            my_rs = 0;
-            my_len = 0;
-            if (g < n_groups) {
-                if (probe) {
-                    my_len = N;
-                } else {
-                    const int b = sg[g];
-                    my_rs = ko[b];
-                    my_len = ko[b + 1] - my_rs;
+    // Register split (the host launches only when the kernel was built with
+    // kLaunchRegs registers per thread): warpgroup 2 (producer, MMA, two idle
+    // warps) drops to kRegsOther, the two softmax warpgroups rise to
+    // kRegsSoftmax, which keeps the S row of 128 fp32 values in registers.
+    if (warp >= 8) {
+        setmaxnreg_dec<kRegsOther>();
+        if (warp == 8) {
+            // ------------------------------------------------ TMA producer (whole warp)
+            // A window of 32 selected K/V groups is held one per lane; a warp
+            // prefix sum of their 8-row slot counts places every group in the
+            // item's slot sequence.  For each 128-key tile the lanes whose group
+            // overlaps it record one run (first row, slot count) and the valid
+            // row count of each slot; runs are then issued by their own lanes as
+            // the fewest power-of-two boxes.
+            const CUtensorMap* tq = (it.a < 0) ? &maps.qp : &maps.q;
+            if (lane == 0) {
+                prefetch_tmap(tq);
+                for (int k = 0; k < NBOX; ++k) {
+                    prefetch_tmap(&maps.k[k]);
+                    prefetch_tmap(&maps.v[k]);
                 }
-            }
-            const int ns = (my_len + 7) >> 3;
-            int incl = ns;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            my_sb = w_begin + incl - ns;
-            my_se = w_begin + incl;
-            w_end = w_begin + __shfl_sync(0xffffffffu, incl, 31);
-        };
-        load_window();
-        int issued_k = 0, issued_v = 0;
-        auto lane0_wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
-            int ok = 1;
-            if (lane == 0 && !mbar_wait(b, parity, abort_flag, kSpin)) {
-                record_status(status, SPARSEPR_TIMEOUT, where);
-                *abort_flag = 1;
-                ok = 0;
-            }
-            return __shfl_sync(0xffffffffu, ok, 0) != 0;
-        };
-        auto issue = [&](uint32_t dst, const CUtensorMap* mp, uint32_t b) {
-            if (lane < 16) {
-                const int2 rn = runs[lane];   // (first global row, slots) of a run starting at slot lane
-                int done = 0;
-                while (done < rn.y) {
-                    int k = 31 - __clz(rn.y - done);
-                    if (k > NBOX - 1) k = NBOX - 1;
-                    const int y = (rn.x == total_rows) ? total_rows : rn.x + 8 * done;
+                const int qrow = (it.a < 0) ? it.bh * Mp + it.row0 : it.bh * N + it.row0;
+                mbar_arrive_expect_tx(bar(B_Q), nq * L::QB);
+                for (int t = 0; t < nq; ++t)
                     for (int hh = 0; hh < D / 64; ++hh)
-                        tma_load_2d(dst + hh * BN * 128 + (lane + done) * 1024, &mp[k], b, hh * 64, y);
-                    done += 1 << k;
-                }
+                        tma_load_2d(sQ + t * L::QB + hh * BM * 128, tq, bar(B_Q), hh * 64, qrow + t * BM);
             }
-        };
-        for (int j = 0; j < n_tiles; ++j) {
-            const int stage = j % NS, use = j / NS, ring = j % RING;
-            const int T0 = 16 * j;
-            if (j >= RING && !lane0_wait(bar(B_ME + ring), ((j / RING) - 1) & 1, 40)) break;
-            uint8_t* vm = meta + ring * 16;
-            if (lane < 16) {
-                vm[lane] = 0;
-                runs[lane] = make_int2(0, 0);
-            }
-            __syncwarp();
-            while (true) {
-                const int lo = max(my_sb, T0), hi = min(my_se, T0 + 16);
-                if (lo < hi) {
-                    const int o = lo - my_sb;
-                    runs[lo - T0] = make_int2(it.bh * N + my_rs + 8 * o, hi - lo);
-                    for (int t = lo; t < hi; ++t) vm[t - T0] = (uint8_t)min(8, my_len - 8 * (t - my_sb));
-                }
-                if (w_end >= T0 + 16 || gbase + 32 >= n_groups) break;
-                gbase += 32;
-                w_begin = w_end;
-                load_window();
-            }
-            if (lane == 0 && w_end < T0 + 16) {   // past the last group: zero-filled padding slots
-                const int ps = max(w_end, T0);
-                runs[ps - T0] = make_int2(total_rows, T0 + 16 - ps);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_MF + ring));
-            if (j >= NS && !lane0_wait(bar(B_KE + stage), (use - 1) & 1, 41)) break;
-            if (lane == 0) mbar_arrive_expect_tx(bar(B_KF + stage), L::KB);
-            __syncwarp();
-            issue(sK + stage * L::KB, maps.k, bar(B_KF + stage));
-            issued_k = j + 1;
-            if (j >= NS && !lane0_wait(bar(B_VE + stage), (use - 1) & 1, 42)) break;
-            if (lane == 0) mbar_arrive_expect_tx(bar(B_VF + stage), L::KB);
-            __syncwarp();
-            issue(sV + stage * L::KB, maps.v, bar(B_VF + stage));
-            issued_v = j + 1;
-            __syncwarp();
-        }
-        // every copy this CTA issued lands before the CTA can exit (abort or not)
-        if (lane == 0) {
-            mbar_wait(bar(B_Q), 0, nullptr, kSpin);
-            for (int t = max(0, issued_k - NS); t < issued_k; ++t)
-                mbar_wait(bar(B_KF + t % NS), (t / NS) & 1, nullptr, kSpin);
-            for (int t = max(0, issued_v - NS); t < issued_v; ++t)
-                mbar_wait(bar(B_VF + t % NS), (t / NS) & 1, nullptr, kSpin);
-        }
-    } else if (warp == 9) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_f32acc(128, 128, kFmtBF16, false);
-            constexpr uint32_t idesc_pv = idesc_f32acc(128, D, kFmtF16, true);
-            auto issue_s = [&](int t, int stage) {
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t a = smem_desc(sQ + t * L::QB + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
-                    const uint64_t b = smem_desc(sK + stage * L::KB + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
-                    mma_f16_ss(tmem + 128 * t, a, b, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-            };
-            auto issue_pv = [&](int t, int jj) {
-                const int stage = jj % NS;
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
-                    mma_f16_ts(tmem + 256 + D * t, tmem + 128 * t + kk * 8, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-            };
-            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int stage = j % NS;
-                if (!mbar_wait(bar(B_KF + stage), (j / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
-                if (j >= 1 && !mbar_wait(bar(B_VF + (j - 1) % NS), ((j - 1) / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
-                for (int t = 0; t < nq; ++t) {
-                    if (j >= 1) {
-                        if (!mbar_wait(bar(B_PF + t), (j - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
-                        tc_fence_after();
-                        issue_pv(t, j - 1);
+            const bool probe = it.a < 0;
+            const int32_t* sg = sel_groups + ((size_t)it.bh * Cq + (probe ? 0 : it.a)) * Ck;
+            const int32_t* ko = kv_off + (size_t)it.bh * (Ck + 1);
+            const int n_groups = probe ? 1 : sel_count[(size_t)it.bh * Cq + it.a];
+            int2* runs = reinterpret_cast<int2*>(sm + L::oRun);
+            int gbase = 0, w_begin = 0, w_end = 0, my_rs = 0, my_len = 0, my_sb = 0, my_se = 0;
+            auto load_window = [&]() {
+                const int g = gbase + lane;
+                my_rs = 0;
+                my_len = 0;
+                if (g < n_groups) {
+                    if (probe) {
+                        my_len = N;
+                    } else {
+                        const int b = sg[g];
+                        my_rs = ko[b];
+                        my_len = ko[b + 1] - my_rs;
                     }
-                    tc_fence_after();
-                    issue_s(t, stage);
-                    mma_commit(bar(B_SF + t));
                 }
+                const int ns = (my_len + 7) >> 3;
+                int incl = ns;
+    #pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                my_sb = w_begin + incl - ns;
+                my_se = w_begin + incl;
+                w_end = w_begin + __shfl_sync(0xffffffffu, incl, 31);
+            };
+            load_window();
+            int issued_k = 0, issued_v = 0;
+            auto lane0_wait = [&](uint32_t b, uint32_t parity, int where) -> bool {
+                int ok = 1;
+                if (lane == 0 && !mbar_wait(b, parity, abort_flag, kSpin)) {
+                    record_status(status, SPARSEPR_TIMEOUT, where);
+                    *abort_flag = 1;
+                    ok = 0;
+                }
+                return __shfl_sync(0xffffffffu, ok, 0) != 0;
+            };
+            auto issue = [&](uint32_t dst, const CUtensorMap* mp, uint32_t b) {
+                if (lane < 16) {
+                    const int2 rn = runs[lane];   // (first global row, slots) of a run starting at slot lane
+                    int done = 0;
+                    while (done < rn.y) {
+                        int k = 31 - __clz(rn.y - done);
+                        if (k > NBOX - 1) k = NBOX - 1;
+                        const int y = (rn.x == total_rows) ? total_rows : rn.x + 8 * done;
+                        for (int hh = 0; hh < D / 64; ++hh)
+                            tma_load_2d(dst + hh * BN * 128 + (lane + done) * 1024, &mp[k], b, hh * 64, y);
+                        done += 1 << k;
+                    }
+                }
+            };
+            for (int j = 0; j < n_tiles; ++j) {
+                const int stage = j % NS, use = j / NS, ring = j % RING;
+                const int T0 = 16 * j;
+                if (j >= RING && !lane0_wait(bar(B_ME + ring), ((j / RING) - 1) & 1, 40)) break;
+                uint8_t* vm = meta + ring * 16;
+                if (lane < 16) {
+                    vm[lane] = 0;
+                    runs[lane] = make_int2(0, 0);
+                }
+                __syncwarp();
+                while (true) {
+                    const int lo = max(my_sb, T0), hi = min(my_se, T0 + 16);
+                    if (lo < hi) {
+                        const int o = lo - my_sb;
+                        runs[lo - T0] = make_int2(it.bh * N + my_rs + 8 * o, hi - lo);
+                        for (int t = lo; t < hi; ++t) vm[t - T0] = (uint8_t)min(8, my_len - 8 * (t - my_sb));
+                    }
+                    if (w_end >= T0 + 16 || gbase + 32 >= n_groups) break;
+                    gbase += 32;
+                    w_begin = w_end;
+                    load_window();
+                }
+                if (lane == 0 && w_end < T0 + 16) {   // past the last group: zero-filled padding slots
+                    const int ps = max(w_end, T0);
+                    runs[ps - T0] = make_int2(total_rows, T0 + 16 - ps);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_MF + ring));
+                if (j >= NS && !lane0_wait(bar(B_KE + stage), (use - 1) & 1, 41)) break;
+                if (lane == 0) mbar_arrive_expect_tx(bar(B_KF + stage), L::KB);
+                __syncwarp();
+                issue(sK + stage * L::KB, maps.k, bar(B_KF + stage));
+                issued_k = j + 1;
+                if (j >= NS && !lane0_wait(bar(B_VE + stage), (use - 1) & 1, 42)) break;
+                if (lane == 0) mbar_arrive_expect_tx(bar(B_VF + stage), L::KB);
+                __syncwarp();
+                issue(sV + stage * L::KB, maps.v, bar(B_VF + stage));
+                issued_v = j + 1;
+                __syncwarp();
+            }
+            // every copy this CTA issued lands before the CTA can exit (abort or not)
+            if (lane == 0) {
+                mbar_wait(bar(B_Q), 0, nullptr, kSpin);
+                for (int t = max(0, issued_k - NS); t < issued_k; ++t)
+                    mbar_wait(bar(B_KF + t % NS), (t / NS) & 1, nullptr, kSpin);
+                for (int t = max(0, issued_v - NS); t < issued_v; ++t)
+                    mbar_wait(bar(B_VF + t % NS), (t / NS) & 1, nullptr, kSpin);
+            }
+        } else if (warp == 9) {
+            // ------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc_qk = idesc_f32acc(128, 128, kFmtBF16, false);
+                constexpr uint32_t idesc_pv = idesc_f32acc(128, D, kFmtF16, true);
+                auto issue_s = [&](int t, int stage) {
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t a = smem_desc(sQ + t * L::QB + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
+                        const uint64_t b = smem_desc(sK + stage * L::KB + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
+                        mma_f16_ss(tmem + 128 * t, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                };
+                auto issue_pv = [&](int t, int jj) {
+                    const int stage = jj % NS;
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
+                        mma_f16_ts(tmem + 256 + D * t, tmem + 128 * t + kk * 8, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                };
+                bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
+                for (int j = 0; ok && j < n_tiles; ++j) {
+                    const int stage = j % NS;
+                    if (!mbar_wait(bar(B_KF + stage), (j / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    if (j >= 1 && !mbar_wait(bar(B_VF + (j - 1) % NS), ((j - 1) / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    for (int t = 0; t < nq; ++t) {
+                        if (j >= 1) {
+                            if (!mbar_wait(bar(B_PF + t), (j - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                            tc_fence_after();
+                            issue_pv(t, j - 1);
+                        }
+                        tc_fence_after();
+                        issue_s(t, stage);
+                        mma_commit(bar(B_SF + t));
+                    }
+                    if (!ok) break;
+                    mma_commit(bar(B_KE + stage));
+                    if (j >= 1) mma_commit(bar(B_VE + (j - 1) % NS));
+                }
+                if (ok && n_tiles > 0) {
+                    const int jl = n_tiles - 1;
+                    if (!mbar_wait(bar(B_VF + jl % NS), (jl / NS) & 1, abort_flag, kSpin)) ok = false;
+                    for (int t = 0; ok && t < nq; ++t) {
+                        if (!mbar_wait(bar(B_PF + t), jl & 1, abort_flag, kSpin)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(t, jl);
+                    }
+                    if (ok) {
+                        mma_commit(bar(B_VE + jl % NS));
+                        mma_commit(bar(B_OF));
+                    }
+                }
+                if (!ok) {
+                    record_status(status, SPARSEPR_TIMEOUT, 43);
+                    *abort_flag = 1;
+                }
+                // every MMA issued above completes before TMEM is released
+                mma_commit(bar(B_DR));
+                mbar_wait(bar(B_DR), 0, nullptr, kSpin);
+            }
+        }
+    } else {
+        setmaxnreg_inc<kRegsSoftmax>();
+        if (warp < 4 * nq) {
+            // ------------------------------------------------ softmax of Q tile t (rows = TMEM lanes)
+            // The whole 128-key row of S is held in registers: one TMEM read, the
+            // row maximum, then P = exp2(s * scale - m_ref) as fp16 pairs.
+            const int t = warp >> 2, r = tid - 128 * t;
+            const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+            const uint32_t tS = t_row + 128 * t, tO = t_row + 256 + D * t;
+            float m_ref = -INFINITY;
+            float2 l2 = make_float2(0.f, 0.f);
+            bool ok = true;
+            auto mask_chunk = [&](float (&v)[32], const uint32_t (&vwa)[4], int c4) {
+    #pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int u = c4 * 4 + q;
+                    const int cnt = (int)((vwa[u >> 2] >> (8 * (u & 3))) & 0xffu);
+                    if (cnt < 8) {
+    #pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            if (i >= cnt) v[q * 8 + i] = -INFINITY;
+                    }
+                }
+            };
+            for (int j = 0; j < n_tiles; ++j) {
+                const int ring = j % RING;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + t), j & 1, abort_flag, kSpin));
                 if (!ok) break;
-                mma_commit(bar(B_KE + stage));
-                if (j >= 1) mma_commit(bar(B_VE + (j - 1) % NS));
+                tc_fence_after();
+                float sv[4][32];
+    #pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_MF + ring), (j / RING) & 1, abort_flag, kSpin));
+                tmem_wait_ld();
+                if (!ok) break;
+                const uint4 vw = *reinterpret_cast<const uint4*>(meta + ring * 16);
+                mbar_arrive(bar(B_ME + ring));
+                const uint32_t vwa[4] = {vw.x, vw.y, vw.z, vw.w};
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    #pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    mask_chunk(sv[c], vwa, c);
+    #pragma unroll
+                    for (int i = 0; i < 16; ++i) mx4[i & 3] = fmax3(mx4[i & 3], sv[c][2 * i], sv[c][2 * i + 1]);
+                }
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
+                const float m_new = fmaxf(m_ref, mx);
+                const bool need = (j > 0) && (m_new > m_ref + 8.f);
+                if (j == 0) m_ref = m_new;
+                if (__any_sync(0xffffffffu, need)) {   // O_t is quiescent: PV_t(j-1) completed before S_t(j)
+                    const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
+                    if (need) {
+                        m_ref = m_new;
+                        l2.x *= alpha;
+                        l2.y *= alpha;
+                    }
+    #pragma unroll
+                    for (int c4 = 0; c4 < D / 32; ++c4) {
+                        float v[32];
+                        tmem_ld32(tO + c4 * 32, v);
+                        tmem_wait_ld();
+    #pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                        tmem_st32(tO + c4 * 32, v);
+                    }
+                    tmem_wait_st();
+                }
+                // P = exp2(s * scale - m_ref) <= 2^8 as fp16, keys 2i and 2i+1 in
+                // column i of S's first 64 columns (all of S is already read).
+                // kSoftPairs of every 16 pairs, evenly spread, take the FMA-pipe
+            // exponential, which relieves the MUFU (two exponentials per pair).
+                const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_ref, -m_ref);
+                float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+    #pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t w[16];
+    #pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 x = ffma2(make_float2(sv[c][2 * i], sv[c][2 * i + 1]), sc2, nm2);
+                        float2 pr;
+                        if ((i * kSoftPairs) % 16 < kSoftPairs) {
+                            pr = exp2_fma2(x);
+                        } else {
+                            pr.x = ex2_approx(x.x);
+                            pr.y = ex2_approx(x.y);
+                        }
+                        if (i & 1) lb = fadd2(lb, pr);
+                        else la = fadd2(la, pr);
+                        const __half2 h = __floats2half2_rn(pr.x, pr.y);
+                        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    tmem_st16(tS + 16 * c, w);
+                }
+                l2 = fadd2(l2, fadd2(la, lb));
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_PF + t));
             }
             if (ok && n_tiles > 0) {
-                const int jl = n_tiles - 1;
-                if (!mbar_wait(bar(B_VF + jl % NS), (jl / NS) & 1, abort_flag, kSpin)) ok = false;
-                for (int t = 0; ok && t < nq; ++t) {
-                    if (!mbar_wait(bar(B_PF + t), jl & 1, abort_flag, kSpin)) { ok = false; break; }
-                    tc_fence_after();
-                    issue_pv(t, jl);
-                }
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF), 0, abort_flag, kSpin));
                 if (ok) {
-                    mma_commit(bar(B_VE + jl % NS));
-                    mma_commit(bar(B_OF));
+                    tc_fence_after();
+                    const int nrows = t == 0 ? it.n0 : it.n1;
+                    const int row = it.row0 + BM * t + r;
+                    float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + row) * D
+                                            : O_sp + ((size_t)it.bh * N + row) * D;
+                    const float inv = vscale[it.bh] / (l2.x + l2.y);
+    #pragma unroll
+                    for (int c4 = 0; c4 < D / 32; ++c4) {
+                        float v[32];
+                        tmem_ld32(tO + c4 * 32, v);
+                        tmem_wait_ld();
+                        if (r < nrows) {
+                            float4* o4 = reinterpret_cast<float4*>(out + c4 * 32);
+    #pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                o4[i] = make_float4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv,
+                                                    v[4 * i + 3] * inv);
+                        }
+                    }
                 }
             }
             if (!ok) {
-                record_status(status, SPARSEPR_TIMEOUT, 43);
+                record_status(status, SPARSEPR_TIMEOUT, 44);
                 *abort_flag = 1;
             }
-            // every MMA issued above completes before TMEM is released
-            mma_commit(bar(B_DR));
-            mbar_wait(bar(B_DR), 0, nullptr, kSpin);
-        }
-    } else if (warp < 4 * nq) {
-        // ------------------------------------------------ softmax of Q tile t (rows = TMEM lanes)
-        const int t = warp >> 2, r = tid - 128 * t;
-        const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const uint32_t tS = t_row + 128 * t, tO = t_row + 256 + D * t;
-        float m_ref = -INFINITY, l = 0.f;
-        bool ok = true;
-        auto mask_chunk = [&](float (&v)[32], const uint32_t (&vwa)[4], int c4) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int u = c4 * 4 + q;
-                const int cnt = (int)((vwa[u >> 2] >> (8 * (u & 3))) & 0xffu);
-                if (cnt < 8) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if (i >= cnt) v[q * 8 + i] = -INFINITY;
-                }
-            }
-        };
-        for (int j = 0; j < n_tiles; ++j) {
-            const int ring = j % RING;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SF + t), j & 1, abort_flag, kSpin));
-            if (!ok) break;
-            tc_fence_after();
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_MF + ring), (j / RING) & 1, abort_flag, kSpin));
-            if (!ok) break;
-            const uint4 vw = *reinterpret_cast<const uint4*>(meta + ring * 16);
-            mbar_arrive(bar(B_ME + ring));
-            const uint32_t vwa[4] = {vw.x, vw.y, vw.z, vw.w};
-            // row maximum over the 128 keys, read as two 64-column halves
-            // (ten warps share four register-file partitions: keep the live set small)
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float sv[2][32];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) tmem_ld32(tS + (2 * hf + q) * 32, sv[q]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    mask_chunk(sv[q], vwa, 2 * hf + q);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], sv[q][i]);
-                }
-            }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
-            const float m_new = fmaxf(m_ref, mx);
-            const bool need = (j > 0) && (m_new > m_ref + 8.f);
-            if (j == 0) m_ref = m_new;
-            if (__any_sync(0xffffffffu, need)) {   // O_t is quiescent: PV_t(j-1) completed before S_t(j)
-                const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
-                if (need) {
-                    m_ref = m_new;
-                    l *= alpha;
-                }
-#pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4) {
-                    float v[32];
-                    tmem_ld32(tO + c4 * 32, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                    tmem_st32(tO + c4 * 32, v);
-                }
-                tmem_wait_st();
-            }
-            // P = exp2(s * scale - m_ref) as fp16 (<= 2^8), two per column over S's first 64
-            // columns; one pair in four takes the FMA-pipe exponential to offload the MUFU.
-            // P half hf lands in columns [32 hf, 32 hf + 32), already read in both halves.
-            const float neg_m = -m_ref;
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float sv[2][32];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) tmem_ld32(tS + (2 * hf + q) * 32, sv[q]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    mask_chunk(sv[q], vwa, 2 * hf + q);
-                    uint32_t w[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float x0 = fmaf(sv[q][2 * i], scale_log2, neg_m);
-                        const float x1 = fmaf(sv[q][2 * i + 1], scale_log2, neg_m);
-                        const bool soft = kSoftEvery > 0 && (i % kSoftEvery) == kSoftEvery - 1;
-                        const float p0 = soft ? exp2_poly(x0) : ex2_approx(x0);
-                        const float p1 = soft ? exp2_poly(x1) : ex2_approx(x1);
-                        l4[i & 3] += p0 + p1;
-                        const __half2 pr = __floats2half2_rn(p0, p1);
-                        w[i] = *reinterpret_cast<const uint32_t*>(&pr);
-                    }
-                    tmem_st16(tS + (2 * hf + q) * 16, w);
-                }
-            }
-            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_PF + t));
         }
-        if (ok && n_tiles > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF), 0, abort_flag, kSpin));
-            if (ok) {
-                tc_fence_after();
-                const int nrows = t == 0 ? it.n0 : it.n1;
-                const int row = it.row0 + BM * t + r;
-                float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + row) * D
-                                        : O_sp + ((size_t)it.bh * N + row) * D;
-                const float inv = vscale[it.bh] / l;
-#pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4) {
-                    float v[32];
-                    tmem_ld32(tO + c4 * 32, v);
-                    tmem_wait_ld();
-                    if (r < nrows) {
-                        float4* o4 = reinterpret_cast<float4*>(out + c4 * 32);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            o4[i] = make_float4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv,
-                                                v[4 * i + 3] * inv);
-                    }
-                }
-            }
-        }
-        if (!ok) {
-            record_status(status, SPARSEPR_TIMEOUT, 44);
-            *abort_flag = 1;
-        }
-        tc_fence_before();
     }
     __syncthreads();
     if (warp == 9) {
@@ -782,6 +796,24 @@ bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int b
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The kernel's register split assumes kLaunchRegs registers per thread at
+// launch: with fewer, the softmax warpgroups' increase could never be met.
+bool tc_register_split_ok(int d) {
+    cudaFuncAttributes a;
+    const cudaError_t e = d == 128 ? cudaFuncGetAttributes(&a, attention_tc_kernel<128>)
+                                   : cudaFuncGetAttributes(&a, attention_tc_kernel<64>);
+    if (e != cudaSuccess) {
+        cuda_status(e);
+        return false;
+    }
+    if (a.numRegs != tc::kLaunchRegs || a.maxThreadsPerBlock < tc::kThreads) {
+        snprintf(last_error_buffer(), 256, "attention_tc_kernel<%d>: built with %d registers per thread, %d expected",
+                 d, a.numRegs, tc::kLaunchRegs);
+        return false;
+    }
+    return true;
+}
+
 inline int grid_for(size_t total, int threads) {
     size_t g = (total + threads - 1) / threads;
     return (int)(g > 148 * 64 ? 148 * 64 : (g == 0 ? 1 : g));
@@ -843,17 +875,18 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
         if (Mp > 0) ok = ok && make_rows_map(&maps.qp, qprobe, (uint64_t)BH * Mp, d, 128, false);
         else maps.qp = maps.q;
         if (!ok) return SPARSEPR_CUDA_ERROR;
+        if (!tc_register_split_ok(d)) return SPARSEPR_UNSUPPORTED;
         if (d == 128) {
             auto k = attention_tc_kernel<128>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<128>::smem);
-            count_launch(), k<<<grid2, 320, tc::Layout<128>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
+            count_launch(), k<<<grid2, tc::kThreads, tc::Layout<128>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
                                                                        pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
                                                                        r.sel_count, r.sel_groups, vscale, O_sp,
                                                                        probe_dense, status, visited, scale_log2);
         } else {
             auto k = attention_tc_kernel<64>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<64>::smem);
-            count_launch(), k<<<grid2, 320, tc::Layout<64>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
+            count_launch(), k<<<grid2, tc::kThreads, tc::Layout<64>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
                                                                       pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
                                                                       r.sel_count, r.sel_groups, vscale, O_sp,
                                                                       probe_dense, status, visited, scale_log2);

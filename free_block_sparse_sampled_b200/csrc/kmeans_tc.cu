@@ -25,8 +25,8 @@ constexpr int oA = 0;                                   // 2 buffers x 2 chunks 
 constexpr int oB = oA + 2 * 2 * BP * 128;               // 2 stages x 2 chunks x 256 rows x 128 B
 constexpr int oBar = oB + 2 * 2 * NBMAX * 128;
 constexpr int oRed = oBar + N_BAR * 8;                  // 128 x (score, index) of the upper half
-constexpr int oHn = oRed + BP * 8;                      // 2 x 256 half-norms of the centre block
-constexpr int oMisc = oHn + 2 * NBMAX * 4;
+constexpr int oHn = oRed + BP * 8;                      // negated half-norms of the head's centres
+constexpr int oMisc = oHn + kMaxGroups * 4;
 constexpr int kSmem = oMisc + 64 + 1024;
 
 struct Maps {
@@ -155,57 +155,73 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         float* red_s = reinterpret_cast<float*>(sm + oRed);
         int* red_i = reinterpret_cast<int*>(sm + oRed + BP * 4);
         float* hns = reinterpret_cast<float*>(sm + oHn);
-        int gb = 0;
+        int gb = 0, staged_bh = -1;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
             if (!item_live(w)) continue;
             const int bh = w / tiles_per_head, p = (w % tiles_per_head) * BP + row;
             const bool valid = p < N;
             int32_t* hc = ctl + bh * kCtlStride;
-            // four independent argmax chains (columns c = 4k + q), merged lowest index first
-            float best4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            int bi4[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+            // previous label, read now and used after the last centre block
+            const int old_label = (valid && !first) ? labels[(size_t)bh * N + p] : 0;
+            if (bh != staged_bh) {   // a persistent block's items mostly share a head: stage its centres' -|c|^2/2 once
+                asm volatile("bar.sync 1, 256;" ::: "memory");   // the previous head's table is no longer read
+                for (int c = tid; c < nblk * NB; c += 256) hns[c] = (c < C) ? -hn[(size_t)bh * C + c] : -INFINITY;
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                staged_bh = bh;
+            }
+            // running first maximum over this half's columns, in column order
+            float best = -INFINITY;
+            int bi = 0x7fffffff;
             for (int blk = 0; blk < nblk; ++blk, ++gb) {
                 const int db = gb & 1;
-                // half-norms of this centre block (columns past C never win)
-                float* hb = hns + db * NBMAX;
-                for (int c = tid; c < NB; c += 256) {
-                    const int cg = blk * NB + c;
-                    hb[c] = (cg < C) ? hn[(size_t)bh * C + cg] : INFINITY;
-                }
-                asm volatile("bar.sync 1, 256;" ::: "memory");
+                const float* hb = hns + blk * NB;   // columns past C hold -inf and never win
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + db), (gb >> 1) & 1, abort_flag, kSpin));
                 if (!ok) break;
                 tc_fence_after();
-                for (int c0 = 0; c0 < hw; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(t_row + db * NB + half * hw + c0, v);
+                for (int c0 = 0; c0 < hw; c0 += 64) {
+                    const bool two = c0 + 32 < hw;   // warp-uniform
+                    float v[2][32];
+                    tmem_ld32(t_row + db * NB + half * hw + c0, v[0]);
+                    if (two) tmem_ld32(t_row + db * NB + half * hw + c0 + 32, v[1]);
                     tmem_wait_ld();
-                    const int cb = blk * NB + half * hw + c0;
-                    const float* hr = hb + half * hw + c0;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float sc = v[i] - hr[i];
-                        if (DBG) {
-                            if (valid && cb + i < C) dbg_scores[((size_t)bh * N + p) * C + cb + i] = sc;
+                    for (int q = 0; q < 2; ++q) {
+                        if (q == 1 && !two) break;
+                        const int cb = blk * NB + half * hw + c0 + 32 * q;
+                        const float2* hr = reinterpret_cast<const float2*>(hb + half * hw + c0 + 32 * q);
+                        float sc[32];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float2 x = fadd2(make_float2(v[q][2 * i], v[q][2 * i + 1]), hr[i]);
+                            sc[2 * i] = x.x;
+                            sc[2 * i + 1] = x.y;
                         }
-                        if (sc > best4[i & 3]) {
-                            best4[i & 3] = sc;
-                            bi4[i & 3] = cb + i;
+                        if (DBG) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (valid && cb + i < C) dbg_scores[((size_t)bh * N + p) * C + cb + i] = sc[i];
+                        }
+                        // chunk maximum as a tree of three-way maxima
+                        float m3[11];
+#pragma unroll
+                        for (int i = 0; i < 10; ++i) m3[i] = fmax3(sc[3 * i], sc[3 * i + 1], sc[3 * i + 2]);
+                        m3[10] = fmaxf(sc[30], sc[31]);
+                        const float m = fmaxf(fmax3(fmax3(m3[0], m3[1], m3[2]), fmax3(m3[3], m3[4], m3[5]),
+                                                    fmax3(m3[6], m3[7], m3[8])),
+                                              fmaxf(m3[9], m3[10]));
+                        if (m > best) {   // a later chunk only wins with a strictly larger score
+                            int idx = 31;
+#pragma unroll
+                            for (int i = 30; i >= 0; --i) idx = (sc[i] == m) ? i : idx;
+                            best = m;
+                            bi = cb + idx;
                         }
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(bar(B_DE + db));
             }
-            float best = best4[0];
-            int bi = bi4[0];
-#pragma unroll
-            for (int q = 1; q < 4; ++q)
-                if (best4[q] > best || (best4[q] == best && bi4[q] < bi)) {
-                    best = best4[q];
-                    bi = bi4[q];
-                }
             if (!ok) break;
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (half == 1) {
@@ -224,7 +240,7 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                 int changed = 0;
                 if (valid) {
                     int32_t* lp = labels + (size_t)bh * N + p;
-                    changed = (!first) && (*lp != bi);
+                    changed = (!first) && (old_label != bi);
                     *lp = bi;
                     if (dbg_hist != nullptr) dbg_hist[((size_t)bh * max_iter + hc[kCtlIters]) * N + p] = bi;
                 }

@@ -404,45 +404,65 @@ __global__ void __launch_bounds__(1024) label_hist_kernel(const int32_t* __restr
     for (int c = threadIdx.x; c < C; c += blockDim.x) dst[c] = h[c];
 }
 
-// Turns the per-tile counts into scatter bases and writes group offsets [C+1].
-__global__ void __launch_bounds__(1024) label_scan_kernel(int32_t* __restrict__ hist, int N, int C,
-                                                          int n_tiles, int32_t* __restrict__ offs,
-                                                          const int32_t* __restrict__ ctl) {
+// Per label c: exclusive prefix of the per-tile counts over the tiles (in
+// place) and the label's total, written to offs[c].  One thread per label.
+__global__ void __launch_bounds__(256) label_colscan_kernel(int32_t* __restrict__ hist, int C, int n_tiles,
+                                                            int32_t* __restrict__ offs,
+                                                            const int32_t* __restrict__ ctl) {
+    const int bh = blockIdx.y, c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (ctl != nullptr && ctl[bh * kCtlStride + kCtlDone]) return;
+    if (c >= C) return;
+    int32_t* hh = hist + (size_t)bh * n_tiles * C + c;
+    int run = 0;
+    int t = 0;
+    for (; t + 8 <= n_tiles; t += 8) {   // eight loads in flight
+        int v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = hh[(size_t)(t + u) * C];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            hh[(size_t)(t + u) * C] = run;
+            run += v[u];
+        }
+    }
+    for (; t < n_tiles; ++t) {
+        const int v = hh[(size_t)t * C];
+        hh[(size_t)t * C] = run;
+        run += v;
+    }
+    offs[(size_t)bh * (C + 1) + c] = run;
+}
+
+// Label totals -> group offsets [C+1] (exclusive scan, offs[C] = N).
+__global__ void __launch_bounds__(1024) label_offsets_kernel(int32_t* __restrict__ offs, int N, int C,
+                                                             const int32_t* __restrict__ ctl) {
     const int bh = blockIdx.x;
     if (ctl != nullptr && ctl[bh * kCtlStride + kCtlDone]) return;
     __shared__ int tot[kMaxGroups];
     __shared__ int scratch[33];
-    int32_t* hh = hist + (size_t)bh * n_tiles * C;
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-        int run = 0;
-        for (int t = 0; t < n_tiles; ++t) {
-            const int v = hh[(size_t)t * C + c];
-            hh[(size_t)t * C + c] = run;
-            run += v;
-        }
-        tot[c] = run;
-    }
+    int32_t* oo = offs + (size_t)bh * (C + 1);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) tot[c] = oo[c];
     __syncthreads();
     block_exclusive_scan(tot, C, scratch);
-    int32_t* oo = offs + (size_t)bh * (C + 1);
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-        const int base = tot[c];
-        oo[c] = base;
-        for (int t = 0; t < n_tiles; ++t) hh[(size_t)t * C + c] += base;
-    }
+    for (int c = threadIdx.x; c < C; c += blockDim.x) oo[c] = tot[c];
     if (threadIdx.x == 0) oo[C] = N;
 }
 
+// Scatter of one tile's points to their sorted positions: the label's group
+// offset + the counts of earlier tiles + the rank among equal labels of
+// lower index in this tile (warps in order), so the sort is stable.
 __global__ void __launch_bounds__(1024) label_scatter_kernel(const int32_t* __restrict__ labels, int N,
                                                              int C, int n_tiles,
                                                              const int32_t* __restrict__ hist,
+                                                             const int32_t* __restrict__ offs,
                                                              int32_t* __restrict__ sorted,
                                                              const int32_t* __restrict__ ctl) {
     const int bh = blockIdx.y, tile = blockIdx.x;
     if (ctl != nullptr && ctl[bh * kCtlStride + kCtlDone]) return;
     __shared__ int cnt[kMaxGroups];
     const int32_t* base = hist + ((size_t)bh * n_tiles + tile) * C;
-    for (int c = threadIdx.x; c < C; c += blockDim.x) cnt[c] = base[c];
+    const int32_t* go = offs + (size_t)bh * (C + 1);
+    for (int c = threadIdx.x; c < C; c += blockDim.x) cnt[c] = base[c] + go[c];
     __syncthreads();
     const int i = tile * kSortTile + threadIdx.x;
     const int lab = (i < N) ? labels[(size_t)bh * N + i] : -1;
@@ -464,61 +484,78 @@ __global__ void __launch_bounds__(1024) label_scatter_kernel(const int32_t* __re
     }
 }
 
-// Centre update: member mean in sorted (index) order, rounded to TF32; empty
-// centres keep their value.  One warp per centre.
+// Centre update: member mean, rounded to TF32; empty centres keep their
+// value.  One warp per centre: a member row is read as R/4 float4 lanes, so
+// one warp load covers 32/(R/4) rows (lanes past that stay idle for R = 48).
+// Rows are assigned to (load, row slot) by their position in the sorted
+// member list and the partial sums are combined in a fixed order, so the
+// result depends only on the labels.
 template <int R>
 __global__ void centre_update_kernel(const float* __restrict__ phi, const int32_t* __restrict__ sorted,
                                      const int32_t* __restrict__ offs, int N, int C,
                                      float* __restrict__ cen, float* __restrict__ hn,
                                      const int32_t* __restrict__ ctl) {
+    static_assert(R % 16 == 0 && R >= 16 && R <= 64, "coordinate rows of 16..64 floats");
+    constexpr int LPR = R / 4;        // lanes per row
+    constexpr int RPL = 32 / LPR;     // rows per warp load
+    constexpr int LOADS = 32 / RPL;   // loads per 32 listed members
+    constexpr int U = 4;              // independent accumulators per lane
     const int bh = blockIdx.y, lane = threadIdx.x & 31;
     if (ctl[bh * kCtlStride + kCtlDone]) return;
     const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (c >= C) return;
     const int s = offs[(size_t)bh * (C + 1) + c], e = offs[(size_t)bh * (C + 1) + c + 1];
     if (e == s) return;
-    constexpr int PL = (R + 31) / 32;
-    constexpr int U = 8;   // member rows in flight per lane; partial sums combined in a fixed order
-    float acc[U][PL];
+    const int slot = lane / LPR, part = lane % LPR;
+    const bool active = slot < RPL;
+    float4 acc[U];
 #pragma unroll
-    for (int k = 0; k < U; ++k)
-#pragma unroll
-        for (int u = 0; u < PL; ++u) acc[k][u] = 0.f;
-    const float* ph = phi + (size_t)bh * N * R;
+    for (int k = 0; k < U; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* ph = reinterpret_cast<const float4*>(phi + (size_t)bh * N * R) + part;
     const int32_t* so = sorted + (size_t)bh * N;
     for (int p0 = s; p0 < e; p0 += 32) {
-        const int my = (p0 + lane < e) ? so[p0 + lane] : -1;   // 32 member indices per load
+        const int my = (p0 + lane < e) ? so[p0 + lane] : 0;   // 32 member indices per load
         const int n = min(32, e - p0);
-        for (int q0 = 0; q0 < n; q0 += U) {
 #pragma unroll
-            for (int k = 0; k < U; ++k) {
-                const int row = __shfl_sync(0xffffffffu, my, (q0 + k) & 31);
-                if (q0 + k < n) {
-                    const float* rp = ph + (size_t)row * R;
-#pragma unroll
-                    for (int u = 0; u < PL; ++u) {
-                        const int t = lane + 32 * u;
-                        if (t < R) acc[k][u] += rp[t];
-                    }
-                }
+        for (int k = 0; k < LOADS; ++k) {
+            const int q = RPL * k + slot;
+            const int row = __shfl_sync(0xffffffffu, my, q & 31);
+            if (active && q < n) {
+                const float4 x = ph[(size_t)row * LPR];
+                float4& a = acc[k % U];
+                a.x += x.x;
+                a.y += x.y;
+                a.z += x.z;
+                a.w += x.w;
             }
         }
     }
+    float4 t = acc[0];
 #pragma unroll
-    for (int u = 0; u < PL; ++u)
-        acc[0][u] = ((acc[0][u] + acc[1][u]) + (acc[2][u] + acc[3][u])) +
-                    ((acc[4][u] + acc[5][u]) + (acc[6][u] + acc[7][u]));
+    for (int k = 1; k < U; ++k) {
+        t.x += acc[k].x;
+        t.y += acc[k].y;
+        t.z += acc[k].z;
+        t.w += acc[k].w;
+    }
+    // row slots -> slot 0 (lane = slot * LPR + part), fixed tree order
+#pragma unroll
+    for (int o = LPR; o < RPL * LPR; o <<= 1) {
+        t.x += __shfl_down_sync(0xffffffffu, t.x, o);
+        t.y += __shfl_down_sync(0xffffffffu, t.y, o);
+        t.z += __shfl_down_sync(0xffffffffu, t.z, o);
+        t.w += __shfl_down_sync(0xffffffffu, t.w, o);
+    }
     const float count = (float)(e - s);
     float ss = 0.f;
-    float* dst = cen + ((size_t)bh * C + c) * R;
-#pragma unroll
-    for (int u = 0; u < PL; ++u) {
-        const int t = lane + 32 * u;
-        if (t < R) {
-            const float m = tf32_round(acc[0][u] / count);
-            dst[t] = m;
-            ss = fmaf(m, m, ss);
-        }
+    if (lane < LPR) {
+        float4 m;
+        m.x = tf32_round(t.x / count);
+        m.y = tf32_round(t.y / count);
+        m.z = tf32_round(t.z / count);
+        m.w = tf32_round(t.w / count);
+        reinterpret_cast<float4*>(cen + ((size_t)bh * C + c) * R)[part] = m;
+        ss = fmaf(m.x, m.x, fmaf(m.y, m.y, fmaf(m.z, m.z, m.w * m.w)));
     }
     ss = warp_sum(ss);
     if (lane == 0) hn[(size_t)bh * C + c] = 0.5f * ss;
@@ -656,13 +693,15 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
     count_launch(), kmeans_reset_kernel<<<bgrid, 128, 0, st>>>(ctl, BH, save_slot);
     count_launch(), kmeans_init_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, N, C, p.seed, stage, cen, hn);
     const dim3 agrid((N + 127) / 128, BH);
-    const dim3 tgrid(pl.n_sort_tiles, BH);
+    const dim3 tgrid(pl.n_sort_tiles, BH), cgrid((C + 255) / 256, BH);
     for (int it = 0; it < p.kmeans_iters; ++it) {
         const int first = it == 0;
         if (!first) {
             count_launch(), label_hist_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, ctl);
-            count_launch(), label_scan_kernel<<<BH, 1024, 0, st>>>(hist, N, C, pl.n_sort_tiles, offs, ctl);
-            count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, sorted, ctl);
+            count_launch(), label_colscan_kernel<<<cgrid, 256, 0, st>>>(hist, C, pl.n_sort_tiles, offs, ctl);
+            count_launch(), label_offsets_kernel<<<BH, 1024, 0, st>>>(offs, N, C, ctl);
+            count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, offs,
+                                                                              sorted, ctl);
             count_launch(), centre_update_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, sorted, offs, N, C, cen, hn, ctl);
         }
         if (!launch_kmeans_assign_tc(phi, cen, hn, BH, N, C, R, raw, ctl, first, dbg_scores, dbg_hist,
@@ -709,8 +748,11 @@ void finalize_groups(const Plan& pl, void* ws, int C, int which, int32_t* label_
     const int BH = pl.BH, N = pl.N;
     const dim3 tgrid(pl.n_sort_tiles, BH);
     count_launch(), label_hist_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, nullptr);
-    count_launch(), label_scan_kernel<<<BH, 1024, 0, st>>>(hist, N, C, pl.n_sort_tiles, offs, nullptr);
-    count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, sorted, nullptr);
+    count_launch(), label_colscan_kernel<<<dim3((C + 255) / 256, BH), 256, 0, st>>>(hist, C, pl.n_sort_tiles, offs,
+                                                                                   nullptr);
+    count_launch(), label_offsets_kernel<<<BH, 1024, 0, st>>>(offs, N, C, nullptr);
+    count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, offs, sorted,
+                                                                      nullptr);
     count_launch(), compact_groups_kernel<<<BH, 1024, 0, st>>>(offs, C, N, newid, offs_out, ng, which);
     count_launch(), relabel_kernel<<<grid_for((size_t)BH * N, 256), 256, 0, st>>>(raw, newid, sorted, BH, N, C,
                                                                   label_out, perm_out, pos_out);

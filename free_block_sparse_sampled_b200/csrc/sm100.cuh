@@ -153,18 +153,60 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t ab_fo
            | ((uint32_t)(M >> 4) << 24);
 }
 
-// 2^x on the FMA pipe, for x <= 127: Cody-Waite range reduction x = n + f with
-// n = floor(x) (exact for base 2), then 2^f on [0,1) from a cubic fitted here by
-// least squares on Chebyshev nodes (relative error below 7.5e-5, under the
-// fp16 rounding of the attention weights), and 2^n added to the exponent bits.
-// Results below 2^-126 flush to zero.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -127.f);
-    const float n = floorf(x);
-    const float f = x - n;
-    const float p = fmaf(fmaf(fmaf(0.07802443f, f, 0.22606729f), f, 0.69583350f), f, 0.99992520f);
-    const int ni = __float2int_rn(n);
-    return ni < -126 ? 0.f : __int_as_float(__float_as_int(p) + ni * (1 << 23));
+// ---------------------------------------------------------------- packed fp32 (two lanes per instruction)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for two lanes on the FMA pipe, x <= 15 (smaller x clamps at -125).
+// x = j + f with j = rint(x), taken by adding and removing 1.5 * 2^23, and
+// f in [-0.5, 0.5]; 2^f is a cubic fitted here to 2^f on that interval for
+// minimum relative error (7.5e-5, below the 2^-11 rounding of the fp16 P it
+// feeds); j is then added to the exponent field.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kShift = 12582912.f;   // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = fadd2(x, make_float2(kShift, kShift));
+    const float2 jf = fadd2(t, make_float2(-kShift, -kShift));
+    const float2 f = fadd2(x, make_float2(-jf.x, -jf.y));
+    float2 p = ffma2(make_float2(0.05517115443944931f, 0.05517115443944931f), f,
+                     make_float2(0.2426101416349411f, 0.2426101416349411f));
+    p = ffma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    p = ffma2(p, f, make_float2(0.9999281167984009f, 0.9999281167984009f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same instruction).  An increase waits until registers released by other
+// warpgroups of the block cover it, so the shares must add up to the launch's.
+template <int R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
 }
 
 // Hardware base-2 exponential (MUFU); exp2(-inf) = +0.
