@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wide")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with this many heads (smaller cases for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the dense/e2e/accuracy extras")
@@ -58,6 +60,22 @@ def measured_peaks():
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
     except (OSError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profiled_traffic(w):
+    """DRAM bytes per attention launch from the committed ncu capture
+    (profiles/attention_tc_wide_h4.json), scaled from its head count to w's;
+    None when the kernel source has changed since the capture or the
+    workload is not the one captured."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "attention_tc_wide_h4.json")))
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, ValueError, KeyError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec["source_sha256"] or w.name.split("_h")[0] != "wide":
+        return None
+    return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * (w.B * w.H) / rec["heads"]
 
 
 # --------------------------------------------------------------------- clocks
@@ -306,7 +324,7 @@ def run_ours(args, w):
     peaks, peak_kind = measured_peaks()
     achieved = attn_flops / (ms_attn * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic(w),
                 "kernel": "attention_tc_kernel<128> (+ work list and probe gathers)",
                 "peak_source": f"{peak_kind} bf16 dense (burst)"}
 
@@ -399,6 +417,8 @@ def main():
     args = parse()
     from synthetic import get_workload
     w = get_workload(args.workload)
+    if args.heads is not None:
+        w = w.replace(name=f"{w.name}_h{args.heads}", H=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
     else:
