@@ -596,16 +596,16 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
             float m_ref = -INFINITY;
             float2 l2 = make_float2(0.f, 0.f);
             bool ok = true;
-            auto mask_chunk = [&](float (&v)[32], const uint32_t (&vwa)[4], int c4) {
-    #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int u = c4 * 4 + q;
-                    const int cnt = (int)((vwa[u >> 2] >> (8 * (u & 3))) & 0xffu);
-                    if (cnt < 8) {
-    #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            if (i >= cnt) v[q * 8 + i] = -INFINITY;
-                    }
+            // Keys past a group's end in a partial 8-key slot, and padding slots,
+            // get -inf.  w holds the valid counts of the chunk's four slots; a
+            // chunk of full slots (the common case) takes one uniform test.
+            auto mask_chunk = [&](float (&v)[32], uint32_t w) {
+                if (w != 0x08080808u) {
+                    uint32_t valid = 0;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) valid |= ((1u << ((w >> (8 * q)) & 0xffu)) - 1u) << (8 * q);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = ((valid >> i) & 1u) ? v[i] : -INFINITY;
                 }
             };
             for (int j = 0; j < n_tiles; ++j) {
@@ -625,7 +625,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    mask_chunk(sv[c], vwa, c);
+                    mask_chunk(sv[c], vwa[c]);
     #pragma unroll
                     for (int i = 0; i < 16; ++i) mx4[i & 3] = fmax3(mx4[i & 3], sv[c][2 * i], sv[c][2 * i + 1]);
                 }
