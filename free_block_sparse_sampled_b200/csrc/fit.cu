@@ -283,6 +283,8 @@ sparsepr_status run_apply(const sparsepr_params& p, const Plan& pl, const sparse
     if (pl.Mp > 0)
         count_launch(), probe_slot_kernel<<<(pl.BH * pl.Mp + 255) / 256, 256, 0, st>>>(r.probe_idx, part.pos_q, pl.BH, pl.N, pl.Mp,
                                                                        pslot);
+    if (launch_apply_tc(pl, part, O_sp, probe_dense, f, pslot, O_out, at<DevStatus>(ws, pl.o_status), st))
+        return cuda_status(cudaGetLastError());
     const int d = pl.d;
     const size_t smem = (size_t)(d * d + 64 * (d + 4) + 3 * d) * sizeof(float);
     const dim3 grid((pl.N + 63) / 64, pl.BH);

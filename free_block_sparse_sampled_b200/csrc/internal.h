@@ -20,6 +20,10 @@ bool launch_route_tc(const Plan& pl, const sparsepr_partition_out& part, void* w
 bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, int BH, int N, int C, int R,
                              int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
                              int max_iter, DevStatus* status, cudaStream_t st);
+// Tensor-core corrected output (d = 64 or 128); false if d is not supported.
+bool launch_apply_tc(const Plan& pl, const sparsepr_partition_out& part, const float* O_sp, const float* probe_dense,
+                     const sparsepr_fit_out& f, const int32_t* pslot, float* O_out, DevStatus* status,
+                     cudaStream_t st);
 sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
                               const sparsepr_route_out& r, float* O_sp, float* probe_dense,
                               float* probe_sparse, void* ws, cudaStream_t st);

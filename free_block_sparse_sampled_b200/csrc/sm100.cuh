@@ -154,8 +154,8 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
 }
 
 // Instruction descriptor for kind::f16 with FP32 accumulation; A and B share
-// one format: 0 = F16, 1 = BF16.
-constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1;
+// one format: 0 = F16, 1 = BF16 (kind::f16), 2 = TF32 (kind::tf32).
+constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1, kFmtTF32 = 2;
 __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, uint32_t ab_format, bool b_mn_major) {
     return (1u << 4)                       // D format: F32
            | (ab_format << 7)              // A format
@@ -249,6 +249,16 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
 }
 
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread completes.
+// D[tmem] (+)= A[smem] * B[smem], TF32 operands (fp32 storage)
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
