@@ -228,28 +228,18 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + stage), (t >> 1) & 1, abort_flag, kSpin));
             if (!ok) break;
             tc_fence_after();
-            float x[BK];
+            const int ncol = min(BK, j_end - j0);
+            // pass 1: the tile's maximum logit (log2 units) moves the open group's reference
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c4 = 0; c4 < BK / 32; ++c4) {
                 float v[32];
                 tmem_ld32(t_row + stage * BK + c4 * 32, v);
+                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[c4 * 32 + i] = v[i] * cs;
+                for (int i = 0; i < 32; ++i)
+                    if (c4 * 32 + i < ncol) m4[i & 3] = fmaxf(m4[i & 3], v[i] * cs);
             }
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(B_DE + stage));
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_MF + ring), (t / RING) & 1, abort_flag, kSpin));
-            if (!ok) break;
-            const float* meta = reinterpret_cast<const float*>(sm + L::oMeta + ring * L::META);
-            const uint32_t* endm = reinterpret_cast<const uint32_t*>(meta + 2 * BK);
-            const int ncol = min(BK, j_end - j0);
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int c = 0; c < BK; c += 4)
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (c + q < ncol) m4[q] = fmaxf(m4[q], x[c + q]);
             const float Mn = fmaxf(Mr, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
             if (Mn > Mr) {
                 const float f = (Mr == -INFINITY) ? 0.f : ex2_approx(Mr - Mn);
@@ -257,26 +247,42 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
                 t2 *= f * f;
                 Mr = Mn;
             }
-            uint32_t em[4] = {endm[0], endm[1], endm[2], endm[3]};
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_MF + ring), (t / RING) & 1, abort_flag, kSpin));
+            if (!ok) break;
+            const float* meta = reinterpret_cast<const float*>(sm + L::oMeta + ring * L::META);
+            const uint32_t* endm = reinterpret_cast<const uint32_t*>(meta + 2 * BK);
+            // pass 2, one 32-key chunk at a time (a rolled loop keeps the code small):
+            // segment sums, flushed at every key-group end
+#pragma unroll 1
+            for (int c4 = 0; c4 < BK / 32; ++c4) {
+                float v[32];
+                tmem_ld32(t_row + stage * BK + c4 * 32, v);
+                tmem_wait_ld(v);
+                const uint32_t em = endm[c4];
+                const float* u = meta + c4 * 32;
+                const float* wv = meta + BK + c4 * 32;
 #pragma unroll
-            for (int c = 0; c < BK; ++c) {
-                if (c < ncol) {
-                    const float e = ex2_approx(x[c] - Mr);
-                    t1 = fmaf(e, meta[c], t1);
-                    t2 = fmaf(e * e, meta[BK + c], t2);
-                    if (em[c >> 5] & (1u << (c & 31))) {   // group b ends at this key (same for every row)
-                        if (a < Cqp) {
-                            const size_t idx = ((size_t)bh * Cq + a) * Ck + b;
-                            mloc[idx] = Mr * 0.6931471805599453f;   // back to natural-log units
-                            t1o[idx] = t1;
-                            t2o[idx] = t2;
+                for (int i = 0; i < 32; ++i) {
+                    if (c4 * 32 + i < ncol) {
+                        const float e = ex2_approx(fmaf(v[i], cs, -Mr));
+                        t1 = fmaf(e, u[i], t1);
+                        t2 = fmaf(e * e, wv[i], t2);
+                        if (em & (1u << i)) {   // group b ends at this key (same for every row)
+                            if (a < Cqp) {
+                                const size_t idx = ((size_t)bh * Cq + a) * Ck + b;
+                                mloc[idx] = Mr * 0.6931471805599453f;   // back to natural-log units
+                                t1o[idx] = t1;
+                                t2o[idx] = t2;
+                            }
+                            ++b;
+                            t1 = 0.f;
+                            t2 = 0.f;
                         }
-                        ++b;
-                        t1 = 0.f;
-                        t2 = 0.f;
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(bar(B_DE + stage));
             mbar_arrive(bar(B_ME + ring));
         }
         if (!ok) {
