@@ -1,6 +1,7 @@
 // Stage entry points shared by the C ABI (api.cu) and the stage files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -20,6 +21,14 @@ bool launch_route_tc(const Plan& pl, const sparsepr_partition_out& part, void* w
 bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, int BH, int N, int C, int R,
                              int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
                              int max_iter, DevStatus* status, cudaStream_t st);
+// 2-D tensor map over [rows, cols] row-major elements (4-byte fp32, or 2-byte
+// fp16 / bf16 chosen by is_float), boxes of box_cols x box_rows, 128-byte swizzle.
+bool encode_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int elem_bytes, bool is_float,
+                     uint32_t box_cols, uint32_t box_rows);
+// Tensor-core projection phi = X F (bf16 X, R in {16,32,48,64}, optional RMS
+// normalisation); false if it cannot run (its tensor map could not be built).
+bool launch_project_tc(const void* X, const float* F, int BH, int N, int d, int R, bool rms, const int32_t* r_eff,
+                       float eps, float* phi, DevStatus* status, cudaStream_t st);
 // Tensor-core corrected output (d = 64 or 128); false if d is not supported.
 bool launch_apply_tc(const Plan& pl, const sparsepr_partition_out& part, const float* O_sp, const float* probe_dense,
                      const sparsepr_fit_out& f, const int32_t* pslot, float* O_out, DevStatus* status,

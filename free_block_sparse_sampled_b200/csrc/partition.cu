@@ -725,7 +725,8 @@ void kmeans_dispatch(int R, const Plan& pl, const sparsepr_params& p, void* ws, 
 
 template <typename T, bool RMS>
 void project_dispatch(int R, const T* X, const float* F, int BH, int N, int d, const int32_t* r_eff,
-                      float eps, float* phi, cudaStream_t st) {
+                      float eps, float* phi, DevStatus* status, cudaStream_t st) {
+    if (sizeof(T) == 2 && launch_project_tc(X, F, BH, N, d, R, RMS, r_eff, eps, phi, status, st)) return;
     const dim3 grid((N + 127) / 128, BH);
     const size_t smem = (size_t)d * R * sizeof(float);
     switch (R) {
@@ -793,7 +794,7 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff, mat);
     count_launch(), jacobi<<<BH, 512, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d),
                                                       nullptr, 16);
-    project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, st);
+    project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
     // 3. paired K/V groups
     kmeans_dispatch(pl.RKp, pl, p, ws, phiK, pl.Ck, 0, cenK, hnK, dbg ? out.debug_kv_scores : nullptr,
                     dbg ? out.debug_kv_hist : nullptr, -1, st);
@@ -810,7 +811,7 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
                                                                           out.n_groups, pl.Ck, d, mat);
     count_launch(), jacobi<<<BH, 512, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16);
-    project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, st);
+    project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, at<DevStatus>(ws, pl.o_status), st);
     // 5. query groups
     kmeans_dispatch(pl.RQp, pl, p, ws, phiQ, pl.Cq, 1, cenQ, hnQ, dbg ? out.debug_q_scores : nullptr,
                     dbg ? out.debug_q_hist : nullptr, kCtlItersK, st);
