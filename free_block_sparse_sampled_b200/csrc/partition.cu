@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256) centred_gram_kernel(const float* __restri
 // (descending, ties to the lower index) and zero columns up to Rp.
 // For the query factor (ng != nullptr) r = max(1, min(r_req, d, C_k' - 1)).
 template <int d>
-__global__ void __launch_bounds__(512) jacobi_factor_kernel(const float* __restrict__ Ain,
+__global__ void __launch_bounds__(1024) jacobi_factor_kernel(const float* __restrict__ Ain,
                                                             float* __restrict__ F, int Rp,
                                                             int r_req, const int32_t* ng,
                                                             float scale, int32_t* r_out,
@@ -415,12 +415,12 @@ __global__ void __launch_bounds__(256) label_colscan_kernel(int32_t* __restrict_
     int32_t* hh = hist + (size_t)bh * n_tiles * C + c;
     int run = 0;
     int t = 0;
-    for (; t + 8 <= n_tiles; t += 8) {   // eight loads in flight
-        int v[8];
+    for (; t + 32 <= n_tiles; t += 32) {   // 32 loads in flight
+        int v[32];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = hh[(size_t)(t + u) * C];
+        for (int u = 0; u < 32; ++u) v[u] = hh[(size_t)(t + u) * C];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 32; ++u) {
             hh[(size_t)(t + u) * C] = run;
             run += v[u];
         }
@@ -792,7 +792,7 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
 
     // 1-2. key-response metric and factor (§4.1)
     count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff, mat);
-    count_launch(), jacobi<<<BH, 512, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d),
+    count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d),
                                                       nullptr, 16);
     project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
     // 3. paired K/V groups
@@ -810,7 +810,7 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), centroid_mean_kernel<<<BH, d, 0, st>>>(out.k_centroid, out.n_groups, pl.Ck, d, muK);
     count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
                                                                           out.n_groups, pl.Ck, d, mat);
-    count_launch(), jacobi<<<BH, 512, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16);
+    count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16);
     project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, at<DevStatus>(ws, pl.o_status), st);
     // 5. query groups
     kmeans_dispatch(pl.RQp, pl, p, ws, phiQ, pl.Cq, 1, cenQ, hnQ, dbg ? out.debug_q_scores : nullptr,
