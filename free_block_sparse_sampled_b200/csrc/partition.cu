@@ -112,11 +112,8 @@ __global__ void __launch_bounds__(1024) jacobi_factor_kernel(const float* __rest
     const int ld = d + 1, half = d / 2;
     float* A = sm;
     float* V = A + d * ld;
-    float* cs = V + d * ld;
-    float* sn = cs + half;
-    int* pp = reinterpret_cast<int*>(sn + half);
-    int* qq = pp + half;
-    float* red = reinterpret_cast<float*>(qq + half);   // 64 floats
+    float4* par = reinterpret_cast<float4*>(V + d * ld);   // per pair: c, s, p, q (int bits)
+    float* red = reinterpret_cast<float*>(par + half);      // 64 floats
     int* order = reinterpret_cast<int*>(red + 64);      // d ints
 
     const float* Ah = Ain + (size_t)bh * d * d;
@@ -184,31 +181,36 @@ __global__ void __launch_bounds__(1024) jacobi_factor_kernel(const float* __rest
                     c = 1.f / sqrtf(t * t + 1.f);
                     s = t * c;
                 }
-                cs[k] = c;
-                sn[k] = s;
-                pp[k] = p;
-                qq[k] = q;
+                par[k] = make_float4(c, s, __int_as_float(p), __int_as_float(q));
             }
             __syncthreads();
-            for (int e = tid; e < half * d; e += nt) {   // rows p, q of J^T A
-                const int k = e / d, j = e % d;
-                const int p = pp[k], q = qq[k];
-                const float c = cs[k], s = sn[k];
-                const float ap = A[p * ld + j], aq = A[q * ld + j];
-                A[p * ld + j] = c * ap - s * aq;
-                A[q * ld + j] = s * ap + c * aq;
-            }
-            __syncthreads();
-            for (int e = tid; e < half * d; e += nt) {   // columns p, q of (J^T A) J and V J
-                const int k = e / d, i = e % d;
-                const int p = pp[k], q = qq[k];
-                const float c = cs[k], s = sn[k];
-                const float ap = A[i * ld + p], aq = A[i * ld + q];
-                A[i * ld + p] = c * ap - s * aq;
-                A[i * ld + q] = s * ap + c * aq;
-                const float vp = V[i * ld + p], vq = V[i * ld + q];
-                V[i * ld + p] = c * vp - s * vq;
-                V[i * ld + q] = s * vp + c * vq;
+            // J^T A J in one pass: each thread owns whole 2 x 2 blocks (rows of
+            // pair P, columns of pair Q), rotating the rows and then the
+            // columns in registers; V J rotates the column pairs of V.  The
+            // thread's column pair Q is fixed (nt is a multiple of d / 2), so
+            // its rotation is read once.
+            {
+                const int Q = tid % half;
+                const float4 fQ = par[Q];
+                const int r = __float_as_int(fQ.z), t = __float_as_int(fQ.w);
+                const float cQ = fQ.x, sQ = fQ.y;
+                for (int P = tid / half; P < half; P += nt / half) {
+                    const float4 fP = par[P];
+                    const int p = __float_as_int(fP.z), q = __float_as_int(fP.w);
+                    const float cP = fP.x, sP = fP.y;
+                    const float apr = A[p * ld + r], apt = A[p * ld + t], aqr = A[q * ld + r], aqt = A[q * ld + t];
+                    const float bpr = cP * apr - sP * aqr, bpt = cP * apt - sP * aqt;   // rows p, q
+                    const float bqr = sP * apr + cP * aqr, bqt = sP * apt + cP * aqt;
+                    A[p * ld + r] = cQ * bpr - sQ * bpt;                                 // columns r, t
+                    A[p * ld + t] = sQ * bpr + cQ * bpt;
+                    A[q * ld + r] = cQ * bqr - sQ * bqt;
+                    A[q * ld + t] = sQ * bqr + cQ * bqt;
+                }
+                for (int i = tid / half; i < d; i += nt / half) {
+                    const float vr = V[i * ld + r], vt = V[i * ld + t];
+                    V[i * ld + r] = cQ * vr - sQ * vt;
+                    V[i * ld + t] = sQ * vr + cQ * vt;
+                }
             }
             __syncthreads();
         }
@@ -785,8 +787,7 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     int32_t* ctl = at<int32_t>(ws, pl.o_ctl);
     const bool dbg = (p.flags & SPARSEPR_FLAG_DEBUG_EXPORT) != 0;
 
-    const size_t jac_smem = (size_t)(2 * d * (d + 1) + 2 * (d / 2) + 64) * sizeof(float) +
-                            (size_t)(2 * (d / 2) + d) * sizeof(int);
+    const size_t jac_smem = (size_t)(2 * d * (d + 1) + 4 * (d / 2) + 64) * sizeof(float) + (size_t)d * sizeof(int);
     auto jacobi = (d == 128) ? jacobi_factor_kernel<128> : jacobi_factor_kernel<64>;
     cudaFuncSetAttribute(jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jac_smem);
 
