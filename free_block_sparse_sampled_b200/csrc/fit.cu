@@ -68,40 +68,49 @@ __global__ void fit_stats_kernel(const float* __restrict__ Xs, const float* __re
 }
 
 // Rows i0..i0+7 of G = Xbar^T W Xbar + lambda I and of RHS = Xbar^T W Rbar.
+// Probes are taken kGramChunk at a time: their weights times the block's
+// eight standardised rows are staged in shared memory, then each thread
+// accumulates its column j (probes in index order).
+constexpr int kGramChunk = 1024;
 __global__ void fit_gram_kernel(const float* __restrict__ Xs, const float* __restrict__ Xd,
                                 const int32_t* __restrict__ probe_group, const int32_t* __restrict__ alloc,
                                 const int32_t* __restrict__ q_off, const int32_t* __restrict__ psum, int Cq, int Mp,
                                 int d, double lambda, const double* __restrict__ fstat, double* __restrict__ G,
                                 double* __restrict__ rhs) {
     constexpr int RI = 8;
+    extern __shared__ double xbi[];   // [kGramChunk][RI] W_p * Xbar[p][i0 + u]
     const int bh = blockIdx.y, i0 = blockIdx.x * RI, j = threadIdx.x;
     const float* X = Xs + (size_t)bh * Mp * d;
-    const float* D = Xd + (size_t)bh * Mp * d;
+    const float* Dp = Xd + (size_t)bh * Mp * d;
     const int32_t* pg = probe_group + (size_t)bh * Mp;
     const int32_t* al = alloc + (size_t)bh * Cq;
     const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
     const double* fs = fstat + (size_t)bh * 3 * d;
     const double sw = (double)psum[bh];
     const double mxj = fs[j], sgj = fs[d + j], mrj = fs[2 * d + j];
-    double mxi[RI], sgi[RI];
-#pragma unroll
-    for (int u = 0; u < RI; ++u) {
-        mxi[u] = fs[i0 + u];
-        sgi[u] = fs[d + i0 + u];
-    }
     double g[RI], h[RI];
 #pragma unroll
     for (int u = 0; u < RI; ++u) g[u] = h[u] = 0.0;
-    for (int p = 0; p < Mp; ++p) {
-        const double wt = (double)Mp * probe_alpha(p, pg, al, qo, sw);
-        const double xj = (double)X[(size_t)p * d + j];
-        const double xbj = (xj - mxj) / sgj;
-        const double rbj = ((double)D[(size_t)p * d + j] - xj) - mrj;
+    for (int c0 = 0; c0 < Mp; c0 += kGramChunk) {
+        const int n = min(kGramChunk, Mp - c0);
+        __syncthreads();   // the previous chunk is consumed
+        for (int e = j; e < n * RI; e += blockDim.x) {
+            const int p = c0 + e / RI, u = e % RI;
+            const double wt = (double)Mp * probe_alpha(p, pg, al, qo, sw);
+            xbi[e] = wt * (((double)X[(size_t)p * d + i0 + u] - fs[i0 + u]) / fs[d + i0 + u]);
+        }
+        __syncthreads();
+        for (int q = 0; q < n; ++q) {
+            const int p = c0 + q;
+            const double xj = (double)X[(size_t)p * d + j];
+            const double xbj = (xj - mxj) / sgj;
+            const double rbj = ((double)Dp[(size_t)p * d + j] - xj) - mrj;
 #pragma unroll
-        for (int u = 0; u < RI; ++u) {
-            const double xbi = wt * (((double)X[(size_t)p * d + i0 + u] - mxi[u]) / sgi[u]);
-            g[u] += xbi * xbj;
-            h[u] += xbi * rbj;
+            for (int u = 0; u < RI; ++u) {
+                const double xb = xbi[q * RI + u];
+                g[u] += xb * xbj;
+                h[u] += xb * rbj;
+            }
         }
     }
 #pragma unroll
@@ -266,8 +275,11 @@ sparsepr_status run_fit(const sparsepr_params& p, const Plan& pl, const sparsepr
     count_launch(), fit_stats_kernel<<<BH, d, 0, st>>>(probe_sparse, probe_dense, r.probe_group, alloc, part.q_offsets,
                                        part.n_groups, psum, pl.Cq, Mp, d, p.eps_std, fstat, f.mu_x, f.sigma,
                                        f.mu_r);
-    count_launch(), fit_gram_kernel<<<dim3(d / 8, BH), d, 0, st>>>(probe_sparse, probe_dense, r.probe_group, alloc, part.q_offsets,
-                                                   psum, pl.Cq, Mp, d, p.lambda, fstat, G, rhs);
+    const size_t gsmem = (size_t)kGramChunk * 8 * sizeof(double);   // 8 staged rows per probe of a chunk
+    cudaFuncSetAttribute(fit_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem);
+    count_launch(), fit_gram_kernel<<<dim3(d / 8, BH), d, gsmem, st>>>(probe_sparse, probe_dense, r.probe_group, alloc,
+                                                                       part.q_offsets, psum, pl.Cq, Mp, d, p.lambda,
+                                                                       fstat, G, rhs);
     const size_t smem = (size_t)d * (d + 1) * sizeof(double);
     cudaFuncSetAttribute(fit_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     count_launch(), fit_solve_kernel<<<BH, d, smem, st>>>(G, rhs, d, f.B, status);
