@@ -332,27 +332,38 @@ def run_ours(args, w):
     pairs_exec, pairs_route = int(br[0]["pairs_exec"]), int(br[0]["pairs_route"])
     launches = int(br[0]["launches"])
 
-    # dominant kernel: the attention stage alone (staged API), CUDA events on its stream
+    # Dominant kernel: the attention stage.  Its time inside a whole call comes
+    # from the library's own CUDA events on the call's stream (the breakdown
+    # calls above, run right after the timed region, whose clocks stayed at
+    # their maximum: hence the burst peak).  The staged API is timed alone as a
+    # cross-check, with the clocks sampled over that loop: back-to-back
+    # attention launches can reach the power cap.
     part = S.partition(cfg, q, k, v, ws)
     rt = S.route(cfg, part, ws)
     for _ in range(2):
         S.attention(cfg, part, rt, ws)
     torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_attn = max(3, args.steps)
+    n_attn = 3
+    clk_a = ClockSampler(local)
+    clk_a.start()
     a0.record()
     for _ in range(n_attn):
         O_sp, pd, ps = S.attention(cfg, part, rt, ws)
     a1.record()
     torch.cuda.synchronize()
-    ms_attn = a0.elapsed_time(a1) / n_attn
+    clocks_attn = clk_a.stop()
+    ms_attn_alone = a0.elapsed_time(a1) / n_attn
+    ms_attn = st["ms_attention"]
     attn_flops = 4.0 * cfg.d * pairs_exec          # QK^T and PV on every executed pair
     peaks, peak_kind = measured_peaks()
     achieved = attn_flops / (ms_attn * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic(w),
                 "kernel": "attention_tc_kernel<128> (+ work list and probe gathers)",
-                "peak_source": f"{peak_kind} bf16 dense (burst)"}
+                "peak_source": f"{peak_kind} bf16 dense (burst)",
+                "duration_ms": ms_attn, "duration_source": "attention stage of whole calls (library CUDA events on the call's stream)",
+                "staged_alone_ms": ms_attn_alone, "staged_alone_clocks": clocks_attn}
 
     extras = {}
     if not args.quick:
@@ -391,29 +402,28 @@ def run_ours(args, w):
                                      "rows": "2048 evenly spaced rows per head, probes excluded"}
     e2e = None
     if not args.no_e2e and not args.quick:
+        # End to end from pinned host memory through the package's HostPipeline:
+        # every call copies its inputs in and its output out; the copies of
+        # neighbouring calls overlap the current call's compute.
         hq = [t.cpu().pin_memory() for t in (q, k, v)]
-        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        dq = [torch.empty_like(t) for t in (q, k, v)]
-        for _ in range(2):
-            for dst, src in zip(dq, hq):
-                dst.copy_(src, non_blocking=True)
-            S.call(cfg, *dq, ws, out)
-            hout.copy_(out, non_blocking=True)
-        torch.cuda.synchronize()
+        n_e2e = max(3, args.steps)
+        houts = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+        pipe = S.HostPipeline(cfg, dev)
+        pipe.run([hq] * 2, houts)                        # warm-up
+        same = bool(torch.equal(houts[1][0, 0], out[0, 0].cpu()))
         barrier()
         h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_e2e = max(3, min(args.steps, 5))
         h0.record()
-        for _ in range(n_e2e):
-            for dst, src in zip(dq, hq):
-                dst.copy_(src, non_blocking=True)
-            S.call(cfg, *dq, ws, out)
-            hout.copy_(out, non_blocking=True)
+        pipe.run([hq] * n_e2e, [houts[i & 1] for i in range(n_e2e)])
         h1.record()
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(h0.elapsed_time(h1) / n_e2e)
-        e2e = {"value": whole_job_ms_per_call(e2e_ms, world), "unit": "ms/call", "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in hq)),
-               "d2h_bytes_per_step": int(hout.numel() * hout.element_size())}
+        e2e = {"value": whole_job_ms_per_call(e2e_ms, world), "unit": "ms/call",
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in hq)),
+               "d2h_bytes_per_step": int(houts[0].numel() * houts[0].element_size()),
+               "calls": n_e2e, "pipeline": "copies of neighbouring calls overlap compute (HostPipeline)",
+               "output_matches_device_call": same}
+        del pipe
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -4,6 +4,6 @@ The library (libsparsepr.so, built from csrc/ by ``build.py``) implements the
 whole call in CUDA; this package only marshals arguments.
 """
 
-from .api import (SparsePRConfig, alloc_workspace, apply, attention, call, device_status,  # noqa: F401
+from .api import (HostPipeline, SparsePRConfig, alloc_workspace, apply, attention, call, device_status,  # noqa: F401
                   partition, probe_fit, probe_fit_static, route, validate, workspace_bytes)
 from ._abi import EXPORTED, LIB_PATH, SparsePRError, lib  # noqa: F401

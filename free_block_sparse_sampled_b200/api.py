@@ -247,3 +247,54 @@ def device_status(ws: torch.Tensor) -> int:
     v = ctypes.c_int32(0)
     A.check("sparsepr_get_device_status", A.lib().sparsepr_get_device_status(_p(ws), _stream(), ctypes.byref(v)))
     return int(v.value)
+
+
+class HostPipeline:
+    """A sequence of calls whose inputs and outputs live in pinned host memory.
+
+    The inputs of call i + 1 are copied to the device on one stream while call
+    i runs on another, and the output of call i is copied back on a third, so
+    host<->device traffic overlaps compute.  Device inputs and outputs are
+    double-buffered; one workspace serves every call (calls run in order on
+    the compute stream)."""
+
+    def __init__(self, cfg: SparsePRConfig, device="cuda"):
+        self.cfg = cfg
+        dev = torch.device(device)
+        shape = (cfg.B, cfg.H, cfg.N, cfg.d)
+        self.din = [[torch.empty(shape, dtype=cfg.torch_dtype, device=dev) for _ in range(3)] for _ in range(2)]
+        self.dout = [torch.empty(shape, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.ws = alloc_workspace(cfg, dev)
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]
+        self.in_ready, self.in_free, self.out_ready, self.out_free = ev(), ev(), ev(), ev()
+
+    def run(self, inputs, outputs) -> None:
+        """inputs: sequence of (q, k, v) pinned host tensors [B, H, N, d] in the
+        call's dtype; outputs: matching pinned fp32 host tensors.  Returns once
+        every output is on the host."""
+        cur = torch.cuda.current_stream()
+        for s in (self.s_in, self.s_run, self.s_out):
+            s.wait_stream(cur)
+        for i, ((hq, hk, hv), hout) in enumerate(zip(inputs, outputs)):
+            b = i & 1
+            with torch.cuda.stream(self.s_in):
+                if i >= 2:
+                    self.s_in.wait_event(self.in_free[b])      # call i - 2 no longer reads this buffer
+                for dst, src in zip(self.din[b], (hq, hk, hv)):
+                    dst.copy_(src, non_blocking=True)
+                self.in_ready[b].record(self.s_in)
+            with torch.cuda.stream(self.s_run):
+                self.s_run.wait_event(self.in_ready[b])
+                if i >= 2:
+                    self.s_run.wait_event(self.out_free[b])    # call i - 2's output has left this buffer
+                call(self.cfg, *self.din[b], self.ws, self.dout[b])
+                self.in_free[b].record(self.s_run)
+                self.out_ready[b].record(self.s_run)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.out_ready[b])
+                hout.copy_(self.dout[b], non_blocking=True)
+                self.out_free[b].record(self.s_out)
+        for s in (self.s_in, self.s_run, self.s_out):
+            cur.wait_stream(s)
+        torch.cuda.synchronize()

@@ -167,3 +167,21 @@ def test_mid_call_every_head():
                                    v[0, bh].astype(np.float64))
         check_attention(hv, cfg, TOL_ATTN)
         check_fit_and_apply(hv, cfg)
+
+
+def test_host_pipeline_matches_device_call():
+    """HostPipeline (host buffers, copies overlapped with compute) returns
+    exactly what sparsepr_call returns on device-resident inputs."""
+    import free_block_sparse_sampled_b200 as S
+    w = SMALL["bf16_d128"]
+    cfg = _cfg(w)
+    q, k, v = generate_inputs(w)
+    dq, dk, dv = to_device(w, (q, k, v))
+    ws = S.alloc_workspace(cfg)
+    ref, _ = S.call(cfg, dq, dk, dv, ws)
+    torch.cuda.synchronize()
+    hin = [t.cpu().pin_memory() for t in (dq, dk, dv)]
+    outs = [torch.empty(ref.shape, dtype=torch.float32, pin_memory=True) for _ in range(3)]
+    S.HostPipeline(cfg).run([hin] * 3, outs)
+    for o in outs:
+        assert torch.equal(o, ref.cpu())
