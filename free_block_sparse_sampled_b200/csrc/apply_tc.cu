@@ -178,7 +178,8 @@ __global__ void __maxnreg__(168) apply_tc_kernel(
                 float acc[2][32];
                 tmem_ld32(t_row + d * D + 64 * hh, acc[0]);
                 tmem_ld32(t_row + d * D + 64 * hh + 32, acc[1]);
-                tmem_wait_ld();
+                tmem_wait_ld(acc[0]);
+                tmem_wait_ld(acc[1]);
                 if (live && slot < 0) {
                     const float4* x = reinterpret_cast<const float4*>(O_sp + src * D) + 16 * hh;
                     const float4* mr = reinterpret_cast<const float4*>(mu_r + (size_t)bh * D) + 16 * hh;

@@ -644,7 +644,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         float v[32];
                         tmem_ld32(tO + c4 * 32, v);
-                        tmem_wait_ld();
+                        tmem_wait_ld(v);
     #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] *= alpha;
                         tmem_st32(tO + c4 * 32, v);
@@ -695,7 +695,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         float v[32];
                         tmem_ld32(tO + c4 * 32, v);
-                        tmem_wait_ld();
+                        tmem_wait_ld(v);
                         if (r < nrows) {
                             float4* o4 = reinterpret_cast<float4*>(out + c4 * 32);
     #pragma unroll

@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                     float v[2][32];
                     tmem_ld32(t_row + db * NB + half * hw + c0, v[0]);
                     if (two) tmem_ld32(t_row + db * NB + half * hw + c0 + 32, v[1]);
-                    tmem_wait_ld();
+                    tmem_wait_ld(v[0]);
+                    if (two) tmem_wait_ld(v[1]);
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         if (q == 1 && !two) break;

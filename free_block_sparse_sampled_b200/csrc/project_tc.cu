@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(prtc::kThreads, 1) project_tc_kernel(
             for (int c = 0; c < R; c += 16) {
                 float v[16];
                 tmem_ld16(t_row + d * (kCols / 2) + c, v);
-                tmem_wait_ld();
+                tmem_wait_ld(v);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) acc[c + u] = v[u];
             }

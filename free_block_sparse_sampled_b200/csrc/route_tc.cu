@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
             for (int c4 = 0; c4 < BK / 32; ++c4) {
                 float v[32];
                 tmem_ld32(t_row + stage * BK + c4 * 32, v);
-                tmem_wait_ld();
+                tmem_wait_ld(v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     if (c4 * 32 + i < ncol) m4[i & 3] = fmaxf(m4[i & 3], v[i] * cs);
