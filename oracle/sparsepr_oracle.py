@@ -38,6 +38,24 @@ R7  Probe allocation (lost in the extraction of A.2): largest remainder on
     the m_a rows with smallest (d_i, i); every row when M >= N_q.
 R8  Residual-span projection at full rank is the identity because every row
     of B_lambda lies in the row space of R-bar (§4.2; C.1 default uses none).
+R13 Warm start, metric factors (paper C.1: "two subspace iterations
+    initialized from the previous factors and using Cholesky factorization"):
+    Q_0 = the previous factor; twice  Y = M Q,  Y^T Y = L L^T,  Q = Y L^-T
+    (Cholesky QR); then F = Q C with C C^T = Q^T M Q (Cholesky), times
+    1/sqrt(d) for the key factor (R2).  F F^T = Q Q^T M Q Q^T, the metric
+    restricted to the iterated subspace; at an exact eigenbasis it equals the
+    cold factor's F F^T.  The page does not say what happens when the previous
+    factor has fewer columns than the current rank or a Cholesky pivot
+    vanishes; then the call takes the cold factor (eigendecomposition).  A
+    pivot "vanishes" when its square is not above 1e-12 times the largest
+    diagonal entry of the matrix being factored.
+R14 Warm start, centres (paper C.1: "previous centroids in the original space
+    projected into the current response coordinates"): centre b of the key
+    k-means is kbar_b F_K, centre a of the query k-means is RMSNorm(qbar_a F_Q),
+    for the previous call's nonempty groups; centres past their count are
+    drawn as in a cold start (R3).
+R15 Later calls run at most 2 k-means assignments (Table C.1, "initial /
+    subsequent k means iteration limits 25/2"); the caller passes the limit.
 """
 
 from __future__ import annotations
@@ -178,11 +196,12 @@ def kmeans_stop_count(tol: float, N: int) -> int:
     return int(math.floor(tol * N))
 
 
-def kmeans(X: np.ndarray, init_idx: np.ndarray, max_iter: int, stop_changed: int):
+def kmeans(X: np.ndarray, init_idx: np.ndarray, max_iter: int, stop_changed: int,
+           init_centres: Optional[np.ndarray] = None):
     """Lloyd k-means (§4.1, C.1, Table C.1) under reading R3.  Returns
     (labels, centres used by the last assignment, number of assignments,
-    label history)."""
-    centres = X[init_idx].copy()
+    label history).  ``init_centres`` replaces the sampled rows (R14)."""
+    centres = (X[init_idx] if init_centres is None else init_centres).copy()
     labels, _ = kmeans_assign(X, centres)
     history = [labels]
     n_assign = 1
@@ -196,6 +215,55 @@ def kmeans(X: np.ndarray, init_idx: np.ndarray, max_iter: int, stop_changed: int
         if changed <= stop_changed:
             break
     return labels, centres, n_assign, history
+
+
+WARM_PIVOT_REL = 1e-12
+
+
+def cholesky_checked(G: np.ndarray) -> Optional[np.ndarray]:
+    """Lower Cholesky factor of G, or None when a pivot vanishes (R13)."""
+    try:
+        L = np.linalg.cholesky(G)
+    except np.linalg.LinAlgError:
+        return None
+    if not np.all(np.diag(L) ** 2 > WARM_PIVOT_REL * np.max(np.diag(G))):
+        return None
+    return L
+
+
+def warm_factor(M: np.ndarray, F_prev: np.ndarray, r: int, scale: float,
+                iters: int = 2) -> Optional[np.ndarray]:
+    """R13: subspace iteration from the previous factor with Cholesky QR, then
+    the metric's Cholesky factor on the iterated subspace; d x r, or None
+    when the cold factor must be used instead."""
+    if F_prev.shape[1] < r:
+        return None
+    Q = F_prev[:, :r].copy()
+    for _ in range(iters):
+        Y = M @ Q
+        L = cholesky_checked(Y.T @ Y)
+        if L is None:
+            return None
+        Q = np.linalg.solve(L, Y.T).T          # Y L^-T
+    C = cholesky_checked(Q.T @ M @ Q)
+    if C is None:
+        return None
+    return (Q @ C) * scale
+
+
+def warm_centres(Y: np.ndarray, cbar_prev: np.ndarray, F: np.ndarray, C: int, init_idx: np.ndarray,
+                 rms_eps: Optional[float] = None) -> np.ndarray:
+    """R14: previous centroids (original space) projected into the current
+    coordinates, RMS-normalised for the query side; the remaining centres are
+    the cold start's rows of Y (the current coordinates)."""
+    centres = Y[init_idx].copy()
+    n = min(C, cbar_prev.shape[0])
+    z = cbar_prev[:n] @ F
+    if rms_eps is not None:
+        rms = np.sqrt((z * z).sum(axis=1) / F.shape[1])
+        z = z / np.maximum(rms, rms_eps)[:, None]
+    centres[:n] = z
+    return centres
 
 
 def compact_labels(labels: np.ndarray, C: int):
@@ -417,10 +485,12 @@ def error_reduction(mean_err_method: float, mean_err_base: float) -> float:
 def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: int,
                   lam: float, Cq: int, Ck: int, rK: int, rQ: int, kmeans_iters: int,
                   kmeans_tol: float, eps_rms: float = 1e-6, eps_std: float = 1e-6,
-                  want_dense: bool = False) -> Dict[str, object]:
+                  want_dense: bool = False, warm: Optional[Dict[str, np.ndarray]] = None) -> Dict[str, object]:
     """One SparsePR call on one head, steps in the paper's order:
     partition (§4.1) -> route (§4.3, B.3) -> sparse attention (Eq. 2) ->
-    probes (A.2) -> weighted ridge (A.3) -> corrected output (§4.2)."""
+    probes (A.2) -> weighted ridge (A.3) -> corrected output (§4.2).
+    ``warm`` (F_K, F_Q, kbar, qbar of the previous call) selects the warm
+    start of R13-R15; the caller also lowers ``kmeans_iters``."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -430,23 +500,32 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     # 1-2. key-response metric and factor
     idx = sample_indices(N, Ms)
     M_K = key_metric(q, idx)
-    F_K = key_factor(M_K, rK, len(idx))
+    r_k = min(rK, d, len(idx))
+    F_K = None if warm is None else warm_factor(M_K, warm["F_K"], r_k, 1.0 / math.sqrt(d))
+    warm_K = F_K is not None
+    if F_K is None:
+        F_K = key_factor(M_K, rK, len(idx))
     phi_K = k @ F_K
     # 3. paired K/V groups
     init_k = kmeans_init_indices(seed, bh, 0, Ck, N)
     stop = kmeans_stop_count(kmeans_tol, N)
-    kv_raw, _, it_k, _ = kmeans(phi_K, init_k, kmeans_iters, stop)
+    cen_k = None if warm is None else warm_centres(phi_K, warm["kbar"], F_K, Ck, init_k)
+    kv_raw, _, it_k, _ = kmeans(phi_K, init_k, kmeans_iters, stop, cen_k)
     kv_labels, Ck2, kv_sizes = compact_labels(kv_raw, Ck)
     # 4. centroids, query metric and factor
     kbar = group_means(k, kv_labels, Ck2)
     vbar = group_means(v, kv_labels, Ck2)
     M_Q = query_metric(kbar)
     rq = query_rank(rQ, d, Ck2)
-    F_Q = query_factor(M_Q, rq)
+    F_Q = None if warm is None else warm_factor(M_Q, warm["F_Q"], rq, 1.0)
+    warm_Q = F_Q is not None
+    if F_Q is None:
+        F_Q = query_factor(M_Q, rq)
     phi_Q = query_coords(q, F_Q, eps_rms)
     # 5. query groups
     init_q = kmeans_init_indices(seed, bh, 1, Cq, N)
-    q_raw, _, it_q, _ = kmeans(phi_Q, init_q, kmeans_iters, stop)
+    cen_q = None if warm is None else warm_centres(phi_Q, warm["qbar"], F_Q, Cq, init_q, eps_rms)
+    q_raw, _, it_q, _ = kmeans(phi_Q, init_q, kmeans_iters, stop, cen_q)
     q_labels, Cq2, q_sizes = compact_labels(q_raw, Cq)
     qbar = group_means(q, q_labels, Cq2)
     _, d_i = query_distances(phi_Q, q_labels, Cq2)
@@ -476,10 +555,16 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
                pairs_route=p_route, pairs_exec=executed_pairs(p_route, Mp, N),
                perm_q=perm_q, q_offsets=q_off, perm_k=perm_k, k_offsets=k_off,
                O_sp=O_sp, m=m, probes=P, w=w, alpha=alpha, wt=wt, O_dense_probes=O_dense_P,
-               fit=fit, O=O_hat)
+               fit=fit, O=O_hat, warm_factor_used=(warm is not None and warm_K, warm is not None and warm_Q))
     if want_dense:
         out["O_dense"] = dense_attention(q, k, v)
     return out
+
+
+def warm_state(out: Dict[str, object]) -> Dict[str, np.ndarray]:
+    """The state a later call starts from (R13, R14): the metric factors and
+    the raw-space centroids of the nonempty groups of ``out``."""
+    return dict(F_K=out["F_K"], F_Q=out["F_Q"], kbar=out["kbar"], qbar=out["qbar"])
 
 
 def workload_kwargs(w) -> Dict[str, object]:

@@ -502,3 +502,130 @@ def test_whole_call_all_rows_probes_is_exact():
     kw["M"] = w.N
     r = O.sparsepr_head(q, k, v, bh=0, want_dense=True, **kw)
     np.testing.assert_array_equal(r["O"], r["O_dense"])
+
+
+# ------------------------------------------------------------- warm start (C.1)
+def _spd(d, seed, gap=None):
+    """Symmetric positive definite d x d matrix; with ``gap`` its spectrum is
+    geometric with that ratio between neighbours."""
+    U, _ = np.linalg.qr(_rand((d, d), seed))
+    w = (gap ** -np.arange(d)) if gap else np.exp(_rand(d, seed + 1))
+    return U @ np.diag(w) @ U.T
+
+
+@pytest.mark.parametrize("scale", [1.0, 1.0 / math.sqrt(8)])
+def test_warm_factor_from_exact_eigenbasis_is_cold_factor(scale):
+    """Started from the cold factor of the same metric, the subspace iteration
+    stays on the leading eigenspace, so F F^T is the truncated metric."""
+    d, r = 8, 3
+    M = _spd(d, 60)
+    w, U = O.eigh_desc(M)
+    F0 = U[:, :r] * np.sqrt(w[:r])           # spans the leading eigenspace, not orthonormal
+    F = O.warm_factor(M, F0, r, scale)
+    want = U[:, :r] @ np.diag(w[:r]) @ U[:, :r].T * scale * scale
+    np.testing.assert_allclose(F @ F.T, want, atol=1e-12 * np.abs(want).max())
+
+
+def test_warm_factor_is_projected_metric_of_iterated_subspace():
+    """Independent route: F F^T = P M P with P the orthogonal projector on
+    span(M^2 F_prev), built by Householder QR."""
+    d, r = 10, 4
+    M = _spd(d, 61)
+    F0 = _rand((d, r), 62)
+    F = O.warm_factor(M, F0, r, 0.5, iters=2)
+    Qh, _ = np.linalg.qr(M @ M @ F0)
+    P = Qh @ Qh.T
+    np.testing.assert_allclose(F @ F.T, 0.25 * P @ M @ P, atol=1e-11 * np.abs(M).max())
+    # one iteration: projector on span(M F_prev)
+    F1 = O.warm_factor(M, F0, r, 1.0, iters=1)
+    Q1, _ = np.linalg.qr(M @ F0)
+    np.testing.assert_allclose(F1 @ F1.T, Q1 @ Q1.T @ M @ Q1 @ Q1.T, atol=1e-11 * np.abs(M).max())
+
+
+def test_warm_factor_exact_on_metric_of_rank_r():
+    d, r = 9, 3
+    A = _rand((r, d), 63)
+    M = A.T @ A
+    F = O.warm_factor(M, _rand((d, r), 64), r, 1.0, iters=1)
+    np.testing.assert_allclose(F @ F.T, M, atol=1e-10 * np.abs(M).max())
+
+
+def test_warm_factor_converges_to_cold_factor():
+    d, r = 12, 4
+    M = _spd(d, 65, gap=1.6)
+    w, U = O.eigh_desc(M)
+    want = U[:, :r] @ np.diag(w[:r]) @ U[:, :r].T
+    errs = []
+    for it in (1, 2, 8, 80):
+        F = O.warm_factor(M, _rand((d, r), 66), r, 1.0, iters=it)
+        errs.append(np.abs(F @ F.T - want).max())
+    assert errs[0] > errs[1] > errs[2] > errs[3]
+    assert errs[3] < 1e-10 * w[0]
+
+
+def test_warm_factor_falls_back_to_cold():
+    d = 6
+    M = _spd(d, 67)
+    assert O.warm_factor(M, _rand((d, 2), 68), 3, 1.0) is None          # fewer columns than the rank
+    F0 = _rand((d, 3), 69)
+    F0[:, 1] = 0.0                                                        # a vanishing pivot
+    assert O.warm_factor(M, F0, 3, 1.0) is None
+    assert O.cholesky_checked(np.diag([4.0, 1e-13])) is None
+    np.testing.assert_allclose(O.cholesky_checked(np.diag([4.0, 1.0])), np.diag([2.0, 1.0]))
+
+
+def test_warm_centres_projection_and_rmsnorm():
+    N, d, r, C = 40, 5, 3, 6
+    Y = _rand((N, r), 70)
+    cbar = _rand((4, d), 71)
+    F = _rand((d, r), 72)
+    init = O.kmeans_init_indices(3, 0, 0, C, N)
+    cen = O.warm_centres(Y, cbar, F, C, init)
+    for b in range(4):
+        for j in range(r):
+            assert abs(cen[b, j] - sum(cbar[b, t] * F[t, j] for t in range(d))) < 1e-12
+    np.testing.assert_array_equal(cen[4:], Y[init[4:]])
+    # query side: a group of identical rows has its coordinate as the centre
+    q = np.repeat(_rand((3, d), 73), [5, 7, 4], axis=0)
+    labels = np.repeat(np.arange(3), [5, 7, 4])
+    phi = O.query_coords(q, F, 1e-6)
+    qbar = O.group_means(q, labels, 3)
+    cq = O.warm_centres(phi, qbar, F, 3, np.zeros(3, np.int64), rms_eps=1e-6)
+    np.testing.assert_allclose(cq, O.group_means(phi, labels, 3), atol=1e-12)
+    # RMS floor: a zero centroid stays zero
+    cz = O.warm_centres(phi, np.zeros((1, d)), F, 3, np.zeros(3, np.int64), rms_eps=1e-6)
+    assert np.all(cz[0] == 0.0)
+
+
+def test_warm_start_from_converged_keys_is_a_fixed_point():
+    """Converged K/V groups are reproduced by one warm assignment: the
+    projected previous centroids are the converged centres (phi_K is linear)."""
+    rng = np.random.default_rng(74)
+    N, d, C = 240, 6, 5
+    k = np.repeat(rng.standard_normal((C, d)) * 4, N // C, axis=0) + rng.standard_normal((N, d)) * 0.3
+    q = rng.standard_normal((N, d))
+    F = O.key_factor(O.key_metric(q, O.sample_indices(N, 64)), 4, 64)
+    init = O.kmeans_init_indices(5, 0, 0, C, N)
+    lab, _, _, _ = O.kmeans(k @ F, init, 200, 0)
+    lab_c, C2, _ = O.compact_labels(lab, C)
+    assert C2 == C
+    kbar = O.group_means(k, lab_c, C2)
+    cen = O.warm_centres(k @ F, kbar, F, C, init)
+    lab_w, _, n_it, _ = O.kmeans(k @ F, init, 2, 0, cen)
+    assert np.array_equal(O.compact_labels(lab_w, C)[0], lab_c)
+    assert n_it == 2                       # the second assignment changes nothing
+
+
+def test_warm_call_on_same_input_keeps_converged_kv_groups():
+    w, q, k, v = _tiny_head()
+    kw = O.workload_kwargs(w)
+    kw.update(kmeans_iters=200, kmeans_tol=0.0)
+    cold = O.sparsepr_head(q, k, v, bh=0, **kw)
+    kw["kmeans_iters"] = 2
+    warm = O.sparsepr_head(q, k, v, bh=0, warm=O.warm_state(cold), **kw)
+    assert warm["warm_factor_used"] == (True, True)
+    np.testing.assert_allclose(warm["F_K"] @ warm["F_K"].T, cold["F_K"] @ cold["F_K"].T,
+                               atol=1e-9 * np.abs(cold["F_K"]).max() ** 2)
+    assert np.array_equal(warm["kv_labels"], cold["kv_labels"])
+    assert warm["kmeans_iters_k"] <= 2 and warm["kmeans_iters_q"] <= 2
+    assert warm["pairs_exec"] / w.N / w.N >= w.density - 1e-12
