@@ -400,6 +400,32 @@ def run_ours(args, w):
                                      "mean_before_correction": float(esp.mean()),
                                      "p99_before_correction": float(torch.quantile(esp, 0.99)),
                                      "rows": "2048 evenly spaced rows per head, probes excluded"}
+        # Later calls of a denoising loop: warm start from the state the previous
+        # call left in the workspace, 2 k-means assignments (paper C.1, Table C.1).
+        import dataclasses
+        from free_block_sparse_sampled_b200 import _abi
+        wcfg = dataclasses.replace(cfg, kmeans_iters=2, flags=cfg.flags | _abi.FLAG_WARM_START)
+        S.call(cfg, q, k, v, ws, out)
+        for _ in range(2):
+            S.call(wcfg, q, k, v, ws, out)
+        torch.cuda.synchronize()
+        w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0.record()
+        for _ in range(3):
+            S.call(wcfg, q, k, v, ws, out)
+        w1.record()
+        torch.cuda.synchronize()
+        ms_warm = w0.elapsed_time(w1) / 3
+        _, wst = S.call(wcfg, q, k, v, ws, out, stats=True)
+        errw = (out[:, :, rows] - ref).norm(dim=-1) / (ref.norm(dim=-1) + 1e-8)
+        extras["warm_call"] = {
+            "ms_per_call": ms_warm, "speedup_vs_dense_sdpa": ms_dense / ms_warm,
+            "breakdown_ms": {k_: wst[k_] for k_ in ("ms_partition", "ms_route", "ms_attention", "ms_fit",
+                                                     "ms_apply", "ms_total")},
+            "rel_l2_unprobed_mean": float(errw[keep].double().mean()), "kmeans_iters": 2,
+            "device_status": S.device_status(ws),
+            "inputs": "the same Q/K/V as the cold call; the state is the previous call's"}
+        S.call(cfg, q, k, v, ws, out)                   # the cold call's output again
     e2e = None
     if not args.no_e2e and not args.quick:
         # End to end from pinned host memory through the package's HostPipeline:

@@ -13,11 +13,12 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE_TOO_S
 BF16, F32 = 0, 1
 FLAG_DEBUG_EXPORT = 1
 FLAG_SIMT_ATTENTION = 2
+FLAG_WARM_START = 4
 
 EXPORTED = ["sparsepr_status_string", "sparsepr_validate", "sparsepr_workspace_size",
             "sparsepr_partition", "sparsepr_route", "sparsepr_attention", "sparsepr_probe_fit",
             "sparsepr_apply", "sparsepr_call", "sparsepr_last_error_string", "sparsepr_get_device_status",
-            "sparsepr_probe_fit_static"]
+            "sparsepr_probe_fit_static", "sparsepr_partition_warm"]
 
 # size of the static scratch array behind sparsepr_probe_fit_static
 FIT_STATIC_SCRATCH_BYTES = 8 << 20
@@ -47,6 +48,13 @@ FIT_FIELDS = ["B", "mu_x", "sigma", "mu_r"]
 
 class PartitionOut(ctypes.Structure):
     _fields_ = [(n, P) for n in PARTITION_FIELDS]
+
+
+WARM_FIELDS = ["F_K", "F_Q", "k_centroid", "q_centroid", "n_groups"]
+
+
+class WarmState(ctypes.Structure):
+    _fields_ = [(n, P) for n in WARM_FIELDS]
 
 
 class RouteOut(ctypes.Structure):
@@ -86,6 +94,9 @@ def lib() -> ctypes.CDLL:
         L.sparsepr_partition.restype = ctypes.c_int32
         L.sparsepr_partition.argtypes = [ctypes.POINTER(Params), P, P, P, ctypes.POINTER(PartitionOut), P,
                                          ctypes.c_size_t, P]
+        L.sparsepr_partition_warm.restype = ctypes.c_int32
+        L.sparsepr_partition_warm.argtypes = [ctypes.POINTER(Params), P, P, P, ctypes.POINTER(WarmState),
+                                              ctypes.POINTER(PartitionOut), P, ctypes.c_size_t, P]
         L.sparsepr_route.restype = ctypes.c_int32
         L.sparsepr_route.argtypes = [ctypes.POINTER(Params), ctypes.POINTER(PartitionOut),
                                      ctypes.POINTER(RouteOut), P, ctypes.c_size_t, P]

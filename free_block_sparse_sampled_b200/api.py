@@ -116,8 +116,10 @@ def _check_qkv(cfg: SparsePRConfig, *ts: torch.Tensor) -> None:
 
 
 def partition(cfg: SparsePRConfig, q, k, v, ws: torch.Tensor, debug: bool = False,
-              extras: bool = False) -> Dict[str, torch.Tensor]:
-    """sparsepr_partition: returns the outputs as tensors (per-head slices contiguous)."""
+              extras: bool = False, warm: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+    """sparsepr_partition (or sparsepr_partition_warm when ``warm`` holds the
+    F_K, F_Q, k_centroid, q_centroid and n_groups of an earlier partition of
+    the same config): returns the outputs as tensors (per-head slices contiguous)."""
     _check_qkv(cfg, q, k, v)
     dev = q.device
     BH, N, d, Cq, Ck = cfg.BH, cfg.N, cfg.d, cfg.Cq, cfg.Ck
@@ -147,8 +149,22 @@ def partition(cfg: SparsePRConfig, q, k, v, ws: torch.Tensor, debug: bool = Fals
                   "debug_q_hist": torch.full((BH, cfg.kmeans_iters, N), -1, **i32)})
     s = A.PartitionOut(*[_p(o.get(n)) for n in A.PARTITION_FIELDS])
     p = c.c_params()
-    A.check("sparsepr_partition", A.lib().sparsepr_partition(ctypes.byref(p), _p(q), _p(k), _p(v), ctypes.byref(s),
-                                                             _p(ws), ws.numel(), _stream()))
+    if warm is None:
+        A.check("sparsepr_partition", A.lib().sparsepr_partition(ctypes.byref(p), _p(q), _p(k), _p(v),
+                                                                 ctypes.byref(s), _p(ws), ws.numel(), _stream()))
+    else:
+        shapes = {"F_K": (BH, d, cfg.RKp), "F_Q": (BH, d, cfg.RQp), "k_centroid": (BH, Ck, d),
+                  "q_centroid": (BH, Cq, d), "n_groups": (BH, 2)}
+        for n, shp in shapes.items():
+            t = warm[n]
+            want = torch.int32 if n == "n_groups" else torch.float32
+            if not (t.is_cuda and t.is_contiguous() and t.dtype == want and tuple(t.shape) == shp):
+                raise ValueError(f"warm[{n!r}] must be a contiguous CUDA {want} tensor of shape {shp}")
+        ws_state = A.WarmState(*[_p(warm[n]) for n in A.WARM_FIELDS])
+        A.check("sparsepr_partition_warm", A.lib().sparsepr_partition_warm(
+            ctypes.byref(p), _p(q), _p(k), _p(v), ctypes.byref(ws_state), ctypes.byref(s), _p(ws), ws.numel(),
+            _stream()))
+        o["_warm_struct"] = ws_state
     o["_struct"] = s
     return o
 

@@ -84,6 +84,7 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_uw = bump(c, BH * N * 8);
     pl.o_lbar = bump(c, BH * Cq * Ck * 4);
     pl.o_vv = bump(c, BH * Ck * 4);
+    pl.o_warm = bump(c, (1 + 2 * BH) * 4);
     // outputs owned by the workspace (fused call)
     pl.o_Qp = bump(c, BH * N * d * es);
     pl.o_Kp = bump(c, BH * N * d * es);
@@ -246,7 +247,28 @@ sparsepr_status sparsepr_partition(const sparsepr_params* p, const void* Q, cons
         return SPARSEPR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     if (cudaMemsetAsync(at<void>(ws, pl.o_status), 0, 256, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
+    // the workspace no longer holds a complete fused-call state
+    if (cudaMemsetAsync(at<void>(ws, pl.o_warm), 0, 4, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
     return run_partition(*p, pl, Q, K, V, *part, ws, st);
+}
+
+sparsepr_status sparsepr_partition_warm(const sparsepr_params* p, const void* Q, const void* K, const void* V,
+                                        const sparsepr_warm_state* prev, const sparsepr_partition_out* part,
+                                        void* ws, size_t bytes, void* stream) {
+    Plan pl;
+    sparsepr_status s = check_ws(p, pl, ws, bytes);
+    if (s != SPARSEPR_OK) return s;
+    if (!Q || !K || !V || !partition_ok(part)) return SPARSEPR_INVALID_ARG;
+    if (!prev || !prev->F_K || !prev->F_Q || !prev->k_centroid || !prev->q_centroid || !prev->n_groups)
+        return SPARSEPR_INVALID_ARG;
+    if ((p->flags & SPARSEPR_FLAG_DEBUG_EXPORT) &&
+        !(part->debug_kv_scores && part->debug_q_scores && part->debug_kv_hist && part->debug_q_hist))
+        return SPARSEPR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemsetAsync(at<void>(ws, pl.o_status), 0, 256, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
+    if (cudaMemsetAsync(at<void>(ws, pl.o_warm), 0, 4, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
+    const WarmSource src{prev->F_K, prev->F_Q, prev->k_centroid, prev->q_centroid, prev->n_groups, nullptr};
+    return run_partition(*p, pl, Q, K, V, *part, ws, st, &src);
 }
 
 sparsepr_status sparsepr_route(const sparsepr_params* p, const sparsepr_partition_out* part,
@@ -315,7 +337,12 @@ sparsepr_status sparsepr_call(const sparsepr_params* p, const void* Q, const voi
     const long long launches0 = launch_counter();
     sparsepr_params q = *p;
     q.flags &= ~SPARSEPR_FLAG_DEBUG_EXPORT;
-    if ((s = run_partition(q, pl, Q, K, V, part, ws, st)) != SPARSEPR_OK) return s;
+    int32_t* warm_word = at<int32_t>(ws, pl.o_warm);
+    const WarmSource src{at<float>(ws, pl.o_FK), at<float>(ws, pl.o_FQ), part.k_centroid, part.q_centroid,
+                         part.n_groups, warm_word};
+    const bool warm = (p->flags & SPARSEPR_FLAG_WARM_START) != 0;
+    if ((s = run_partition(q, pl, Q, K, V, part, ws, st, warm ? &src : nullptr)) != SPARSEPR_OK) return s;
+    launch_set_word(warm_word, kWarmMagic, st);
     if (stats) cudaEventRecord(ev[1], st);
     if ((s = run_route(q, pl, part, route, ws, st)) != SPARSEPR_OK) return s;
     if (stats) cudaEventRecord(ev[2], st);

@@ -8,8 +8,40 @@
 
 namespace spr {
 
+// Warm start (paper C.1): where the previous call's state lives.  `valid`
+// (or nullptr) points at a word that must equal kWarmMagic for it to be used.
+struct WarmSource {
+    const float* F_K;
+    const float* F_Q;
+    const float* k_centroid;
+    const float* q_centroid;
+    const int32_t* n_groups;
+    const int32_t* valid;
+};
 sparsepr_status run_partition(const sparsepr_params& p, const Plan& pl, const void* Q, const void* K,
-                              const void* V, const sparsepr_partition_out& out, void* ws, cudaStream_t st);
+                              const void* V, const sparsepr_partition_out& out, void* ws, cudaStream_t st,
+                              const WarmSource* warm = nullptr);
+// Initial centres of a warm k-means: previous centroids `cbar` ([BH,C,d]) of
+// the first ng_prev[bh*2+which] groups projected by F ([BH,d,R]).
+struct WarmInit {
+    const float* cbar;
+    const int32_t* ng_prev;
+    int which;
+    const float* F;
+    int d;
+    bool rms;
+    const int32_t* r_eff;
+    float eps;
+    const int32_t* valid;
+};
+void launch_warm_init(const WarmInit& w, int R, const float* phi, int BH, int N, int C, uint64_t seed, int stage,
+                      float* cen, float* hn, cudaStream_t st);
+// *word = value, in stream order (one thread).
+void launch_set_word(int32_t* word, int32_t value, cudaStream_t st);
+// Warm metric factor; heads it cannot factor get cold[bh] = 1 (else 0).
+void launch_warm_factor(const float* M, const float* Fprev, int ld_prev, int r_req, const int32_t* ng, float scale,
+                        float* F, int Rp, int32_t* r_out, int32_t* cold, const int32_t* valid, int BH, int d,
+                        cudaStream_t st);
 sparsepr_status run_route(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
                           const sparsepr_route_out& r, void* ws, cudaStream_t st);
 bool attention_uses_tc(const sparsepr_params& p);

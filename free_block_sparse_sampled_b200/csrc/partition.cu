@@ -101,14 +101,16 @@ __global__ void __launch_bounds__(256) centred_gram_kernel(const float* __restri
 // F[:, c] = u_c sqrt(max(lambda_c, 0)) * scale for the r leading eigenpairs
 // (descending, ties to the lower index) and zero columns up to Rp.
 // For the query factor (ng != nullptr) r = max(1, min(r_req, d, C_k' - 1)).
+// With run_if, only heads whose run_if entry is nonzero are factored.
 template <int d>
 __global__ void __launch_bounds__(1024) jacobi_factor_kernel(const float* __restrict__ Ain,
                                                             float* __restrict__ F, int Rp,
                                                             int r_req, const int32_t* ng,
                                                             float scale, int32_t* r_out,
-                                                            int max_sweeps) {
+                                                            int max_sweeps, const int32_t* run_if) {
     extern __shared__ float sm[];
     const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    if (run_if != nullptr && run_if[bh] == 0) return;     // factored by the warm start
     const int ld = d + 1, half = d / 2;
     float* A = sm;
     float* V = A + d * ld;
@@ -684,7 +686,7 @@ inline int grid_for(size_t total, int threads) {
 template <int R>
 void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float* phi, int C,
                 int stage, float* cen, float* hn, float* dbg_scores, int32_t* dbg_hist,
-                int save_slot, cudaStream_t st) {
+                int save_slot, const WarmInit* wi, cudaStream_t st) {
     int32_t* ctl = at<int32_t>(ws, pl.o_ctl);
     int32_t* raw = at<int32_t>(ws, pl.o_raw);
     int32_t* hist = at<int32_t>(ws, pl.o_hist);
@@ -693,7 +695,10 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
     const int BH = pl.BH, N = pl.N;
     const int bgrid = (BH + 127) / 128;
     count_launch(), kmeans_reset_kernel<<<bgrid, 128, 0, st>>>(ctl, BH, save_slot);
-    count_launch(), kmeans_init_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, N, C, p.seed, stage, cen, hn);
+    if (wi != nullptr)
+        launch_warm_init(*wi, R, phi, BH, N, C, p.seed, stage, cen, hn, st);
+    else
+        count_launch(), kmeans_init_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, N, C, p.seed, stage, cen, hn);
     const dim3 agrid((N + 127) / 128, BH);
     const dim3 tgrid(pl.n_sort_tiles, BH), cgrid((C + 255) / 256, BH);
     for (int it = 0; it < p.kmeans_iters; ++it) {
@@ -716,12 +721,12 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
 
 void kmeans_dispatch(int R, const Plan& pl, const sparsepr_params& p, void* ws, const float* phi,
                      int C, int stage, float* cen, float* hn, float* dbg_scores, int32_t* dbg_hist,
-                     int save_slot, cudaStream_t st) {
+                     int save_slot, const WarmInit* wi, cudaStream_t st) {
     switch (R) {
-        case 16: kmeans_run<16>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
-        case 32: kmeans_run<32>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
-        case 48: kmeans_run<48>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
-        default: kmeans_run<64>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, st); break;
+        case 16: kmeans_run<16>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
+        case 32: kmeans_run<32>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
+        case 48: kmeans_run<48>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
+        default: kmeans_run<64>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
     }
 }
 
@@ -771,7 +776,7 @@ void gather(const void* X, const int32_t* perm, const Plan& pl, void* Xp, cudaSt
 template <typename T>
 sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const T* Q, const T* K,
                                 const T* V, const sparsepr_partition_out& out, void* ws,
-                                cudaStream_t st) {
+                                cudaStream_t st, const WarmSource* warm) {
     const int BH = pl.BH, N = pl.N, d = pl.d;
     float* mat = at<float>(ws, pl.o_mat);
     float* FK = at<float>(ws, pl.o_FK);
@@ -793,12 +798,24 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
 
     // 1-2. key-response metric and factor (§4.1)
     count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff, mat);
+    // warm start (C.1): subspace iteration from the previous factor; heads it
+    // cannot factor (or every head, without a previous state) take Jacobi
+    int32_t* coldK = at<int32_t>(ws, pl.o_warm) + 1;
+    int32_t* coldQ = coldK + BH;
+    if (warm)
+        launch_warm_factor(mat, warm->F_K, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d), FK, pl.RKp, nullptr,
+                           coldK, warm->valid, BH, d, st);
     count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d),
-                                                      nullptr, 16);
+                                                      nullptr, 16, warm ? coldK : nullptr);
     project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
     // 3. paired K/V groups
+    WarmInit wiK{}, wiQ{};
+    if (warm) {
+        wiK = WarmInit{warm->k_centroid, warm->n_groups, 1, FK, d, false, nullptr, 0.f, warm->valid};
+        wiQ = WarmInit{warm->q_centroid, warm->n_groups, 0, FQ, d, true, rq, p.eps_rms, warm->valid};
+    }
     kmeans_dispatch(pl.RKp, pl, p, ws, phiK, pl.Ck, 0, cenK, hnK, dbg ? out.debug_kv_scores : nullptr,
-                    dbg ? out.debug_kv_hist : nullptr, -1, st);
+                    dbg ? out.debug_kv_hist : nullptr, -1, warm ? &wiK : nullptr, st);
     if (out.kv_centres) cudaMemcpyAsync(out.kv_centres, cenK, (size_t)BH * pl.Ck * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
     finalize_groups(pl, ws, pl.Ck, 1, out.kv_label, out.perm_kv, nullptr, out.kv_offsets, out.n_groups, st);
     gather(K, out.perm_kv, pl, out.Kp, st);
@@ -811,11 +828,15 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), centroid_mean_kernel<<<BH, d, 0, st>>>(out.k_centroid, out.n_groups, pl.Ck, d, muK);
     count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
                                                                           out.n_groups, pl.Ck, d, mat);
-    count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16);
+    if (warm)
+        launch_warm_factor(mat, warm->F_Q, pl.RQp, p.rQ, out.n_groups, 1.f, FQ, pl.RQp, rq, coldQ, warm->valid, BH, d,
+                           st);
+    count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16,
+                                                      warm ? coldQ : nullptr);
     project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, at<DevStatus>(ws, pl.o_status), st);
     // 5. query groups
     kmeans_dispatch(pl.RQp, pl, p, ws, phiQ, pl.Cq, 1, cenQ, hnQ, dbg ? out.debug_q_scores : nullptr,
-                    dbg ? out.debug_q_hist : nullptr, kCtlItersK, st);
+                    dbg ? out.debug_q_hist : nullptr, kCtlItersK, warm ? &wiQ : nullptr, st);
     count_launch(), kmeans_reset_kernel<<<(BH + 127) / 128, 128, 0, st>>>(ctl, BH, kCtlItersQ);
     if (out.q_centres) cudaMemcpyAsync(out.q_centres, cenQ, (size_t)BH * pl.Cq * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
     finalize_groups(pl, ws, pl.Cq, 0, out.q_label, out.perm_q, out.pos_q, out.q_offsets, out.n_groups, st);
@@ -839,13 +860,13 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
 
 sparsepr_status run_partition(const sparsepr_params& p, const Plan& pl, const void* Q, const void* K,
                               const void* V, const sparsepr_partition_out& out, void* ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, const WarmSource* warm) {
     if (p.dtype == SPARSEPR_BF16)
         return partition_typed<__nv_bfloat16>(p, pl, static_cast<const __nv_bfloat16*>(Q),
                                               static_cast<const __nv_bfloat16*>(K),
-                                              static_cast<const __nv_bfloat16*>(V), out, ws, st);
+                                              static_cast<const __nv_bfloat16*>(V), out, ws, st, warm);
     return partition_typed<float>(p, pl, static_cast<const float*>(Q), static_cast<const float*>(K),
-                                  static_cast<const float*>(V), out, ws, st);
+                                  static_cast<const float*>(V), out, ws, st, warm);
 }
 
 }  // namespace spr

@@ -7,6 +7,8 @@
  * below with the section or formula that defines each step:
  *
  *   partition  response-coupled partitioning           paper §4.1, B.1, B.2, C.1
+ *              (cold, or warm-started from a previous  paper C.1 "Warm start",
+ *              call of the same problem shape)         Table C.1
  *   route      value-error score + prefix budget rule   paper §4.3, B.3, A.2
  *   attention  renormalised block-sparse attention       paper §3 Eq. (2), §4.3
  *              and exact attention on the probe rows
@@ -62,6 +64,10 @@ typedef enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 } sparsepr_dtype;
 /* flags */
 #define SPARSEPR_FLAG_DEBUG_EXPORT 1   /* fill the debug_* outputs of partition */
 #define SPARSEPR_FLAG_SIMT_ATTENTION 2 /* bf16: use the CUDA-core attention kernel */
+#define SPARSEPR_FLAG_WARM_START 4     /* sparsepr_call: warm-start the partition from the state the
+                                          previous sparsepr_call with the same *p left in this
+                                          workspace (see sparsepr_partition_warm); without such a
+                                          state the call is cold */
 
 /* Problem statement (paper §3 / §4 notation).  All fields are read on the host. */
 typedef struct {
@@ -102,9 +108,10 @@ typedef struct {
     float* v_centroid;    /* [BH,Ck,d] vbar_b */
     float* q_dist;        /* [BH,N] d_i = |phi_Q(q_i) - c_a| by original row (A.2) */
     /* optional */
-    float* F_K;           /* [BH,d,rK] key factor (columns beyond r_K' zero) */
-    float* F_Q;           /* [BH,d,rQ] query factor (columns beyond r_Q' zero) */
-    float* phi_K;         /* [BH,N,RKp] key coordinates, RKp = rK rounded up to 16 */
+    float* F_K;           /* [BH,d,RKp] key factor (columns beyond r_K' zero) */
+    float* F_Q;           /* [BH,d,RQp] query factor, RQp = min(rQ,d) rounded up to 16
+                             (at least 32; columns beyond r_Q' zero) */
+    float* phi_K;         /* [BH,N,RKp] key coordinates, RKp = r_K' rounded up to 16 (at least 32) */
     float* phi_Q;         /* [BH,N,RQp] query coordinates (after RMSNorm) */
     float* kv_centres;    /* [BH,Ck,RKp] k-means centres used by the last assignment */
     float* q_centres;     /* [BH,Cq,RQp] */
@@ -165,6 +172,37 @@ size_t sparsepr_workspace_size(const sparsepr_params* p);
 sparsepr_status sparsepr_partition(const sparsepr_params* p, const void* Q, const void* K,
                                    const void* V, const sparsepr_partition_out* part,
                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* State a warm-started partition starts from (paper C.1 "Warm start"): the
+ * outputs of an earlier partition of the same *p (e.g. the previous denoising
+ * step of the same layer).  DEVICE pointers, caller-owned, read only. */
+typedef struct {
+    const float* F_K;         /* [BH,d,RKp] that call's part->F_K */
+    const float* F_Q;         /* [BH,d,RQp] that call's part->F_Q */
+    const float* k_centroid;  /* [BH,Ck,d] that call's kbar_b */
+    const float* q_centroid;  /* [BH,Cq,d] that call's qbar_a */
+    const int32_t* n_groups;  /* [BH,2] that call's (C_q', C_k') */
+} sparsepr_warm_state;
+
+/* sparsepr_partition started from a previous call's state (paper C.1):
+ *  - metric factors: two subspace iterations from the previous factor
+ *    (Y = M Q, Q = Y L^-T with L L^T = Y^T Y), then F = Q C with
+ *    C C^T = Q^T M Q (times 1/sqrt(d) for F_K), in place of the
+ *    eigendecomposition.  A head whose Cholesky pivot vanishes (square not
+ *    above 1e-12 x the largest diagonal entry), or whose previous F_Q has
+ *    fewer nonzero columns than this call's r_Q', takes the cold factor.
+ *  - k-means: initial centre b < C_k'(prev) of the K/V groups is kbar_b F_K,
+ *    initial centre a < C_q'(prev) of the query groups is RMSNorm(qbar_a F_Q)
+ *    (both TF32-rounded); later centres are the cold start's sampled rows.
+ *    p->kmeans_iters is the limit of this call (Table C.1 uses 2 after the
+ *    first call).
+ * Every other step, output and error is that of sparsepr_partition.  `prev`
+ * may point into `part` of the previous call: each previous value is read
+ * before this call overwrites it. */
+sparsepr_status sparsepr_partition_warm(const sparsepr_params* p, const void* Q, const void* K,
+                                        const void* V, const sparsepr_warm_state* prev,
+                                        const sparsepr_partition_out* part, void* workspace,
+                                        size_t workspace_bytes, void* stream);
 
 /* §4.3, B.3, A.2: routing scores, per-query-group prefix selection at the key
  * budget beta = (density - M/N) N, executed-pair counts, stratified probe

@@ -6,4 +6,4 @@ oracle and the CUDA path may import it without sharing method code.
 """
 
 from .workloads import WORKLOADS, Workload, get_workload  # noqa: F401
-from .video_grid import generate_head, generate_inputs, bf16_round  # noqa: F401
+from .video_grid import generate_head, generate_inputs, bf16_round, drift_inputs  # noqa: F401

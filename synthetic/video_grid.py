@@ -122,6 +122,18 @@ def generate_inputs(w: Workload, heads=None, bits: bool = False):
     return tuple(out)
 
 
+def drift_inputs(w: Workload, qkv, step: int = 1, rel: float = 0.05):
+    """Inputs of a later call of the same layer (the next denoising step):
+    each of Q, K, V plus Gaussian noise of ``rel`` times its own std, from a
+    stream seeded by (workload seed, step).  bf16 workloads are re-rounded."""
+    rng = np.random.default_rng([int(w.seed), int(step), 515151])
+    out = []
+    for x in qkv:
+        y = x + np.float32(rel) * np.float32(x.std()) * rng.standard_normal(x.shape, dtype=np.float32)
+        out.append(bf16_round(y) if w.dtype == "bf16" else y.astype(np.float32))
+    return tuple(out)
+
+
 def planted_map(w: Workload, b: int, h: int, rank: int = 8, scale: float = 0.05):
     """Seeded affine map (b*, U, V^T) of rank ``rank`` for the planted variant:
     planted dense probe rows are  O_sp + b* + O_sp U V^T."""

@@ -210,9 +210,10 @@ def check_fit_and_apply(h, cfg):
     assert np.array_equal(h["out"][h["probe_idx"]], D)
 
 
-def check_partition_floats(h, cfg, q, k, v):
+def check_partition_floats(h, cfg, q, k, v, warm=None):
     """Float outputs of the partition against fp64 recomputation from the
-    GPU's own integer decisions."""
+    GPU's own integer decisions.  ``warm`` (F_K, F_Q of the state a warm call
+    started from, fp64) switches the factor references to the warm factor."""
     kl, ql = h["kv_label"], h["q_label"]
     np.testing.assert_allclose(h["k_centroid"], O.group_means(k, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
     np.testing.assert_allclose(h["v_centroid"], O.group_means(v, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
@@ -233,13 +234,21 @@ def check_partition_floats(h, cfg, q, k, v):
     ref = U[:, :r] @ np.diag(w[:r]) @ U[:, :r].T / cfg.d
     FK = h["F_K"]
     gap_ok = r == cfg.d or (w[r - 1] - w[r]) > 1e-2 * w[0]
-    if gap_ok:
+    Fw = None if warm is None else O.warm_factor(MK, warm["F_K"], r, 1.0 / math.sqrt(cfg.d))
+    if Fw is not None:
+        ref = Fw @ Fw.T
+        assert np.abs(FK @ FK.T - ref).max() <= 2e-4 * np.abs(ref).max(), "warm F_K"
+    elif gap_ok:
         assert np.abs(FK @ FK.T - ref).max() <= 2e-4 * np.abs(ref).max()
     MQ = O.query_metric(h["k_centroid"])
     wq, Uq = O.eigh_desc(MQ)
     refq = Uq[:, :rq] @ np.diag(wq[:rq]) @ Uq[:, :rq].T
     FQ = h["F_Q"]
-    if rq >= int((wq > 1e-9 * wq[0]).sum()) or (wq[rq - 1] - wq[rq]) > 1e-2 * wq[0]:
+    Fwq = None if warm is None else O.warm_factor(MQ, warm["F_Q"], rq, 1.0)
+    if Fwq is not None:
+        refq = Fwq @ Fwq.T
+        assert np.abs(FQ @ FQ.T - refq).max() <= 2e-4 * np.abs(refq).max(), "warm F_Q"
+    elif rq >= int((wq > 1e-9 * wq[0]).sum()) or (wq[rq - 1] - wq[rq]) > 1e-2 * wq[0]:
         assert np.abs(FQ @ FQ.T - refq).max() <= 2e-4 * np.abs(refq).max()
     # routing scores vs the direct sum on the GPU's groups and centroids
     s_ref = O.routing_score(h["q_centroid"], k, v, h["k_centroid"], h["v_centroid"], kl)
