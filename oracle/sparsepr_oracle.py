@@ -56,6 +56,12 @@ R14 Warm start, centres (paper C.1: "previous centroids in the original space
     drawn as in a cold start (R3).
 R15 Later calls run at most 2 k-means assignments (Table C.1, "initial /
     subsequent k means iteration limits 25/2"); the caller passes the limit.
+R16 Semantic partition (§3's reference partition, Table 2's baseline): the
+    same k-means (initial rows, limit, stop rule) on the raw key rows and on
+    the raw query rows, V inheriting its key's group; d_i is the distance to
+    the raw-space query-group mean.  Routing, probes, fit and apply are
+    unchanged.  Table 2's key-response variant keeps the response K/V groups
+    and takes semantic query groups.
 """
 
 from __future__ import annotations
@@ -485,12 +491,18 @@ def error_reduction(mean_err_method: float, mean_err_base: float) -> float:
 def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: int,
                   lam: float, Cq: int, Ck: int, rK: int, rQ: int, kmeans_iters: int,
                   kmeans_tol: float, eps_rms: float = 1e-6, eps_std: float = 1e-6,
-                  want_dense: bool = False, warm: Optional[Dict[str, np.ndarray]] = None) -> Dict[str, object]:
+                  want_dense: bool = False, warm: Optional[Dict[str, np.ndarray]] = None,
+                  partition: str = "response") -> Dict[str, object]:
     """One SparsePR call on one head, steps in the paper's order:
     partition (§4.1) -> route (§4.3, B.3) -> sparse attention (Eq. 2) ->
     probes (A.2) -> weighted ridge (A.3) -> corrected output (§4.2).
     ``warm`` (F_K, F_Q, kbar, qbar of the previous call) selects the warm
-    start of R13-R15; the caller also lowers ``kmeans_iters``."""
+    start of R13-R15; the caller also lowers ``kmeans_iters``.
+    ``partition``: "response" (§4.1), "semantic" or "key_response" (R16)."""
+    if partition not in ("response", "semantic", "key_response"):
+        raise ValueError(partition)
+    semantic_keys = partition == "semantic"
+    semantic_queries = partition in ("semantic", "key_response")
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -501,9 +513,11 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     idx = sample_indices(N, Ms)
     M_K = key_metric(q, idx)
     r_k = min(rK, d, len(idx))
-    F_K = None if warm is None else warm_factor(M_K, warm["F_K"], r_k, 1.0 / math.sqrt(d))
+    F_K = None if (warm is None or semantic_keys) else warm_factor(M_K, warm["F_K"], r_k, 1.0 / math.sqrt(d))
     warm_K = F_K is not None
-    if F_K is None:
+    if semantic_keys:
+        F_K = np.eye(d)
+    elif F_K is None:
         F_K = key_factor(M_K, rK, len(idx))
     phi_K = k @ F_K
     # 3. paired K/V groups
@@ -517,14 +531,19 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     vbar = group_means(v, kv_labels, Ck2)
     M_Q = query_metric(kbar)
     rq = query_rank(rQ, d, Ck2)
-    F_Q = None if warm is None else warm_factor(M_Q, warm["F_Q"], rq, 1.0)
+    F_Q = None if (warm is None or semantic_queries) else warm_factor(M_Q, warm["F_Q"], rq, 1.0)
     warm_Q = F_Q is not None
-    if F_Q is None:
-        F_Q = query_factor(M_Q, rq)
-    phi_Q = query_coords(q, F_Q, eps_rms)
+    if semantic_queries:
+        F_Q = np.eye(d)
+        phi_Q = q.copy()
+    else:
+        if F_Q is None:
+            F_Q = query_factor(M_Q, rq)
+        phi_Q = query_coords(q, F_Q, eps_rms)
     # 5. query groups
     init_q = kmeans_init_indices(seed, bh, 1, Cq, N)
-    cen_q = None if warm is None else warm_centres(phi_Q, warm["qbar"], F_Q, Cq, init_q, eps_rms)
+    cen_q = None if warm is None else warm_centres(phi_Q, warm["qbar"], F_Q, Cq, init_q,
+                                                   None if semantic_queries else eps_rms)
     q_raw, _, it_q, _ = kmeans(phi_Q, init_q, kmeans_iters, stop, cen_q)
     q_labels, Cq2, q_sizes = compact_labels(q_raw, Cq)
     qbar = group_means(q, q_labels, Cq2)

@@ -629,3 +629,67 @@ def test_warm_call_on_same_input_keeps_converged_kv_groups():
     assert np.array_equal(warm["kv_labels"], cold["kv_labels"])
     assert warm["kmeans_iters_k"] <= 2 and warm["kmeans_iters_q"] <= 2
     assert warm["pairs_exec"] / w.N / w.N >= w.density - 1e-12
+
+
+# ------------------------------------------------------ semantic partition (R16)
+def _blob_keys(seed=80, N=160, d=6):
+    """Keys in two far blobs along e_0, a direction no query has: raw-key
+    clustering splits the blobs, the response metric cannot see them."""
+    rng = np.random.default_rng(seed)
+    blob = np.arange(N) % 2
+    k = rng.standard_normal((N, d)) * 0.2
+    k[:, 0] += np.where(blob == 1, 50.0, -50.0)
+    k[:, 1:] += rng.standard_normal((N, d - 1)) * 2.0
+    q = rng.standard_normal((N, d))
+    q[:, 0] = 0.0
+    v = rng.standard_normal((N, d))
+    return q, k, v, blob
+
+
+def _kw(**over):
+    kw = dict(seed=3, density=0.5, M=8, Ms=64, lam=1.0, Cq=4, Ck=2, rK=4, rQ=4, kmeans_iters=25,
+              kmeans_tol=0.0)
+    kw.update(over)
+    return kw
+
+
+def test_semantic_keys_split_raw_blobs_response_keys_do_not():
+    q, k, v, blob = _blob_keys()
+    sem = O.sparsepr_head(q, k, v, bh=0, partition="semantic", **_kw())
+    res = O.sparsepr_head(q, k, v, bh=0, partition="response", **_kw())
+    lab = sem["kv_labels"]
+    assert sem["Ck"] == 2 and (np.array_equal(lab, blob) or np.array_equal(lab, 1 - blob))
+    # phi_K = k F_K has no e_0 component, so the blobs coincide in response coordinates
+    assert np.abs(res["F_K"][0]).max() < 1e-12
+    agree = max((res["kv_labels"] == blob).mean(), (res["kv_labels"] != blob).mean())
+    assert agree < 0.75
+
+
+def test_semantic_query_distances_are_raw_space():
+    q, k, v, _ = _blob_keys(81)
+    r = O.sparsepr_head(q, k, v, bh=0, partition="semantic", **_kw())
+    for a in range(r["Cq"]):
+        mem = np.nonzero(r["q_labels"] == a)[0]
+        mean = q[mem].mean(axis=0)
+        for i in mem[:5]:
+            assert abs(r["d_i"][i] - math.sqrt(sum((q[i, t] - mean[t]) ** 2 for t in range(q.shape[1])))) < 1e-12
+
+
+def test_key_response_variant_mixes_the_two():
+    q, k, v, _ = _blob_keys(82)
+    sem = O.sparsepr_head(q, k, v, bh=0, partition="semantic", **_kw())
+    res = O.sparsepr_head(q, k, v, bh=0, partition="response", **_kw())
+    kr = O.sparsepr_head(q, k, v, bh=0, partition="key_response", **_kw())
+    assert np.array_equal(kr["kv_labels"], res["kv_labels"])
+    assert np.array_equal(kr["q_labels"], sem["q_labels"])
+
+
+def test_semantic_call_is_rotation_invariant():
+    """Rotating queries and keys by one orthogonal map changes no distance
+    between raw rows and no logit, so the semantic call's output is unchanged."""
+    q, k, v, _ = _blob_keys(83)
+    R, _ = np.linalg.qr(_rand((6, 6), 84))
+    a = O.sparsepr_head(q, k, v, bh=0, partition="semantic", **_kw(Cq=5, Ck=3))
+    b = O.sparsepr_head(q @ R, k @ R, v, bh=0, partition="semantic", **_kw(Cq=5, Ck=3))
+    assert np.array_equal(a["kv_labels"], b["kv_labels"]) and np.array_equal(a["q_labels"], b["q_labels"])
+    np.testing.assert_allclose(a["O"], b["O"], atol=1e-10)
