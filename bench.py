@@ -288,6 +288,54 @@ def whole_job_ms_per_call(ms_step_max: float, world: int) -> float:
 
 
 # --------------------------------------------------------------------- ours
+def table2_errors(S, cfg, q, k, v, out, part, rt, O_sp, rows, ref, dev):
+    """Mean / p99 relative L2 of the attention output on unprobed rows for the
+    paper's Table 2 partitions at the same density: semantic (k-means on raw
+    Q and K), key-response K/V with semantic queries, response-coupled; each
+    without repair, and semantic and SparsePR with repair.  Each method uses
+    its own stratified probes; rows that are a probe of any method are left out."""
+    import dataclasses
+    import torch
+    from free_block_sparse_sampled_b200 import _abi
+
+    def permuted_rows(O_p, pos):
+        osp = O_p.view(cfg.B, cfg.H, cfg.N, cfg.d)
+        p = pos.view(cfg.B, cfg.H, cfg.N).long()[:, :, rows]
+        return torch.gather(osp, 2, p.unsqueeze(-1).expand(-1, -1, -1, cfg.d))
+
+    def probe_mask(rt_):
+        m = torch.zeros(cfg.B, cfg.H, cfg.N, dtype=torch.bool, device=dev)
+        m.scatter_(2, rt_["probe_idx"].view(cfg.B, cfg.H, -1).long().clamp_min(0), True)
+        return m[:, :, rows]
+
+    outs = {"response": permuted_rows(O_sp, part["pos_q"]), "sparsepr": out[:, :, rows].clone()}
+    probed = probe_mask(rt)
+    for name, flags in (("semantic", _abi.FLAG_SEMANTIC_KEYS | _abi.FLAG_SEMANTIC_QUERIES),
+                        ("key_response", _abi.FLAG_SEMANTIC_QUERIES)):
+        c = dataclasses.replace(cfg, flags=cfg.flags | flags)
+        wsx = S.alloc_workspace(c, dev)
+        px = S.partition(c, q, k, v, wsx)
+        rx = S.route(c, px, wsx)
+        ox, pdx, psx = S.attention(c, px, rx, wsx)
+        outs[name] = permuted_rows(ox, px["pos_q"])
+        if name == "semantic":
+            fx = S.probe_fit(c, px, rx, psx, pdx, wsx)
+            outs["semantic_repair"] = S.apply(c, px, rx, ox, pdx, fx, wsx)[:, :, rows].clone()
+        probed |= probe_mask(rx)
+        torch.cuda.synchronize()
+        del wsx, px, rx, ox, pdx, psx
+    keep = ~probed
+    res = {}
+    for name, o in outs.items():
+        e = ((o - ref).norm(dim=-1) / (ref.norm(dim=-1) + 1e-8))[keep].double()
+        res[name] = {"mean": float(e.mean()), "p99": float(torch.quantile(e, 0.99))}
+    res["error_reduction_vs_semantic"] = 1.0 - res["sparsepr"]["mean"] / res["semantic"]["mean"]
+    res["error_reduction_vs_semantic_repair"] = 1.0 - res["sparsepr"]["mean"] / res["semantic_repair"]["mean"]
+    res["rows"] = "2048 evenly spaced rows per head that no method probes"
+    res["probes"] = "each method's own stratified probes (the paper fixes SparsePR's for its repair comparison)"
+    return res
+
+
 def run_ours(args, w):
     import torch
     import free_block_sparse_sampled_b200 as S
@@ -426,6 +474,7 @@ def run_ours(args, w):
             "device_status": S.device_status(ws),
             "inputs": "the same Q/K/V as the cold call; the state is the previous call's"}
         S.call(cfg, q, k, v, ws, out)                   # the cold call's output again
+        extras["table2_errors"] = table2_errors(S, cfg, q, k, v, out, part, rt, O_sp, rows, ref, dev)
     e2e = None
     if not args.no_e2e and not args.quick:
         # End to end from pinned host memory through the package's HostPipeline:

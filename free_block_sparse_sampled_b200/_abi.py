@@ -14,6 +14,8 @@ BF16, F32 = 0, 1
 FLAG_DEBUG_EXPORT = 1
 FLAG_SIMT_ATTENTION = 2
 FLAG_WARM_START = 4
+FLAG_SEMANTIC_KEYS = 8
+FLAG_SEMANTIC_QUERIES = 16
 
 EXPORTED = ["sparsepr_status_string", "sparsepr_validate", "sparsepr_workspace_size",
             "sparsepr_partition", "sparsepr_route", "sparsepr_attention", "sparsepr_probe_fit",

@@ -66,11 +66,15 @@ class SparsePRConfig:
 
     @property
     def RKp(self) -> int:
+        if self.flags & A.FLAG_SEMANTIC_KEYS:
+            return self.d
         r = min(self.rK, self.d, min(self.Ms, self.N))
         return max(32, (r + 15) // 16 * 16)
 
     @property
     def RQp(self) -> int:
+        if self.flags & A.FLAG_SEMANTIC_QUERIES:
+            return self.d
         return max(32, (min(self.rQ, self.d) + 15) // 16 * 16)
 
     def c_params(self) -> A.Params:

@@ -28,9 +28,12 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     int rk = p.rK < p.d ? p.rK : p.d;
     rk = rk < pl.Ms_eff ? rk : pl.Ms_eff;
     pl.rK_eff = rk;
-    // coordinate rows: a multiple of 16 floats and at least one 128-byte TMA chunk
+    // coordinate rows: a multiple of 16 floats and at least one 128-byte TMA
+    // chunk; the raw rows (d floats) for a semantic side
     pl.RKp = round_up(rk, 16) < 32 ? 32 : round_up(rk, 16);
     pl.RQp = round_up(p.rQ < p.d ? p.rQ : p.d, 16) < 32 ? 32 : round_up(p.rQ < p.d ? p.rQ : p.d, 16);
+    if (p.flags & SPARSEPR_FLAG_SEMANTIC_KEYS) pl.RKp = p.d;
+    if (p.flags & SPARSEPR_FLAG_SEMANTIC_QUERIES) pl.RQp = p.d;
     pl.Mp = p.M < p.N ? p.M : p.N;
     pl.esz = p.dtype == SPARSEPR_BF16 ? 2 : 4;
     pl.n_sort_tiles = (p.N + kSortTile - 1) / kSortTile;

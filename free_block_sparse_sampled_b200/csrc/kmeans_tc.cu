@@ -300,6 +300,7 @@ void kmeans_centre_blocks(int C, int& NB, int& nblk) {
 bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, int BH, int N, int C, int R,
                              int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
                              int max_iter, DevStatus* status, cudaStream_t st) {
+    if (R > kMaxRank) return false;              // shared-memory tiles hold rows of up to 64 floats
     int NB, nblk;
     kmeans_centre_blocks(C, NB, nblk);
     kmtc::Maps maps;

@@ -499,7 +499,7 @@ __global__ void centre_update_kernel(const float* __restrict__ phi, const int32_
                                      const int32_t* __restrict__ offs, int N, int C,
                                      float* __restrict__ cen, float* __restrict__ hn,
                                      const int32_t* __restrict__ ctl) {
-    static_assert(R % 16 == 0 && R >= 16 && R <= 64, "coordinate rows of 16..64 floats");
+    static_assert(R % 16 == 0 && R >= 16 && R <= 128, "coordinate rows of 16..128 floats");
     constexpr int LPR = R / 4;        // lanes per row
     constexpr int RPL = 32 / LPR;     // rows per warp load
     constexpr int LOADS = 32 / RPL;   // loads per 32 listed members
@@ -675,6 +675,27 @@ __global__ void iters_out_kernel(const int32_t* __restrict__ ctl, int BH, int32_
     out[bh * 2 + 1] = ctl[bh * kCtlStride + kCtlItersQ];
 }
 
+// Semantic partition (paper §3 reference partition, Table 2): the k-means
+// coordinates are the raw rows, TF32-rounded (exact for bf16 inputs), and
+// the factor is the identity.
+template <typename T>
+__global__ void raw_coords_kernel(const T* __restrict__ X, size_t n8, float* __restrict__ phi) {
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n8; e += (size_t)gridDim.x * blockDim.x) {
+        float v[8];
+        load8(X + e * 8, v);
+        float4* o = reinterpret_cast<float4*>(phi + e * 8);
+        o[0] = make_float4(tf32_round(v[0]), tf32_round(v[1]), tf32_round(v[2]), tf32_round(v[3]));
+        o[1] = make_float4(tf32_round(v[4]), tf32_round(v[5]), tf32_round(v[6]), tf32_round(v[7]));
+    }
+}
+
+__global__ void identity_factor_kernel(float* __restrict__ F, int d, int Rp, int32_t* __restrict__ r_out) {
+    const int bh = blockIdx.x;
+    float* Fh = F + (size_t)bh * d * Rp;
+    for (int e = threadIdx.x; e < d * Rp; e += blockDim.x) Fh[e] = (e / Rp == e % Rp) ? 1.f : 0.f;
+    if (threadIdx.x == 0 && r_out != nullptr) r_out[bh] = d;
+}
+
 // ================================================================ host side
 namespace {
 
@@ -726,7 +747,8 @@ void kmeans_dispatch(int R, const Plan& pl, const sparsepr_params& p, void* ws, 
         case 16: kmeans_run<16>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
         case 32: kmeans_run<32>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
         case 48: kmeans_run<48>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
-        default: kmeans_run<64>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
+        case 64: kmeans_run<64>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
+        default: kmeans_run<128>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
     }
 }
 
@@ -796,23 +818,33 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     auto jacobi = (d == 128) ? jacobi_factor_kernel<128> : jacobi_factor_kernel<64>;
     cudaFuncSetAttribute(jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jac_smem);
 
-    // 1-2. key-response metric and factor (§4.1)
-    count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff, mat);
-    // warm start (C.1): subspace iteration from the previous factor; heads it
-    // cannot factor (or every head, without a previous state) take Jacobi
+    const bool sem_k = (p.flags & SPARSEPR_FLAG_SEMANTIC_KEYS) != 0;
+    const bool sem_q = (p.flags & SPARSEPR_FLAG_SEMANTIC_QUERIES) != 0;
+    const size_t n8 = (size_t)BH * N * d / 8;
     int32_t* coldK = at<int32_t>(ws, pl.o_warm) + 1;
     int32_t* coldQ = coldK + BH;
-    if (warm)
-        launch_warm_factor(mat, warm->F_K, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d), FK, pl.RKp, nullptr,
-                           coldK, warm->valid, BH, d, st);
-    count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d),
-                                                      nullptr, 16, warm ? coldK : nullptr);
-    project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
+    if (sem_k) {
+        // semantic K/V groups: k-means on the raw key rows (RKp = d)
+        count_launch(), identity_factor_kernel<<<BH, 256, 0, st>>>(FK, d, pl.RKp, nullptr);
+        count_launch(), raw_coords_kernel<T><<<grid_for(n8, 256), 256, 0, st>>>(K, n8, phiK);
+    } else {
+        // 1-2. key-response metric and factor (§4.1)
+        count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff,
+                                                                                                mat);
+        // warm start (C.1): subspace iteration from the previous factor; heads it
+        // cannot factor (or every head, without a previous state) take Jacobi
+        if (warm)
+            launch_warm_factor(mat, warm->F_K, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d), FK, pl.RKp,
+                               nullptr, coldK, warm->valid, BH, d, st);
+        count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr,
+                                                          1.f / sqrtf((float)d), nullptr, 16, warm ? coldK : nullptr);
+        project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
+    }
     // 3. paired K/V groups
     WarmInit wiK{}, wiQ{};
     if (warm) {
         wiK = WarmInit{warm->k_centroid, warm->n_groups, 1, FK, d, false, nullptr, 0.f, warm->valid};
-        wiQ = WarmInit{warm->q_centroid, warm->n_groups, 0, FQ, d, true, rq, p.eps_rms, warm->valid};
+        wiQ = WarmInit{warm->q_centroid, warm->n_groups, 0, FQ, d, !sem_q, rq, p.eps_rms, warm->valid};
     }
     kmeans_dispatch(pl.RKp, pl, p, ws, phiK, pl.Ck, 0, cenK, hnK, dbg ? out.debug_kv_scores : nullptr,
                     dbg ? out.debug_kv_hist : nullptr, -1, warm ? &wiK : nullptr, st);
@@ -825,15 +857,21 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
                                                         out.n_groups, 1, N, pl.Ck, d, out.k_centroid);
     count_launch(), group_mean_kernel<T><<<dim3(pl.Ck, BH), d, 0, st>>>(static_cast<const T*>(out.Vp), out.kv_offsets,
                                                         out.n_groups, 1, N, pl.Ck, d, out.v_centroid);
-    count_launch(), centroid_mean_kernel<<<BH, d, 0, st>>>(out.k_centroid, out.n_groups, pl.Ck, d, muK);
-    count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
-                                                                          out.n_groups, pl.Ck, d, mat);
-    if (warm)
-        launch_warm_factor(mat, warm->F_Q, pl.RQp, p.rQ, out.n_groups, 1.f, FQ, pl.RQp, rq, coldQ, warm->valid, BH, d,
-                           st);
-    count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16,
-                                                      warm ? coldQ : nullptr);
-    project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, at<DevStatus>(ws, pl.o_status), st);
+    if (sem_q) {
+        // semantic query groups: k-means on the raw query rows (RQp = d)
+        count_launch(), identity_factor_kernel<<<BH, 256, 0, st>>>(FQ, d, pl.RQp, rq);
+        count_launch(), raw_coords_kernel<T><<<grid_for(n8, 256), 256, 0, st>>>(Q, n8, phiQ);
+    } else {
+        count_launch(), centroid_mean_kernel<<<BH, d, 0, st>>>(out.k_centroid, out.n_groups, pl.Ck, d, muK);
+        count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
+                                                                              out.n_groups, pl.Ck, d, mat);
+        if (warm)
+            launch_warm_factor(mat, warm->F_Q, pl.RQp, p.rQ, out.n_groups, 1.f, FQ, pl.RQp, rq, coldQ, warm->valid,
+                               BH, d, st);
+        count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16,
+                                                          warm ? coldQ : nullptr);
+        project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, at<DevStatus>(ws, pl.o_status), st);
+    }
     // 5. query groups
     kmeans_dispatch(pl.RQp, pl, p, ws, phiQ, pl.Cq, 1, cenQ, hnQ, dbg ? out.debug_q_scores : nullptr,
                     dbg ? out.debug_q_hist : nullptr, kCtlItersK, warm ? &wiQ : nullptr, st);
@@ -844,7 +882,8 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), group_mean_kernel<T><<<dim3(pl.Cq, BH), d, 0, st>>>(static_cast<const T*>(out.Qp), out.q_offsets,
                                                         out.n_groups, 0, N, pl.Cq, d, out.q_centroid);
     // c_a (phi_Q space) into the query-centre buffer, then d_i (A.2)
-    count_launch(), group_mean_indirect_kernel<<<dim3(pl.Cq, BH), 64, 0, st>>>(phiQ, out.perm_q, out.q_offsets,
+    count_launch(), group_mean_indirect_kernel<<<dim3(pl.Cq, BH), pl.RQp > 64 ? pl.RQp : 64, 0, st>>>(
+                                                              phiQ, out.perm_q, out.q_offsets,
                                                               out.n_groups, N, pl.Cq, pl.RQp, cenQ);
     count_launch(), query_dist_kernel<<<grid_for((size_t)BH * N, 256), 256, 0, st>>>(phiQ, cenQ, out.q_label, BH, N,
                                                                      pl.Cq, pl.RQp, out.q_dist);

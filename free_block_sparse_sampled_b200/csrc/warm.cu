@@ -291,7 +291,8 @@ void launch_warm_init(const WarmInit& w, int R, const float* phi, int BH, int N,
         case 16: warm_init_r<16>(w, phi, BH, N, C, seed, stage, cen, hn, st); break;
         case 32: warm_init_r<32>(w, phi, BH, N, C, seed, stage, cen, hn, st); break;
         case 48: warm_init_r<48>(w, phi, BH, N, C, seed, stage, cen, hn, st); break;
-        default: warm_init_r<64>(w, phi, BH, N, C, seed, stage, cen, hn, st); break;
+        case 64: warm_init_r<64>(w, phi, BH, N, C, seed, stage, cen, hn, st); break;
+        default: warm_init_r<128>(w, phi, BH, N, C, seed, stage, cen, hn, st); break;
     }
 }
 

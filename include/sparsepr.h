@@ -68,6 +68,15 @@ typedef enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 } sparsepr_dtype;
                                           previous sparsepr_call with the same *p left in this
                                           workspace (see sparsepr_partition_warm); without such a
                                           state the call is cold */
+#define SPARSEPR_FLAG_SEMANTIC_KEYS 8  /* K/V groups by k-means on the raw key rows instead of the
+                                          key-response coordinates (paper §3 reference partition,
+                                          Table 2 baseline); F_K is then the d x d identity and
+                                          RKp = d */
+#define SPARSEPR_FLAG_SEMANTIC_QUERIES 16 /* query groups by k-means on the raw query rows (no
+                                          RMSNorm); d_i is the raw-space distance to the group
+                                          mean, F_Q the identity and RQp = d.  With
+                                          SEMANTIC_KEYS: the semantic partition; alone: Table 2's
+                                          key-response K/V variant */
 
 /* Problem statement (paper §3 / §4 notation).  All fields are read on the host. */
 typedef struct {
@@ -108,7 +117,8 @@ typedef struct {
     float* v_centroid;    /* [BH,Ck,d] vbar_b */
     float* q_dist;        /* [BH,N] d_i = |phi_Q(q_i) - c_a| by original row (A.2) */
     /* optional */
-    float* F_K;           /* [BH,d,RKp] key factor (columns beyond r_K' zero) */
+    float* F_K;           /* [BH,d,RKp] key factor (columns beyond r_K' zero); RKp = d with
+                             SPARSEPR_FLAG_SEMANTIC_KEYS, likewise RQp with SEMANTIC_QUERIES */
     float* F_Q;           /* [BH,d,RQp] query factor, RQp = min(rQ,d) rounded up to 16
                              (at least 32; columns beyond r_Q' zero) */
     float* phi_K;         /* [BH,N,RKp] key coordinates, RKp = r_K' rounded up to 16 (at least 32) */

@@ -210,20 +210,35 @@ def check_fit_and_apply(h, cfg):
     assert np.array_equal(h["out"][h["probe_idx"]], D)
 
 
-def check_partition_floats(h, cfg, q, k, v, warm=None):
+def _tf32(x):
+    """Round fp64 values (fp32-representable) to TF32, nearest even."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + np.uint64(0xFFF) + ((u >> np.uint64(13)) & np.uint64(1))) & np.uint64(0xFFFFE000)
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, semantic_queries=False):
     """Float outputs of the partition against fp64 recomputation from the
     GPU's own integer decisions.  ``warm`` (F_K, F_Q of the state a warm call
-    started from, fp64) switches the factor references to the warm factor."""
+    started from, fp64) switches the factor references to the warm factor;
+    a semantic side has the raw rows (TF32-rounded) as coordinates and the
+    identity as its factor."""
     kl, ql = h["kv_label"], h["q_label"]
     np.testing.assert_allclose(h["k_centroid"], O.group_means(k, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
     np.testing.assert_allclose(h["v_centroid"], O.group_means(v, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
     np.testing.assert_allclose(h["q_centroid"], O.group_means(q, ql, h["Cq"]), rtol=1e-4, atol=1e-5)
     # phi_K = K F_K with the GPU factor; phi_Q = RMSNorm(q F_Q) with its factor
     rq = O.query_rank(cfg.rQ, cfg.d, h["Ck"])
-    np.testing.assert_allclose(h["phi_K"], k @ h["F_K"], rtol=TOL_TF32, atol=1e-4 * np.abs(h["phi_K"]).max())
-    z = q @ h["F_Q"]
-    rms = np.sqrt((z * z).sum(1) / rq)
-    np.testing.assert_allclose(h["phi_Q"], z / np.maximum(rms, cfg.eps_rms)[:, None], rtol=TOL_TF32, atol=1e-4)
+    if semantic_keys:
+        assert np.array_equal(h["phi_K"], _tf32(k)) and np.array_equal(h["F_K"], np.eye(cfg.d))
+    else:
+        np.testing.assert_allclose(h["phi_K"], k @ h["F_K"], rtol=TOL_TF32, atol=1e-4 * np.abs(h["phi_K"]).max())
+    if semantic_queries:
+        assert np.array_equal(h["phi_Q"], _tf32(q)) and np.array_equal(h["F_Q"], np.eye(cfg.d))
+    else:
+        z = q @ h["F_Q"]
+        rms = np.sqrt((z * z).sum(1) / rq)
+        np.testing.assert_allclose(h["phi_Q"], z / np.maximum(rms, cfg.eps_rms)[:, None], rtol=TOL_TF32, atol=1e-4)
     _, dist = O.query_distances(h["phi_Q"], ql, h["Cq"])
     np.testing.assert_allclose(h["q_dist"], dist, rtol=1e-4, atol=1e-5)
     # metric factors: F F^T reproduces the (truncated) metric
@@ -233,7 +248,7 @@ def check_partition_floats(h, cfg, q, k, v, warm=None):
     r = min(cfg.rK, cfg.d, len(idx))
     ref = U[:, :r] @ np.diag(w[:r]) @ U[:, :r].T / cfg.d
     FK = h["F_K"]
-    gap_ok = r == cfg.d or (w[r - 1] - w[r]) > 1e-2 * w[0]
+    gap_ok = (r == cfg.d or (w[r - 1] - w[r]) > 1e-2 * w[0]) and not semantic_keys
     Fw = None if warm is None else O.warm_factor(MK, warm["F_K"], r, 1.0 / math.sqrt(cfg.d))
     if Fw is not None:
         ref = Fw @ Fw.T
@@ -248,7 +263,7 @@ def check_partition_floats(h, cfg, q, k, v, warm=None):
     if Fwq is not None:
         refq = Fwq @ Fwq.T
         assert np.abs(FQ @ FQ.T - refq).max() <= 2e-4 * np.abs(refq).max(), "warm F_Q"
-    elif rq >= int((wq > 1e-9 * wq[0]).sum()) or (wq[rq - 1] - wq[rq]) > 1e-2 * wq[0]:
+    elif not semantic_queries and (rq >= int((wq > 1e-9 * wq[0]).sum()) or (wq[rq - 1] - wq[rq]) > 1e-2 * wq[0]):
         assert np.abs(FQ @ FQ.T - refq).max() <= 2e-4 * np.abs(refq).max()
     # routing scores vs the direct sum on the GPU's groups and centroids
     s_ref = O.routing_score(h["q_centroid"], k, v, h["k_centroid"], h["v_centroid"], kl)
