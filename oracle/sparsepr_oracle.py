@@ -62,6 +62,21 @@ R16 Semantic partition (§3's reference partition, Table 2's baseline): the
     the raw-space query-group mean.  Routing, probes, fit and apply are
     unchanged.  Table 2's key-response variant keeps the response K/V groups
     and takes semantic query groups.
+R17 Probe variants (Table 4): "random" = M distinct rows drawn uniformly by
+    Floyd's sampling algorithm (Bentley & Floyd 1987) from a SplitMix64
+    stream seeded by mix(seed xor mix((bh+1) gamma xor 0x50524F4245)): for
+    s = 0..M-1, j = N-M+s, draw s+1 gives t = floor(u (j+1) / 2^32) from its
+    top 32 bits u, and the sample gains t, or j when t is already in it.
+    "uniform" = rows floor((2j+1) N / (2M)), evenly spaced over the
+    row-major (t, y, x) grid.  Both keep A.2's coverage weights
+    w_p = |G_a| / m_a with m_a the probes that fall in group a, and list
+    probes by group, then by index.  With M >= N every variant takes all rows.
+R18 Correction families (D.4): with the same standardisation, centring and
+    weights, "mean" has B = 0, "scalar" B = a I with
+    a = tr(Xbar^T W Rbar) / (tr(Xbar^T W Xbar) + lambda d), "diagonal"
+    B = diag(b) with b_j = (Xbar^T W Rbar)_jj / ((Xbar^T W Xbar)_jj + lambda);
+    each minimises the weighted squared error plus lambda |B|_F^2 over its
+    family.  Rank r truncation (D.3) replaces B by B V_r V_r^T.
 """
 
 from __future__ import annotations
@@ -414,6 +429,33 @@ def probe_select(q_labels: np.ndarray, d_i: np.ndarray, m: np.ndarray) -> np.nda
     return np.concatenate(out).astype(np.int64) if out else np.zeros(0, np.int64)
 
 
+PROBE_STREAM = 0x50524F4245
+
+
+def random_probes(seed: int, bh: int, N: int, M: int) -> np.ndarray:
+    """R17: Floyd's algorithm; returns the sampled rows in increasing order."""
+    base = splitmix64_mix((seed & _M64) ^ splitmix64_mix((((bh + 1) * _GAMMA) & _M64) ^ PROBE_STREAM))
+    draws = splitmix64_outputs(base, M)
+    chosen = set()
+    for s_, x in enumerate(draws):
+        j = N - M + s_
+        t = ((x >> 32) * (j + 1)) >> 32
+        chosen.add(j if t in chosen else t)
+    return np.array(sorted(chosen), dtype=np.int64)
+
+
+def uniform_probes(N: int, M: int) -> np.ndarray:
+    """R17: rows floor((2j+1) N / (2M)), j = 0..M-1."""
+    return np.array([((2 * j + 1) * N) // (2 * M) for j in range(M)], dtype=np.int64)
+
+
+def listed_by_group(rows: np.ndarray, q_labels: np.ndarray, C: int):
+    """Probe rows listed by group, then by index, and m_a per group."""
+    order = np.lexsort((rows, q_labels[rows]))
+    P = rows[order]
+    return P, np.bincount(q_labels[P], minlength=C).astype(np.int64)
+
+
 def coverage_weights(probe_groups: np.ndarray, q_sizes: np.ndarray, m: np.ndarray, M: int):
     """A.2 w_p = |G_a| / m_a;  A.3 alpha_p = w_p / sum w;  w~_p = M w_p / sum w."""
     w = q_sizes[probe_groups] / m[probe_groups]
@@ -446,6 +488,27 @@ def ridge_fit(X: np.ndarray, R: np.ndarray, alpha: np.ndarray, wt: np.ndarray,
         raise NumericError("Gram matrix is not positive definite") from e
     B = np.linalg.solve(L.T, np.linalg.solve(L, rhs))
     return {"mu_X": mu_X, "sigma": sigma, "mu_R": mu_R, "B": B, "Xbar": Xb, "Rbar": Rb}
+
+
+def restricted_fit(X: np.ndarray, R: np.ndarray, alpha: np.ndarray, wt: np.ndarray, lam: float,
+                   eps_std: float, family: str) -> Dict[str, np.ndarray]:
+    """R18: the D.4 correction families on ridge_fit's standardised features."""
+    f = ridge_fit(X, R, alpha, wt, lam, eps_std)
+    if family == "full":
+        return f
+    Xb, Rb = f["Xbar"], f["Rbar"]
+    d = X.shape[1]
+    gx = (wt[:, None] * Xb * Xb).sum(axis=0)          # diagonal of Xbar^T W Xbar
+    gr = (wt[:, None] * Xb * Rb).sum(axis=0)          # diagonal of Xbar^T W Rbar
+    if family == "diagonal":
+        B = np.diag(gr / (gx + lam))
+    elif family == "scalar":
+        B = (gr.sum() / (gx.sum() + lam * d)) * np.eye(d)
+    elif family == "mean":
+        B = np.zeros((d, d))
+    else:
+        raise ValueError(family)
+    return {**f, "B": B}
 
 
 def residual_span_projection(B: np.ndarray, Rbar: np.ndarray, wt: np.ndarray,
@@ -492,13 +555,17 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
                   lam: float, Cq: int, Ck: int, rK: int, rQ: int, kmeans_iters: int,
                   kmeans_tol: float, eps_rms: float = 1e-6, eps_std: float = 1e-6,
                   want_dense: bool = False, warm: Optional[Dict[str, np.ndarray]] = None,
-                  partition: str = "response") -> Dict[str, object]:
+                  partition: str = "response", probes: str = "stratified", correction: str = "full",
+                  residual_rank: int = 0) -> Dict[str, object]:
     """One SparsePR call on one head, steps in the paper's order:
     partition (§4.1) -> route (§4.3, B.3) -> sparse attention (Eq. 2) ->
     probes (A.2) -> weighted ridge (A.3) -> corrected output (§4.2).
     ``warm`` (F_K, F_Q, kbar, qbar of the previous call) selects the warm
     start of R13-R15; the caller also lowers ``kmeans_iters``.
-    ``partition``: "response" (§4.1), "semantic" or "key_response" (R16)."""
+    ``partition``: "response" (§4.1), "semantic" or "key_response" (R16).
+    ``probes``: "stratified" (A.2), "random" or "uniform" (R17);
+    ``correction``: "full", "diagonal", "scalar" or "mean" (R18);
+    ``residual_rank``: 0 (no truncation) or r (D.3)."""
     if partition not in ("response", "semantic", "key_response"):
         raise ValueError(partition)
     semantic_keys = partition == "semantic"
@@ -559,12 +626,18 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     O_sp = sparse_attention(q, k, v, q_labels, kv_labels, mask)
     # 10. probes
     Mp = min(M, N)
-    m = probe_allocation(q_sizes, Mp, N)
-    P = probe_select(q_labels, d_i, m)
+    if probes == "stratified" or Mp >= N:
+        m = probe_allocation(q_sizes, Mp, N)
+        P = probe_select(q_labels, d_i, m)
+    else:
+        rows = random_probes(seed, bh, N, Mp) if probes == "random" else uniform_probes(N, Mp)
+        P, m = listed_by_group(rows, q_labels, Cq2)
     w, alpha, wt = coverage_weights(q_labels[P], q_sizes, m, Mp)
     O_dense_P = dense_attention(q[P], k, v)
     # 11. fit and 13. output
-    fit = ridge_fit(O_sp[P], O_dense_P - O_sp[P], alpha, wt, lam, eps_std) if Mp > 0 else None
+    fit = restricted_fit(O_sp[P], O_dense_P - O_sp[P], alpha, wt, lam, eps_std, correction) if Mp > 0 else None
+    if fit is not None and residual_rank > 0:
+        fit = {**fit, "B": residual_span_projection(fit["B"], fit["Rbar"], wt, residual_rank)}
     O_hat = apply_correction(O_sp, P, O_dense_P, fit) if fit is not None else O_sp.copy()
 
     out.update(sample_idx=idx, M_K=M_K, F_K=F_K, phi_K=phi_K, kv_labels=kv_labels,

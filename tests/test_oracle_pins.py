@@ -693,3 +693,95 @@ def test_semantic_call_is_rotation_invariant():
     b = O.sparsepr_head(q @ R, k @ R, v, bh=0, partition="semantic", **_kw(Cq=5, Ck=3))
     assert np.array_equal(a["kv_labels"], b["kv_labels"]) and np.array_equal(a["q_labels"], b["q_labels"])
     np.testing.assert_allclose(a["O"], b["O"], atol=1e-10)
+
+
+# ------------------------------------------------ probe variants and families
+def test_random_probes_are_a_uniform_sample():
+    """Floyd's algorithm draws every M-subset with equal probability: all 20
+    subsets of 3 rows out of 6 appear equally often over 20000 seeds."""
+    counts = {}
+    for seed in range(20000):
+        P = O.random_probes(seed, 0, 6, 3)
+        assert len(P) == 3 and len(set(P.tolist())) == 3 and P.min() >= 0 and P.max() < 6
+        counts[tuple(P)] = counts.get(tuple(P), 0) + 1
+    assert len(counts) == 20
+    exp, sd = 1000.0, math.sqrt(20000 * (1 / 20) * (19 / 20))
+    assert all(abs(c - exp) < 5 * sd for c in counts.values())
+    assert np.array_equal(O.random_probes(1, 3, 9, 9), np.arange(9))
+    assert not np.array_equal(O.random_probes(1, 0, 1000, 10), O.random_probes(1, 1, 1000, 10))
+
+
+def test_uniform_probes_closed_form():
+    assert O.uniform_probes(10, 4).tolist() == [1, 3, 6, 8]
+    assert np.array_equal(O.uniform_probes(7, 7), np.arange(7))
+    P = O.uniform_probes(75600, 512)
+    assert len(np.unique(P)) == 512 and np.all(np.diff(P) >= 147)
+
+
+def test_probes_listed_by_group_then_index():
+    labels = np.array([2, 0, 1, 0, 2, 1, 0])
+    P, m = O.listed_by_group(np.array([6, 0, 3, 4, 5]), labels, 3)
+    assert P.tolist() == [3, 6, 5, 0, 4] and m.tolist() == [2, 1, 2]
+
+
+def _fit_problem(seed=90, M=60, d=5):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((M, d)) * rng.uniform(0.5, 2.0, d) + rng.standard_normal(d)
+    R = rng.standard_normal((M, d))
+    w = rng.uniform(0.5, 2.0, M)
+    alpha = w / w.sum()
+    return X, R, alpha, M * alpha
+
+
+@pytest.mark.parametrize("family", ["diagonal", "scalar"])
+def test_restricted_fits_minimise_the_penalised_objective(family):
+    """D.4: each family minimises sum_p w~_p |Rbar_p - Xbar_p B|^2 + lambda |B|_F^2
+    over its own parameters (zero derivative by central differences)."""
+    X, R, alpha, wt = _fit_problem()
+    lam = 0.7
+    f = O.restricted_fit(X, R, alpha, wt, lam, 1e-6, family)
+    Xb, Rb, B = f["Xbar"], f["Rbar"], f["B"]
+    d = X.shape[1]
+
+    def obj(Bm):
+        E = Rb - Xb @ Bm
+        return float((wt[:, None] * E * E).sum() + lam * (Bm * Bm).sum())
+
+    params = [np.diag(np.eye(d)[j]) for j in range(d)] if family == "diagonal" else [np.eye(d)]
+    for D in params:
+        h = 1e-5
+        g = (obj(B + h * D) - obj(B - h * D)) / (2 * h)
+        assert abs(g) < 1e-6 * max(1.0, obj(B))
+    assert np.count_nonzero(B - np.diag(np.diag(B))) == 0
+    if family == "scalar":
+        assert np.allclose(B, B[0, 0] * np.eye(d))
+
+
+def test_restricted_fits_recover_planted_maps_and_mean_only():
+    X, _, alpha, wt = _fit_problem(91)
+    f0 = O.ridge_fit(X, np.zeros_like(X), alpha, wt, 1.0, 1e-6)
+    Xb = f0["Xbar"]
+    c = np.array([0.5, -1.0, 2.0, 0.0, 3.0])
+    fd = O.restricted_fit(X, Xb * c, alpha, wt, 0.0, 1e-6, "diagonal")      # residual = Xbar diag(c)
+    np.testing.assert_allclose(np.diag(fd["B"]), c, atol=1e-10)
+    fs = O.restricted_fit(X, 1.7 * Xb, alpha, wt, 0.0, 1e-6, "scalar")
+    np.testing.assert_allclose(fs["B"], 1.7 * np.eye(5), atol=1e-10)
+    fm = O.restricted_fit(X, Xb * c + 3.0, alpha, wt, 1.0, 1e-6, "mean")
+    assert not fm["B"].any()
+    np.testing.assert_allclose(fm["mu_R"], alpha @ (Xb * c) + 3.0, atol=1e-12)
+
+
+def test_whole_call_variants_on_tiny():
+    w, q, k, v = _tiny_head()
+    kw = O.workload_kwargs(w)
+    base = O.sparsepr_head(q, k, v, bh=0, want_dense=True, **kw)
+    for probes in ("random", "uniform"):
+        r = O.sparsepr_head(q, k, v, bh=0, probes=probes, **kw)
+        assert len(np.unique(r["probes"])) == w.M and r["m"].sum() == w.M
+        assert abs(r["wt"].sum() - w.M) < 1e-9
+        np.testing.assert_array_equal(r["O_sp"], base["O_sp"])     # the sparse base does not depend on probes
+    full_rank = O.sparsepr_head(q, k, v, bh=0, residual_rank=w.d, **kw)
+    np.testing.assert_allclose(full_rank["O"], base["O"], atol=1e-9)   # R8: full rank is the identity
+    mean = O.sparsepr_head(q, k, v, bh=0, correction="mean", **kw)
+    unp = np.setdiff1d(np.arange(w.N), mean["probes"])
+    np.testing.assert_allclose(mean["O"][unp], base["O_sp"][unp] + mean["fit"]["mu_R"][None, :], atol=1e-12)
