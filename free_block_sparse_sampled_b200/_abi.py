@@ -16,6 +16,8 @@ FLAG_SIMT_ATTENTION = 2
 FLAG_WARM_START = 4
 FLAG_SEMANTIC_KEYS = 8
 FLAG_SEMANTIC_QUERIES = 16
+PROBES = {"stratified": 0, "random": 1, "uniform": 2}
+CORRECTIONS = {"full": 0, "diagonal": 1, "scalar": 2, "mean": 3}
 
 EXPORTED = ["sparsepr_status_string", "sparsepr_validate", "sparsepr_workspace_size",
             "sparsepr_partition", "sparsepr_route", "sparsepr_attention", "sparsepr_probe_fit",
@@ -36,7 +38,8 @@ class Params(ctypes.Structure):
                 ("Ck", ctypes.c_int32), ("rK", ctypes.c_int32), ("rQ", ctypes.c_int32),
                 ("kmeans_iters", ctypes.c_int32), ("kmeans_tol", ctypes.c_double),
                 ("seed", ctypes.c_uint64), ("block", ctypes.c_int32), ("eps_rms", ctypes.c_float),
-                ("eps_std", ctypes.c_float), ("flags", ctypes.c_int32)]
+                ("eps_std", ctypes.c_float), ("flags", ctypes.c_int32), ("probe_select", ctypes.c_int32),
+                ("correction", ctypes.c_int32), ("residual_rank", ctypes.c_int32)]
 
 
 PARTITION_FIELDS = ["Qp", "Kp", "Vp", "q_label", "kv_label", "perm_q", "perm_kv", "pos_q", "q_offsets",

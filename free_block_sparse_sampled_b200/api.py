@@ -42,6 +42,9 @@ class SparsePRConfig:
     eps_rms: float = 1e-6
     eps_std: float = 1e-6
     flags: int = 0
+    probe_select: str = "stratified"   # "stratified" (A.2), "random" or "uniform" (Table 4)
+    correction: str = "full"           # "full", "diagonal", "scalar" or "mean" (D.4)
+    residual_rank: int = 0             # 0: no truncation; r: rank-r residual projection (D.3)
 
     @classmethod
     def from_workload(cls, w, **kw) -> "SparsePRConfig":
@@ -82,7 +85,8 @@ class SparsePRConfig:
                         A.BF16 if self.dtype == "bf16" else A.F32, float(self.density), self.M, self.Ms,
                         float(self.lam), self.Cq, self.Ck, self.rK, self.rQ, self.kmeans_iters,
                         float(self.kmeans_tol), int(self.seed) & ((1 << 64) - 1), self.block,
-                        float(self.eps_rms), float(self.eps_std), self.flags)
+                        float(self.eps_rms), float(self.eps_std), self.flags, A.PROBES[self.probe_select],
+                        A.CORRECTIONS[self.correction], int(self.residual_rank))
 
 
 def validate(cfg: SparsePRConfig) -> int:

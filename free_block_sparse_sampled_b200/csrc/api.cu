@@ -88,6 +88,8 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_lbar = bump(c, BH * Cq * Ck * 4);
     pl.o_vv = bump(c, BH * Ck * 4);
     pl.o_warm = bump(c, (1 + 2 * BH) * 4);
+    pl.o_pbits = bump(c, BH * ((N + 31) / 32) * 4);
+    pl.o_S = bump(c, p.residual_rank > 0 ? BH * d * d * 8 : 256);
     // outputs owned by the workspace (fused call)
     pl.o_Qp = bump(c, BH * N * d * es);
     pl.o_Kp = bump(c, BH * N * d * es);
@@ -224,6 +226,8 @@ sparsepr_status sparsepr_validate(const sparsepr_params* p) {
     if (p->kmeans_iters < 1 || p->kmeans_iters > 1000 || !(p->kmeans_tol >= 0.0)) return SPARSEPR_INVALID_ARG;
     if (!(p->eps_rms > 0.f) || !(p->eps_std >= 0.f)) return SPARSEPR_INVALID_ARG;
     if (p->block != 64 && p->block != 128) return SPARSEPR_INVALID_ARG;
+    if (p->probe_select < 0 || p->probe_select > 2 || p->correction < 0 || p->correction > 3) return SPARSEPR_INVALID_ARG;
+    if (p->residual_rank < 0 || p->residual_rank > p->d) return SPARSEPR_INVALID_ARG;
     if (p->d != 64 && p->d != 128) return SPARSEPR_UNSUPPORTED;
     if (p->Cq > kMaxGroups || p->Ck > kMaxGroups) return SPARSEPR_UNSUPPORTED;
     if (p->rK > kMaxRank || p->rQ > kMaxRank) return SPARSEPR_UNSUPPORTED;

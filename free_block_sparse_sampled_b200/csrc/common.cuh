@@ -109,7 +109,9 @@ struct Plan {
     size_t o_status, o_ctl, o_mat, o_FK, o_FQ, o_rq, o_phiK, o_phiQ, o_cenK, o_hnK, o_cenQ, o_hnQ,
         o_raw, o_hist, o_sorted, o_offs, o_newid, o_muK, o_t1, o_t2, o_mloc, o_pslot, o_palloc,
         o_poff, o_psum, o_qprobe, o_work, o_fstat, o_G, o_rhs, o_vh, o_vmax, o_vscale, o_qsplit, o_uw, o_lbar, o_vv,
-        o_warm;   // [0]: kWarmMagic when the fused call's state is complete; [1 + bh], [1 + BH + bh]: cold K / Q factor
+        o_warm,   // [0]: kWarmMagic when the fused call's state is complete; [1 + bh], [1 + BH + bh]: cold K / Q factor
+        o_pbits,  // [BH][ceil(N/32)] probe membership bits (random / uniform probes)
+        o_S;      // [BH][d][d] fp64 Rbar^T W Rbar (rank truncation)
     // outputs owned by the workspace for sparsepr_call
     size_t o_Qp, o_Kp, o_Vp, o_qlab, o_kvlab, o_permq, o_permk, o_posq, o_qoff, o_kvoff, o_ng, o_its,
         o_qcen, o_kcen, o_vcen, o_qdist, o_score, o_mask, o_selc, o_selg, o_pairs, o_pidx, o_pgrp,

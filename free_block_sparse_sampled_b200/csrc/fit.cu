@@ -67,18 +67,20 @@ __global__ void fit_stats_kernel(const float* __restrict__ Xs, const float* __re
     mu_r[(size_t)bh * d + j] = (float)mr;
 }
 
-// Rows i0..i0+7 of G = Xbar^T W Xbar + lambda I and of RHS = Xbar^T W Rbar.
-// Probes are taken kGramChunk at a time: their weights times the block's
-// eight standardised rows are staged in shared memory, then each thread
-// accumulates its column j (probes in index order).
+// Rows i0..i0+7 of G = Xbar^T W Xbar + lambda I and of RHS = Xbar^T W Rbar
+// (and, with S, of Rbar^T W Rbar).  Probes are taken kGramChunk at a time:
+// their weights times the block's eight standardised rows are staged in
+// shared memory, then each thread accumulates its column j (probes in index
+// order).
 constexpr int kGramChunk = 1024;
 __global__ void fit_gram_kernel(const float* __restrict__ Xs, const float* __restrict__ Xd,
                                 const int32_t* __restrict__ probe_group, const int32_t* __restrict__ alloc,
                                 const int32_t* __restrict__ q_off, const int32_t* __restrict__ psum, int Cq, int Mp,
                                 int d, double lambda, const double* __restrict__ fstat, double* __restrict__ G,
-                                double* __restrict__ rhs) {
+                                double* __restrict__ rhs, double* __restrict__ S) {
     constexpr int RI = 8;
-    extern __shared__ double xbi[];   // [kGramChunk][RI] W_p * Xbar[p][i0 + u]
+    extern __shared__ double xbi[];   // [kGramChunk][RI] W_p * Xbar[p][i0 + u]; then W_p * Rbar (with S)
+    double* rbi = xbi + kGramChunk * RI;
     const int bh = blockIdx.y, i0 = blockIdx.x * RI, j = threadIdx.x;
     const float* X = Xs + (size_t)bh * Mp * d;
     const float* Dp = Xd + (size_t)bh * Mp * d;
@@ -88,16 +90,18 @@ __global__ void fit_gram_kernel(const float* __restrict__ Xs, const float* __res
     const double* fs = fstat + (size_t)bh * 3 * d;
     const double sw = (double)psum[bh];
     const double mxj = fs[j], sgj = fs[d + j], mrj = fs[2 * d + j];
-    double g[RI], h[RI];
+    double g[RI], h[RI], sr[RI];
 #pragma unroll
-    for (int u = 0; u < RI; ++u) g[u] = h[u] = 0.0;
+    for (int u = 0; u < RI; ++u) g[u] = h[u] = sr[u] = 0.0;
     for (int c0 = 0; c0 < Mp; c0 += kGramChunk) {
         const int n = min(kGramChunk, Mp - c0);
         __syncthreads();   // the previous chunk is consumed
         for (int e = j; e < n * RI; e += blockDim.x) {
             const int p = c0 + e / RI, u = e % RI;
             const double wt = (double)Mp * probe_alpha(p, pg, al, qo, sw);
-            xbi[e] = wt * (((double)X[(size_t)p * d + i0 + u] - fs[i0 + u]) / fs[d + i0 + u]);
+            const double xv = (double)X[(size_t)p * d + i0 + u];
+            xbi[e] = wt * ((xv - fs[i0 + u]) / fs[d + i0 + u]);
+            if (S != nullptr) rbi[e] = wt * (((double)Dp[(size_t)p * d + i0 + u] - xv) - fs[2 * d + i0 + u]);
         }
         __syncthreads();
         for (int q = 0; q < n; ++q) {
@@ -111,6 +115,10 @@ __global__ void fit_gram_kernel(const float* __restrict__ Xs, const float* __res
                 g[u] += xb * xbj;
                 h[u] += xb * rbj;
             }
+            if (S != nullptr) {
+#pragma unroll
+                for (int u = 0; u < RI; ++u) sr[u] += rbi[q * RI + u] * rbj;
+            }
         }
     }
 #pragma unroll
@@ -118,6 +126,78 @@ __global__ void fit_gram_kernel(const float* __restrict__ Xs, const float* __res
         const int i = i0 + u;
         G[((size_t)bh * d + i) * d + j] = g[u] + (i == j ? lambda : 0.0);
         rhs[((size_t)bh * d + i) * d + j] = h[u];
+        if (S != nullptr) S[((size_t)bh * d + i) * d + j] = sr[u];
+    }
+}
+
+// Restricted families (D.4) from the diagonals of G = Xbar^T W Xbar + lambda I
+// and RHS = Xbar^T W Rbar: diagonal b_j = RHS_jj / G_jj, scalar
+// a = tr(RHS) / tr(G) (tr G carries lambda d), mean-only B = 0.  One thread per
+// channel j.
+__global__ void fit_restricted_kernel(const double* __restrict__ G, const double* __restrict__ rhs, int d,
+                                      int family, float* __restrict__ Bout) {
+    __shared__ double red[2][32];
+    const int bh = blockIdx.x, j = threadIdx.x, lane = j & 31, wid = j >> 5;
+    const double gjj = G[((size_t)bh * d + j) * d + j];
+    const double hjj = rhs[((size_t)bh * d + j) * d + j];
+    double sg = gjj, sh = hjj;
+    for (int o = 16; o > 0; o >>= 1) {
+        sg += __shfl_xor_sync(0xffffffffu, sg, o);
+        sh += __shfl_xor_sync(0xffffffffu, sh, o);
+    }
+    if (lane == 0) {
+        red[0][wid] = sg;
+        red[1][wid] = sh;
+    }
+    __syncthreads();
+    double tg = 0.0, th = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {   // fixed order
+        tg += red[0][w];
+        th += red[1][w];
+    }
+    double bj = 0.0;
+    if (family == SPARSEPR_CORRECTION_DIAGONAL) bj = hjj / gjj;
+    else if (family == SPARSEPR_CORRECTION_SCALAR) bj = th / tg;
+    float* Bh = Bout + (size_t)bh * d * d;
+    for (int i = 0; i < d; ++i) Bh[(size_t)i * d + j] = (i == j) ? (float)bj : 0.f;
+}
+
+// S (fp64, symmetric) to fp32 for the Jacobi eigen-factor.
+__global__ void to_f32_kernel(const double* __restrict__ S, size_t n, float* __restrict__ out) {
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x)
+        out[e] = (float)S[e];
+}
+
+// Rank truncation (D.3): B <- B U_r U_r^T, U_r the unit-normalised nonzero
+// leading columns of the eigen-factor Fv (d x d, columns u_c sqrt(lambda_c)).
+__global__ void fit_project_kernel(const float* __restrict__ Fv, int d, int r, float* __restrict__ Bm) {
+    extern __shared__ float pj[];
+    float* U = pj;               // [d][r]
+    float* T = pj + d * r;       // [d][r] = B U
+    __shared__ float inv[128];
+    const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const float* Fh = Fv + (size_t)bh * d * d;
+    float* Bh = Bm + (size_t)bh * d * d;
+    for (int c = tid; c < r; c += nt) {
+        double ss = 0.0;
+        for (int k = 0; k < d; ++k) ss += (double)Fh[(size_t)k * d + c] * Fh[(size_t)k * d + c];
+        inv[c] = ss > 0.0 ? (float)(1.0 / sqrt(ss)) : 0.f;
+    }
+    __syncthreads();
+    for (int e = tid; e < d * r; e += nt) U[e] = Fh[(size_t)(e / r) * d + (e % r)] * inv[e % r];
+    __syncthreads();
+    for (int e = tid; e < d * r; e += nt) {
+        const int i = e / r, c = e % r;
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) acc += (double)Bh[(size_t)i * d + k] * U[k * r + c];
+        T[e] = (float)acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < d * d; e += nt) {
+        const int i = e / d, j = e % d;
+        double acc = 0.0;
+        for (int c = 0; c < r; ++c) acc += (double)T[i * r + c] * U[j * r + c];
+        Bh[e] = (float)acc;
     }
 }
 
@@ -275,14 +355,31 @@ sparsepr_status run_fit(const sparsepr_params& p, const Plan& pl, const sparsepr
     count_launch(), fit_stats_kernel<<<BH, d, 0, st>>>(probe_sparse, probe_dense, r.probe_group, alloc, part.q_offsets,
                                        part.n_groups, psum, pl.Cq, Mp, d, p.eps_std, fstat, f.mu_x, f.sigma,
                                        f.mu_r);
-    const size_t gsmem = (size_t)kGramChunk * 8 * sizeof(double);   // 8 staged rows per probe of a chunk
+    const bool trunc = p.residual_rank > 0 && p.residual_rank < d;
+    double* S = trunc ? at<double>(ws, pl.o_S) : nullptr;
+    // 8 staged rows per probe of a chunk (twice with S)
+    const size_t gsmem = (size_t)kGramChunk * 8 * sizeof(double) * (trunc ? 2 : 1);
     cudaFuncSetAttribute(fit_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem);
     count_launch(), fit_gram_kernel<<<dim3(d / 8, BH), d, gsmem, st>>>(probe_sparse, probe_dense, r.probe_group, alloc,
                                                                        part.q_offsets, psum, pl.Cq, Mp, d, p.lambda,
-                                                                       fstat, G, rhs);
-    const size_t smem = (size_t)d * (d + 1) * sizeof(double);
-    cudaFuncSetAttribute(fit_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    count_launch(), fit_solve_kernel<<<BH, d, smem, st>>>(G, rhs, d, f.B, status);
+                                                                       fstat, G, rhs, S);
+    if (p.correction == SPARSEPR_CORRECTION_FULL) {
+        const size_t smem = (size_t)d * (d + 1) * sizeof(double);
+        cudaFuncSetAttribute(fit_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        count_launch(), fit_solve_kernel<<<BH, d, smem, st>>>(G, rhs, d, f.B, status);
+    } else {
+        count_launch(), fit_restricted_kernel<<<BH, d, 0, st>>>(G, rhs, d, p.correction, f.B);
+    }
+    if (trunc) {
+        // leading right singular vectors of W^1/2 Rbar = eigenvectors of Rbar^T W Rbar
+        float* Sf = at<float>(ws, pl.o_mat);
+        float* Fv = reinterpret_cast<float*>(G);       // G is consumed; d x d floats per head fit in it
+        count_launch(), to_f32_kernel<<<(BH * d * d + 255) / 256, 256, 0, st>>>(S, (size_t)BH * d * d, Sf);
+        launch_jacobi_factor(Sf, Fv, d, p.residual_rank, BH, d, st);
+        const size_t psmem = (size_t)2 * d * p.residual_rank * sizeof(float);
+        cudaFuncSetAttribute(fit_project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+        count_launch(), fit_project_kernel<<<BH, 256, psmem, st>>>(Fv, d, p.residual_rank, f.B);
+    }
     return cuda_status(cudaGetLastError());
 }
 

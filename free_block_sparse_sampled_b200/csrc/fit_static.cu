@@ -89,6 +89,10 @@ sparsepr_status sparsepr_probe_fit_static(const sparsepr_params* p, const sparse
     if (p == nullptr) return SPARSEPR_INVALID_ARG;
     const sparsepr_status v = sparsepr_validate(p);
     if (v != SPARSEPR_OK) return v;
+    if (p->residual_rank > 0) {
+        snprintf(last_error_buffer(), 256, "sparsepr_probe_fit_static: rank truncation needs a workspace");
+        return SPARSEPR_UNSUPPORTED;
+    }
     Plan pl;
     if (!make_plan(*p, pl)) return SPARSEPR_INVALID_ARG;
     if (!part || !part->q_offsets || !part->n_groups || !route || !route->probe_alloc ||

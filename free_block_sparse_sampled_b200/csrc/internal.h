@@ -36,6 +36,9 @@ struct WarmInit {
 };
 void launch_warm_init(const WarmInit& w, int R, const float* phi, int BH, int N, int C, uint64_t seed, int stage,
                       float* cen, float* hn, cudaStream_t st);
+// Leading r eigenpairs of BH symmetric d x d fp32 matrices: F[:, c] = u_c
+// sqrt(max(lambda_c, 0)) for c < r, zero up to Rp (parallel cyclic Jacobi).
+void launch_jacobi_factor(const float* A, float* F, int Rp, int r, int BH, int d, cudaStream_t st);
 // *word = value, in stream order (one thread).
 void launch_set_word(int32_t* word, int32_t value, cudaStream_t st);
 // Warm metric factor; heads it cannot factor get cold[bh] = 1 (else 0).

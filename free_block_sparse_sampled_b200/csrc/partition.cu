@@ -697,6 +697,13 @@ __global__ void identity_factor_kernel(float* __restrict__ F, int d, int Rp, int
 }
 
 // ================================================================ host side
+void launch_jacobi_factor(const float* A, float* F, int Rp, int r, int BH, int d, cudaStream_t st) {
+    const size_t jac_smem = (size_t)(2 * d * (d + 1) + 4 * (d / 2) + 64) * sizeof(float) + (size_t)d * sizeof(int);
+    auto jacobi = (d == 128) ? jacobi_factor_kernel<128> : jacobi_factor_kernel<64>;
+    cudaFuncSetAttribute(jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)jac_smem);
+    count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(A, F, Rp, r, nullptr, 1.f, nullptr, 16, nullptr);
+}
+
 namespace {
 
 inline int grid_for(size_t total, int threads) {

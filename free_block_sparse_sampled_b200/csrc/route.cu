@@ -358,6 +358,95 @@ __global__ void __launch_bounds__(256) probe_select_kernel(
     }
 }
 
+// Random (Floyd's algorithm) or uniform-grid probe rows, then m_a, the sum of
+// coverage weights and the probe list by group, then by index.  One block of
+// 1024 threads per head; `bits` is this head's membership bitmap.
+constexpr uint64_t kProbeStream = 0x50524F4245ull;
+__global__ void __launch_bounds__(1024) probe_fixed_kernel(
+    int mode, uint64_t seed, const int32_t* __restrict__ q_off, const int32_t* __restrict__ perm_q,
+    const int32_t* __restrict__ q_label, const int32_t* __restrict__ ng, int Cq, int N, int Mp,
+    uint32_t* __restrict__ bits_all, int32_t* __restrict__ alloc, int32_t* __restrict__ psum,
+    unsigned long long* __restrict__ pairs, int32_t* __restrict__ probe_idx, int32_t* __restrict__ probe_group,
+    float* __restrict__ probe_weight) {
+    __shared__ int hist[kMaxGroups];
+    __shared__ int warp_tot[32];
+    __shared__ int sum_w, run;
+    const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int nwords = (N + 31) / 32;
+    uint32_t* bits = bits_all + (size_t)bh * nwords;
+    const int Cqp = ng[bh * 2 + 0];
+    const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
+    const int32_t* lab = q_label + (size_t)bh * N;
+    for (int e = tid; e < nwords; e += blockDim.x) bits[e] = 0u;
+    for (int a = tid; a < Cqp; a += blockDim.x) hist[a] = 0;
+    if (tid == 0) {
+        sum_w = 0;
+        run = 0;
+    }
+    __syncthreads();
+    if (mode == SPARSEPR_PROBES_RANDOM) {
+        if (tid == 0) {
+            const uint64_t base = sm64_finalise(seed ^ sm64_finalise(((uint64_t)(bh + 1) * kGoldenGamma) ^ kProbeStream));
+            for (int s = 0; s < Mp; ++s) {
+                const int j = N - Mp + s;
+                const uint64_t x = sm64_finalise(base + (uint64_t)(s + 1) * kGoldenGamma);
+                const int t = (int)(((x >> 32) * (uint64_t)(j + 1)) >> 32);
+                const int pick = ((bits[t >> 5] >> (t & 31)) & 1u) ? j : t;
+                bits[pick >> 5] |= 1u << (pick & 31);
+            }
+        }
+    } else {
+        for (int j = tid; j < Mp; j += blockDim.x) {
+            const int r = (int)(((2LL * j + 1) * (long long)N) / (2LL * Mp));
+            atomicOr(&bits[r >> 5], 1u << (r & 31));
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < N; i += blockDim.x)
+        if ((bits[i >> 5] >> (i & 31)) & 1u) atomicAdd(&hist[lab[i]], 1);
+    __syncthreads();
+    for (int a = tid; a < Cqp; a += blockDim.x) {
+        alloc[(size_t)bh * Cq + a] = hist[a];
+        if (hist[a] > 0) atomicAdd(&sum_w, qo[a + 1] - qo[a]);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        psum[bh] = sum_w;
+        pairs[bh * 2 + 1] = pairs[bh * 2 + 0] + (unsigned long long)Mp * (unsigned long long)N;
+    }
+    // list in permuted order (group-major, stable by index): block-wide compaction
+    const int32_t* pq = perm_q + (size_t)bh * N;
+    for (int r0 = 0; r0 < N; r0 += blockDim.x) {
+        const int r = r0 + tid;
+        int i = 0;
+        bool f = false;
+        if (r < N) {
+            i = pq[r];
+            f = (bits[i >> 5] >> (i & 31)) & 1u;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) warp_tot[wid] = __popc(bal);
+        __syncthreads();
+        int before = run;
+        for (int w2 = 0; w2 < wid; ++w2) before += warp_tot[w2];
+        if (f) {
+            const int slot = before + __popc(bal & ((1u << lane) - 1u));
+            const int a = lab[i];
+            probe_idx[(size_t)bh * Mp + slot] = i;
+            probe_group[(size_t)bh * Mp + slot] = a;
+            probe_weight[(size_t)bh * Mp + slot] =
+                (float)((double)Mp * ((double)(qo[a + 1] - qo[a]) / (double)hist[a]) / (double)sum_w);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int t = 0;
+            for (int w2 = 0; w2 < (int)(blockDim.x >> 5); ++w2) t += warp_tot[w2];
+            run += t;
+        }
+        __syncthreads();
+    }
+}
+
 // ================================================================ host side
 namespace {
 
@@ -400,6 +489,13 @@ sparsepr_status run_route(const sparsepr_params& p, const Plan& pl, const sparse
         lbar, vv, t1, t2, ml, part.q_offsets,
         part.kv_offsets, part.n_groups, pl.Cq, pl.Ck, pl.d, (long long)pl.beta, r.score, r.mask,
         r.sel_count, r.sel_groups, reinterpret_cast<unsigned long long*>(r.pairs));
+    if (p.probe_select != SPARSEPR_PROBES_STRATIFIED && pl.Mp > 0 && pl.Mp < pl.N) {
+        count_launch(), probe_fixed_kernel<<<BH, 1024, 0, st>>>(
+            p.probe_select, p.seed, part.q_offsets, part.perm_q, part.q_label, part.n_groups, pl.Cq, pl.N, pl.Mp,
+            at<uint32_t>(ws, pl.o_pbits), alloc, psum, reinterpret_cast<unsigned long long*>(r.pairs), r.probe_idx,
+            r.probe_group, r.probe_weight);
+        return cuda_status(cudaGetLastError());
+    }
     count_launch(), probe_alloc_kernel<<<BH, 1024, 0, st>>>(part.q_offsets, part.n_groups, pl.Cq, pl.N, pl.Mp, alloc, poff, psum,
                                             reinterpret_cast<unsigned long long*>(r.pairs));
     if (pl.Mp > 0)

@@ -61,6 +61,30 @@ typedef enum {
 
 typedef enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 } sparsepr_dtype;
 
+/* Probe selection (paper A.2; Table 4's variants).  With M >= N every
+ * variant takes all rows as probes. */
+typedef enum {
+    SPARSEPR_PROBES_STRATIFIED = 0, /* largest-remainder m_a per query group, the m_a members
+                                       nearest the group mean (A.2) */
+    SPARSEPR_PROBES_RANDOM = 1,     /* M distinct rows uniformly at random: Floyd's algorithm on
+                                       a SplitMix64 stream seeded by
+                                       mix(seed ^ mix((bh+1)*0x9E3779B97F4A7C15 ^ 0x50524F4245));
+                                       draw s (s = 0..M-1, the (s+1)-th output) with top 32 bits u
+                                       gives t = (u*(j+1)) >> 32 for j = N-M+s, and the sample
+                                       gains t, or j if t is already in it */
+    SPARSEPR_PROBES_UNIFORM = 2     /* rows floor((2j+1)N / 2M), j < M: evenly spaced over the
+                                       row-major (t,y,x) grid */
+} sparsepr_probe_select;
+
+/* Correction family (paper D.4); every family keeps the weighted
+ * standardisation, centring and coverage weights of A.3. */
+typedef enum {
+    SPARSEPR_CORRECTION_FULL = 0,     /* unrestricted B (weighted ridge, §4.2) */
+    SPARSEPR_CORRECTION_DIAGONAL = 1, /* B = diag(b), b_j = (X^T W R)_jj / ((X^T W X)_jj + lambda) */
+    SPARSEPR_CORRECTION_SCALAR = 2,   /* B = a I, a = tr(X^T W R) / (tr(X^T W X) + lambda d) */
+    SPARSEPR_CORRECTION_MEAN = 3      /* B = 0: the weighted mean residual only */
+} sparsepr_correction;
+
 /* flags */
 #define SPARSEPR_FLAG_DEBUG_EXPORT 1   /* fill the debug_* outputs of partition */
 #define SPARSEPR_FLAG_SIMT_ATTENTION 2 /* bf16: use the CUDA-core attention kernel */
@@ -96,6 +120,10 @@ typedef struct {
     float eps_rms;             /* RMSNorm floor in phi_Q (B.2) */
     float eps_std;             /* variance floor in the standardisation (D.3) */
     int32_t flags;             /* SPARSEPR_FLAG_* */
+    int32_t probe_select;      /* sparsepr_probe_select (0 = stratified, the paper's method) */
+    int32_t correction;        /* sparsepr_correction (0 = full ridge, the paper's method) */
+    int32_t residual_rank;     /* 0: no truncation (the paper's method); r in 1..d: B V_r V_r^T with
+                                  V_r the leading r right singular vectors of W^1/2 Rbar (D.3) */
 } sparsepr_params;
 
 /* Outputs of sparsepr_partition (paper §4.1).  Required unless marked
@@ -139,11 +167,12 @@ typedef struct {
     int32_t* sel_count;   /* [BH,Cq] number of selected K/V groups of group a */
     int32_t* sel_groups;  /* [BH,Cq,Ck] selected K/V groups of a, ascending, first sel_count */
     int64_t* pairs;       /* [BH,2] (P_route, P_exec = P_route + min(M,N)*N) */
-    int32_t* probe_idx;   /* [BH,M'] probe rows (original index), M' = min(M,N);
-                             ordered by group, then by (d_i, i) */
+    int32_t* probe_idx;   /* [BH,M'] probe rows (original index), M' = min(M,N); ordered by
+                             group, then by (d_i, i) (stratified, or M >= N) or by index */
     int32_t* probe_group; /* [BH,M'] query group of each probe */
     float* probe_weight;  /* [BH,M'] w~_p (unit mean, A.3) */
-    int32_t* probe_alloc; /* [BH,Cq] m_a probes per query group */
+    int32_t* probe_alloc; /* [BH,Cq] m_a probes per query group (for random and uniform
+                             probes: the number that fall in the group) */
 } sparsepr_route_out;
 
 /* Outputs of sparsepr_probe_fit (paper §4.2, A.3). */
@@ -236,7 +265,9 @@ sparsepr_status sparsepr_attention(const sparsepr_params* p, const sparsepr_part
  * centring and the ridge solve B = (Xbar^T W Xbar + lambda I)^-1 Xbar^T W Rbar
  * on R = probe_dense - probe_sparse (Cholesky, fp64 internally).  A
  * non-positive pivot records SPARSEPR_NUMERIC in the device status word and
- * leaves B = 0. */
+ * leaves B = 0.  p->correction selects a restricted family instead (D.4),
+ * and p->residual_rank > 0 projects B onto the leading right singular
+ * vectors of W^1/2 Rbar (fp32 Jacobi eigenvectors of Rbar^T W Rbar; D.3). */
 sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const sparsepr_partition_out* part,
                                    const sparsepr_route_out* route, const float* probe_sparse,
                                    const float* probe_dense, const sparsepr_fit_out* fit,
@@ -248,7 +279,8 @@ sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const sparsepr_part
  * which allows up to 31 heads (B*H) at d = 128 and 125 heads at d = 64. */
 #define SPARSEPR_FIT_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 
-/* sparsepr_probe_fit without a workspace.  The paper has no counterpart: it
+/* sparsepr_probe_fit without a workspace (p->residual_rank must be 0:
+ * the truncation needs workspace scratch; otherwise SPARSEPR_UNSUPPORTED).  The paper has no counterpart: it
  * exists for callers that hold the partition and routing results but cannot
  * allocate device memory where they run the fit -- a host framework whose
  * caching allocator has taken all free HBM, or a loop that must not take the

@@ -59,7 +59,7 @@ def head_view(res, cfg, bh):
     p, r = res["part"], res["route"]
     Cq2, Ck2 = (int(x) for x in npi(p["n_groups"][bh]))
     N, Mp = cfg.N, cfg.Mp
-    h = {"Cq": Cq2, "Ck": Ck2}
+    h = {"Cq": Cq2, "Ck": Ck2, "bh": bh}
     for k in ["q_label", "kv_label", "perm_q", "perm_kv", "pos_q"]:
         h[k] = npi(p[k][bh])
     h["q_offsets"] = npi(p["q_offsets"][bh])[: Cq2 + 1]
@@ -102,7 +102,8 @@ def row_rel_l2(a, b):
 
 
 def check_integer_chain(h, cfg):
-    """Integer steps, each fed the GPU's own upstream values (bit-exact)."""
+    """Integer steps, each fed the GPU's own upstream values (bit-exact);
+    probes follow the config's probe selection."""
     N = cfg.N
     # group-major permutation and offsets from the GPU labels
     for lab_key, perm_key, off_key, C in [("q_label", "perm_q", "q_offsets", h["Cq"]),
@@ -127,9 +128,15 @@ def check_integer_chain(h, cfg):
         assert list(h["sel_groups"][a][:n]) == list(np.nonzero(mask[a])[0])
     # probes from the GPU's labels and fp32 d_i
     if cfg.Mp > 0:
-        m = O.probe_allocation(q_sizes, cfg.Mp, N)
+        if cfg.probe_select == "stratified" or cfg.Mp >= N:
+            m = O.probe_allocation(q_sizes, cfg.Mp, N)
+            P = O.probe_select(h["q_label"], h["q_dist"], m)
+        else:
+            bh = h["bh"]
+            rows = O.random_probes(cfg.seed, bh, N, cfg.Mp) if cfg.probe_select == "random" else \
+                O.uniform_probes(N, cfg.Mp)
+            P, m = O.listed_by_group(rows, h["q_label"], h["Cq"])
         assert np.array_equal(m, h["probe_alloc"])
-        P = O.probe_select(h["q_label"], h["q_dist"], m)
         assert np.array_equal(P, h["probe_idx"])
         assert np.array_equal(h["q_label"][P], h["probe_group"])
         _, _, wt = O.coverage_weights(h["q_label"][P], q_sizes, m, cfg.Mp)
@@ -188,20 +195,28 @@ def check_attention(h, cfg, tol):
     return float(err.max())
 
 
+def fit_reference(h, cfg):
+    """The oracle's fit (family and rank of the config) on the GPU's probe rows."""
+    q_sizes = np.diff(h["q_offsets"])
+    _, alpha, wt = O.coverage_weights(h["probe_group"], q_sizes, h["probe_alloc"], cfg.Mp)
+    X, D = h["probe_sparse"], h["probe_dense"]
+    f = O.restricted_fit(X, D - X, alpha, wt, cfg.lam, cfg.eps_std, cfg.correction)
+    if 0 < cfg.residual_rank < cfg.d:
+        f = {**f, "B": O.residual_span_projection(f["B"], f["Rbar"], wt, cfg.residual_rank)}
+    return f
+
+
 def check_fit_and_apply(h, cfg):
     """Ridge fit and corrected output from the GPU's own sparse / dense probe rows."""
     if cfg.Mp == 0:
         np.testing.assert_array_equal(h["out"], h["O_sp"][h["pos_q"]])
         return
-    q_sizes = np.diff(h["q_offsets"])
-    m = h["probe_alloc"]
-    _, alpha, wt = O.coverage_weights(h["probe_group"], q_sizes, m, cfg.Mp)
     X, D = h["probe_sparse"], h["probe_dense"]
-    f = O.ridge_fit(X, D - X, alpha, wt, cfg.lam, cfg.eps_std)
+    f = fit_reference(h, cfg)
     for k in ["mu_X", "sigma", "mu_R"]:
         g = h["fit_" + {"mu_X": "mu_x", "sigma": "sigma", "mu_R": "mu_r"}[k]]
         np.testing.assert_allclose(g, f[k], rtol=TOL_FIT, atol=TOL_FIT * np.abs(f[k]).max() + 1e-12)
-    Bn = np.abs(f["B"]).max()
+    Bn = max(np.abs(f["B"]).max(), 1e-30)
     assert np.abs(h["fit_B"] - f["B"]).max() <= TOL_FIT * Bn, "ridge B"
     O_sp = h["O_sp"][h["pos_q"]]                           # original order
     ref = O.apply_correction(O_sp, h["probe_idx"], D, f)
