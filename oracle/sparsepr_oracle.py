@@ -77,6 +77,12 @@ R18 Correction families (D.4): with the same standardisation, centring and
     B = diag(b) with b_j = (Xbar^T W Rbar)_jj / ((Xbar^T W Xbar)_jj + lambda);
     each minimises the weighted squared error plus lambda |B|_F^2 over its
     family.  Rank r truncation (D.3) replaces B by B V_r V_r^T.
+R19 GQA (§4.3 "Routing and GQA", C.1): the G query heads of one K/V head
+    share the key metric, F_K and the K/V groups.  The metric's rows are
+    G M_s evenly spaced rows of the G heads' queries stacked in head order
+    (all rows when fewer); the K/V k-means draws its initial rows from the
+    K/V head's stream (head index = K/V head).  Query groups, routing,
+    probes and the fit stay per query head, with the query head's streams.
 """
 
 from __future__ import annotations
@@ -556,7 +562,8 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
                   kmeans_tol: float, eps_rms: float = 1e-6, eps_std: float = 1e-6,
                   want_dense: bool = False, warm: Optional[Dict[str, np.ndarray]] = None,
                   partition: str = "response", probes: str = "stratified", correction: str = "full",
-                  residual_rank: int = 0) -> Dict[str, object]:
+                  residual_rank: int = 0, metric_rows: Optional[np.ndarray] = None,
+                  bh_kv: Optional[int] = None) -> Dict[str, object]:
     """One SparsePR call on one head, steps in the paper's order:
     partition (§4.1) -> route (§4.3, B.3) -> sparse attention (Eq. 2) ->
     probes (A.2) -> weighted ridge (A.3) -> corrected output (§4.2).
@@ -565,7 +572,9 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     ``partition``: "response" (§4.1), "semantic" or "key_response" (R16).
     ``probes``: "stratified" (A.2), "random" or "uniform" (R17);
     ``correction``: "full", "diagonal", "scalar" or "mean" (R18);
-    ``residual_rank``: 0 (no truncation) or r (D.3)."""
+    ``residual_rank``: 0 (no truncation) or r (D.3).
+    ``metric_rows`` / ``bh_kv``: the query rows the key metric samples and
+    the head index of the K/V k-means stream (GQA, R19; default q and bh)."""
     if partition not in ("response", "semantic", "key_response"):
         raise ValueError(partition)
     semantic_keys = partition == "semantic"
@@ -577,8 +586,9 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     out: Dict[str, object] = {}
 
     # 1-2. key-response metric and factor
-    idx = sample_indices(N, Ms)
-    M_K = key_metric(q, idx)
+    mrows = q if metric_rows is None else np.asarray(metric_rows, dtype=np.float64)
+    idx = sample_indices(len(mrows), Ms)
+    M_K = key_metric(mrows, idx)
     r_k = min(rK, d, len(idx))
     F_K = None if (warm is None or semantic_keys) else warm_factor(M_K, warm["F_K"], r_k, 1.0 / math.sqrt(d))
     warm_K = F_K is not None
@@ -588,7 +598,7 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
         F_K = key_factor(M_K, rK, len(idx))
     phi_K = k @ F_K
     # 3. paired K/V groups
-    init_k = kmeans_init_indices(seed, bh, 0, Ck, N)
+    init_k = kmeans_init_indices(seed, bh if bh_kv is None else bh_kv, 0, Ck, N)
     stop = kmeans_stop_count(kmeans_tol, N)
     cen_k = None if warm is None else warm_centres(phi_K, warm["kbar"], F_K, Ck, init_k)
     kv_raw, _, it_k, _ = kmeans(phi_K, init_k, kmeans_iters, stop, cen_k)
@@ -651,6 +661,15 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     if want_dense:
         out["O_dense"] = dense_attention(q, k, v)
     return out
+
+
+def sparsepr_gqa(qs, k, v, *, kvh: int, Ms: int, **kw):
+    """R19: the G query heads qs[g] of K/V head ``kvh`` (query head indices
+    kvh G + g); returns one sparsepr_head result per query head."""
+    G = len(qs)
+    stacked = np.concatenate([np.asarray(x, dtype=np.float64) for x in qs], axis=0)
+    return [sparsepr_head(qs[g], k, v, bh=kvh * G + g, bh_kv=kvh, metric_rows=stacked, Ms=G * Ms, **kw)
+            for g in range(G)]
 
 
 def warm_state(out: Dict[str, object]) -> Dict[str, np.ndarray]:

@@ -785,3 +785,32 @@ def test_whole_call_variants_on_tiny():
     mean = O.sparsepr_head(q, k, v, bh=0, correction="mean", **kw)
     unp = np.setdiff1d(np.arange(w.N), mean["probes"])
     np.testing.assert_allclose(mean["O"][unp], base["O_sp"][unp] + mean["fit"]["mu_R"][None, :], atol=1e-12)
+
+
+# ------------------------------------------------------------------ GQA (R19)
+def test_gqa_metric_is_the_mean_of_the_heads_metrics():
+    """G M_s evenly spaced rows of the stacked heads are each head's own M_s
+    sampled rows, so the shared metric is the mean of the per-head metrics."""
+    G, N, d, Ms = 3, 50, 4, 7
+    qs = [_rand((N, d), 100 + g) for g in range(G)]
+    stacked = np.concatenate(qs)
+    idx = O.sample_indices(G * N, G * Ms)
+    shared = O.key_metric(stacked, idx)
+    per_head = [O.key_metric(x, O.sample_indices(N, Ms)) for x in qs]
+    np.testing.assert_allclose(shared, np.mean(per_head, axis=0), atol=1e-13)
+
+
+def test_gqa_heads_share_the_kv_partition():
+    w, q, k, v = _tiny_head()
+    kw = O.workload_kwargs(w)
+    kw.pop("Ms")
+    qs = [q, q[::-1].copy(), 0.5 * q]
+    res = O.sparsepr_gqa(qs, k, v, kvh=1, Ms=w.Ms, **kw)
+    for r in res[1:]:
+        assert np.array_equal(r["kv_labels"], res[0]["kv_labels"])
+        np.testing.assert_array_equal(r["F_K"], res[0]["F_K"])
+    assert not np.array_equal(res[0]["q_labels"], res[1]["q_labels"])
+    # G = 1 is the single-head call with the K/V stream of head kvh
+    one = O.sparsepr_gqa([q], k, v, kvh=0, Ms=w.Ms, **kw)[0]
+    ref = O.sparsepr_head(q, k, v, bh=0, Ms=w.Ms, **kw)
+    np.testing.assert_array_equal(one["O"], ref["O"])
