@@ -39,7 +39,7 @@ class Params(ctypes.Structure):
                 ("kmeans_iters", ctypes.c_int32), ("kmeans_tol", ctypes.c_double),
                 ("seed", ctypes.c_uint64), ("block", ctypes.c_int32), ("eps_rms", ctypes.c_float),
                 ("eps_std", ctypes.c_float), ("flags", ctypes.c_int32), ("probe_select", ctypes.c_int32),
-                ("correction", ctypes.c_int32), ("residual_rank", ctypes.c_int32)]
+                ("correction", ctypes.c_int32), ("residual_rank", ctypes.c_int32), ("Hkv", ctypes.c_int32)]
 
 
 PARTITION_FIELDS = ["Qp", "Kp", "Vp", "q_label", "kv_label", "perm_q", "perm_kv", "pos_q", "q_offsets",

@@ -45,6 +45,7 @@ class SparsePRConfig:
     probe_select: str = "stratified"   # "stratified" (A.2), "random" or "uniform" (Table 4)
     correction: str = "full"           # "full", "diagonal", "scalar" or "mean" (D.4)
     residual_rank: int = 0             # 0: no truncation; r: rank-r residual projection (D.3)
+    Hkv: int = 0                       # K/V heads (GQA): 0 = H; else a divisor of H
 
     @classmethod
     def from_workload(cls, w, **kw) -> "SparsePRConfig":
@@ -58,6 +59,11 @@ class SparsePRConfig:
     @property
     def BH(self) -> int:
         return self.B * self.H
+
+    @property
+    def Hk(self) -> int:
+        """K/V heads."""
+        return self.Hkv if self.Hkv else self.H
 
     @property
     def Mp(self) -> int:
@@ -86,7 +92,7 @@ class SparsePRConfig:
                         float(self.lam), self.Cq, self.Ck, self.rK, self.rQ, self.kmeans_iters,
                         float(self.kmeans_tol), int(self.seed) & ((1 << 64) - 1), self.block,
                         float(self.eps_rms), float(self.eps_std), self.flags, A.PROBES[self.probe_select],
-                        A.CORRECTIONS[self.correction], int(self.residual_rank))
+                        A.CORRECTIONS[self.correction], int(self.residual_rank), int(self.Hkv))
 
 
 def validate(cfg: SparsePRConfig) -> int:
@@ -116,11 +122,11 @@ def _stream() -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _check_qkv(cfg: SparsePRConfig, *ts: torch.Tensor) -> None:
-    for t in ts:
+def _check_qkv(cfg: SparsePRConfig, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> None:
+    for t, h in ((q, cfg.H), (k, cfg.Hk), (v, cfg.Hk)):
         if not (t.is_cuda and t.is_contiguous() and t.dtype == cfg.torch_dtype and
-                tuple(t.shape) == (cfg.B, cfg.H, cfg.N, cfg.d)):
-            raise ValueError("Q/K/V must be contiguous CUDA tensors of shape [B,H,N,d] and the config dtype")
+                tuple(t.shape) == (cfg.B, h, cfg.N, cfg.d)):
+            raise ValueError("Q must be [B,H,N,d] and K/V [B,Hkv,N,d]: contiguous CUDA tensors of the config dtype")
 
 
 def partition(cfg: SparsePRConfig, q, k, v, ws: torch.Tensor, debug: bool = False,
@@ -134,7 +140,7 @@ def partition(cfg: SparsePRConfig, q, k, v, ws: torch.Tensor, debug: bool = Fals
     i32 = dict(dtype=torch.int32, device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
     o = {
-        "Qp": torch.empty_like(q), "Kp": torch.empty_like(k), "Vp": torch.empty_like(v),
+        "Qp": torch.empty_like(q), "Kp": torch.empty_like(q), "Vp": torch.empty_like(q),
         "q_label": torch.empty(BH, N, **i32), "kv_label": torch.empty(BH, N, **i32),
         "perm_q": torch.empty(BH, N, **i32), "perm_kv": torch.empty(BH, N, **i32),
         "pos_q": torch.empty(BH, N, **i32), "q_offsets": torch.empty(BH, Cq + 1, **i32),
@@ -286,7 +292,8 @@ class HostPipeline:
         self.cfg = cfg
         dev = torch.device(device)
         shape = (cfg.B, cfg.H, cfg.N, cfg.d)
-        self.din = [[torch.empty(shape, dtype=cfg.torch_dtype, device=dev) for _ in range(3)] for _ in range(2)]
+        shapes = [shape, (cfg.B, cfg.Hk, cfg.N, cfg.d), (cfg.B, cfg.Hk, cfg.N, cfg.d)]
+        self.din = [[torch.empty(sh, dtype=cfg.torch_dtype, device=dev) for sh in shapes] for _ in range(2)]
         self.dout = [torch.empty(shape, dtype=torch.float32, device=dev) for _ in range(2)]
         self.ws = alloc_workspace(cfg, dev)
         self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))

@@ -19,6 +19,7 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     if (sparsepr_validate(&p) != SPARSEPR_OK) return false;
     const size_t BH = (size_t)p.B * p.H, N = p.N, d = p.d;
     pl.BH = (int)BH;
+    pl.G = p.Hkv > 0 ? p.H / p.Hkv : 1;
     pl.N = p.N;
     pl.d = p.d;
     pl.Cq = p.Cq;
@@ -90,6 +91,7 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_warm = bump(c, (1 + 2 * BH) * 4);
     pl.o_pbits = bump(c, BH * ((N + 31) / 32) * 4);
     pl.o_S = bump(c, p.residual_rank > 0 ? BH * d * d * 8 : 256);
+    pl.o_rawkv = bump(c, pl.G > 1 ? BH / pl.G * N * 4 : 256);
     // outputs owned by the workspace (fused call)
     pl.o_Qp = bump(c, BH * N * d * es);
     pl.o_Kp = bump(c, BH * N * d * es);
@@ -228,6 +230,8 @@ sparsepr_status sparsepr_validate(const sparsepr_params* p) {
     if (p->block != 64 && p->block != 128) return SPARSEPR_INVALID_ARG;
     if (p->probe_select < 0 || p->probe_select > 2 || p->correction < 0 || p->correction > 3) return SPARSEPR_INVALID_ARG;
     if (p->residual_rank < 0 || p->residual_rank > p->d) return SPARSEPR_INVALID_ARG;
+    if (p->Hkv < 0 || (p->Hkv > 0 && p->H % p->Hkv != 0)) return SPARSEPR_INVALID_ARG;
+    if (p->Hkv > 0 && p->Hkv < p->H && (p->flags & SPARSEPR_FLAG_WARM_START)) return SPARSEPR_UNSUPPORTED;
     if (p->d != 64 && p->d != 128) return SPARSEPR_UNSUPPORTED;
     if (p->Cq > kMaxGroups || p->Ck > kMaxGroups) return SPARSEPR_UNSUPPORTED;
     if (p->rK > kMaxRank || p->rQ > kMaxRank) return SPARSEPR_UNSUPPORTED;
@@ -268,6 +272,7 @@ sparsepr_status sparsepr_partition_warm(const sparsepr_params* p, const void* Q,
     if (!Q || !K || !V || !partition_ok(part)) return SPARSEPR_INVALID_ARG;
     if (!prev || !prev->F_K || !prev->F_Q || !prev->k_centroid || !prev->q_centroid || !prev->n_groups)
         return SPARSEPR_INVALID_ARG;
+    if (pl.G > 1) return SPARSEPR_UNSUPPORTED;   // the warm state is per query head
     if ((p->flags & SPARSEPR_FLAG_DEBUG_EXPORT) &&
         !(part->debug_kv_scores && part->debug_q_scores && part->debug_kv_hist && part->debug_q_hist))
         return SPARSEPR_INVALID_ARG;

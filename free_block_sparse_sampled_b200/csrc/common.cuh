@@ -102,6 +102,7 @@ __device__ __forceinline__ int kmeans_init_row(uint64_t seed, int bh, int stage,
 struct Plan {
     // sizes
     int BH, N, d, Cq, Ck, Cmax, RKp, RQp, rK_eff, Mp, Ms_eff, n_sort_tiles, esz;
+    int G;               // query heads per K/V head (GQA; 1 otherwise)
     int BM, n_items_max, n_probe_items;
     int64_t beta;        // key budget per query group
     int stop_changed;    // k-means stop threshold on changed labels
@@ -111,7 +112,8 @@ struct Plan {
         o_poff, o_psum, o_qprobe, o_work, o_fstat, o_G, o_rhs, o_vh, o_vmax, o_vscale, o_qsplit, o_uw, o_lbar, o_vv,
         o_warm,   // [0]: kWarmMagic when the fused call's state is complete; [1 + bh], [1 + BH + bh]: cold K / Q factor
         o_pbits,  // [BH][ceil(N/32)] probe membership bits (random / uniform probes)
-        o_S;      // [BH][d][d] fp64 Rbar^T W Rbar (rank truncation)
+        o_S,      // [BH][d][d] fp64 Rbar^T W Rbar (rank truncation)
+        o_rawkv;  // [BH/G][N] K/V k-means labels per K/V head (GQA)
     // outputs owned by the workspace for sparsepr_call
     size_t o_Qp, o_Kp, o_Vp, o_qlab, o_kvlab, o_permq, o_permk, o_posq, o_qoff, o_kvoff, o_ng, o_its,
         o_qcen, o_kcen, o_vcen, o_qdist, o_score, o_mask, o_selc, o_selg, o_pairs, o_pidx, o_pgrp,

@@ -608,14 +608,14 @@ __global__ void relabel_kernel(const int32_t* __restrict__ raw, const int32_t* _
 
 // Xp[r] = X[perm[r]] in 16-byte chunks (group-major gather, paper §4.3).
 __global__ void gather_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ perm,
-                                   int BH, int N, int chunks, uint4* __restrict__ Xp) {
+                                   int BH, int N, int chunks, int G, uint4* __restrict__ Xp) {
     const size_t total = (size_t)BH * N * chunks;
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
          e += (size_t)gridDim.x * blockDim.x) {
         const size_t row = e / chunks;
         const int ch = (int)(e - row * chunks);
         const size_t bh = row / N;
-        const size_t src = bh * N + perm[row];
+        const size_t src = (bh / G) * N + perm[row];   // source head: K/V head bh / G under GQA
         Xp[e] = X[src * chunks + ch];
     }
 }
@@ -675,6 +675,33 @@ __global__ void iters_out_kernel(const int32_t* __restrict__ ctl, int BH, int32_
     out[bh * 2 + 1] = ctl[bh * kCtlStride + kCtlItersQ];
 }
 
+// GQA (paper §4.3, C.1): the G query heads of a K/V head share its key
+// metric, which is the mean of their sampled metrics (G*Ms evenly spaced rows
+// of the stacked heads are each head's own Ms rows).
+__global__ void mean_heads_kernel(const float* __restrict__ in, int G, size_t per_head, size_t total,
+                                  float* __restrict__ out) {
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+        const size_t h = e / per_head, i = e - h * per_head;
+        float s = 0.f;
+        for (int g = 0; g < G; ++g) s += in[(h * G + g) * per_head + i];
+        out[e] = s / (float)G;
+    }
+}
+
+// dst head bh = src head bh / G (4-byte words, per_head words per head).
+__global__ void broadcast_heads_kernel(const uint32_t* __restrict__ src, size_t per_head, size_t total, int G,
+                                       uint32_t* __restrict__ dst) {
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+        const size_t h = e / per_head, i = e - h * per_head;
+        dst[e] = src[(h / G) * per_head + i];
+    }
+}
+
+// The K/V k-means count of each K/V head to its query heads (descending, in place).
+__global__ void broadcast_iters_kernel(int32_t* ctl, int BH, int G) {
+    for (int bh = BH - 1; bh >= 0; --bh) ctl[bh * kCtlStride + kCtlIters] = ctl[(bh / G) * kCtlStride + kCtlIters];
+}
+
 // Semantic partition (paper §3 reference partition, Table 2): the k-means
 // coordinates are the raw rows, TF32-rounded (exact for bf16 inputs), and
 // the factor is the identity.
@@ -714,13 +741,12 @@ inline int grid_for(size_t total, int threads) {
 template <int R>
 void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float* phi, int C,
                 int stage, float* cen, float* hn, float* dbg_scores, int32_t* dbg_hist,
-                int save_slot, const WarmInit* wi, cudaStream_t st) {
+                int save_slot, const WarmInit* wi, int nh, int32_t* raw, cudaStream_t st) {
     int32_t* ctl = at<int32_t>(ws, pl.o_ctl);
-    int32_t* raw = at<int32_t>(ws, pl.o_raw);
     int32_t* hist = at<int32_t>(ws, pl.o_hist);
     int32_t* sorted = at<int32_t>(ws, pl.o_sorted);
     int32_t* offs = at<int32_t>(ws, pl.o_offs);
-    const int BH = pl.BH, N = pl.N;
+    const int BH = nh, N = pl.N;
     const int bgrid = (BH + 127) / 128;
     count_launch(), kmeans_reset_kernel<<<bgrid, 128, 0, st>>>(ctl, BH, save_slot);
     if (wi != nullptr)
@@ -749,13 +775,13 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
 
 void kmeans_dispatch(int R, const Plan& pl, const sparsepr_params& p, void* ws, const float* phi,
                      int C, int stage, float* cen, float* hn, float* dbg_scores, int32_t* dbg_hist,
-                     int save_slot, const WarmInit* wi, cudaStream_t st) {
+                     int save_slot, const WarmInit* wi, int nh, int32_t* raw, cudaStream_t st) {
     switch (R) {
-        case 16: kmeans_run<16>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
-        case 32: kmeans_run<32>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
-        case 48: kmeans_run<48>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
-        case 64: kmeans_run<64>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
-        default: kmeans_run<128>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, st); break;
+        case 16: kmeans_run<16>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, nh, raw, st); break;
+        case 32: kmeans_run<32>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, nh, raw, st); break;
+        case 48: kmeans_run<48>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, nh, raw, st); break;
+        case 64: kmeans_run<64>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, nh, raw, st); break;
+        default: kmeans_run<128>(pl, p, ws, phi, C, stage, cen, hn, dbg_scores, dbg_hist, save_slot, wi, nh, raw, st); break;
     }
 }
 
@@ -795,11 +821,11 @@ void finalize_groups(const Plan& pl, void* ws, int C, int which, int32_t* label_
                                                                   label_out, perm_out, pos_out);
 }
 
-void gather(const void* X, const int32_t* perm, const Plan& pl, void* Xp, cudaStream_t st) {
+void gather(const void* X, const int32_t* perm, const Plan& pl, void* Xp, int G, cudaStream_t st) {
     const int chunks = pl.d * pl.esz / 16;
     const size_t total = (size_t)pl.BH * pl.N * chunks;
     count_launch(), gather_rows_kernel<<<grid_for(total, 256), 256, 0, st>>>(
-        static_cast<const uint4*>(X), perm, pl.BH, pl.N, chunks, static_cast<uint4*>(Xp));
+        static_cast<const uint4*>(X), perm, pl.BH, pl.N, chunks, G, static_cast<uint4*>(Xp));
 }
 
 template <typename T>
@@ -830,22 +856,33 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     const size_t n8 = (size_t)BH * N * d / 8;
     int32_t* coldK = at<int32_t>(ws, pl.o_warm) + 1;
     int32_t* coldQ = coldK + BH;
+    // The K/V side runs once per K/V head: BHk = BH / G heads (GQA, §4.3);
+    // K and V are [BHk, N, d].
+    const int G = pl.G, BHk = BH / G;
+    const size_t nk8 = (size_t)BHk * N * d / 8;
     if (sem_k) {
         // semantic K/V groups: k-means on the raw key rows (RKp = d)
-        count_launch(), identity_factor_kernel<<<BH, 256, 0, st>>>(FK, d, pl.RKp, nullptr);
-        count_launch(), raw_coords_kernel<T><<<grid_for(n8, 256), 256, 0, st>>>(K, n8, phiK);
+        count_launch(), identity_factor_kernel<<<BHk, 256, 0, st>>>(FK, d, pl.RKp, nullptr);
+        count_launch(), raw_coords_kernel<T><<<grid_for(nk8, 256), 256, 0, st>>>(K, nk8, phiK);
     } else {
-        // 1-2. key-response metric and factor (§4.1)
+        // 1-2. key-response metric and factor (§4.1); under GQA the mean of
+        // the G query heads' sampled metrics
         count_launch(), sampled_gram_kernel<T><<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(Q, N, d, pl.Ms_eff,
                                                                                                 mat);
+        float* matK = mat;
+        if (G > 1) {
+            matK = at<float>(ws, pl.o_G);   // fit scratch, free during the partition
+            const size_t tot = (size_t)BHk * d * d;
+            count_launch(), mean_heads_kernel<<<grid_for(tot, 256), 256, 0, st>>>(mat, G, (size_t)d * d, tot, matK);
+        }
         // warm start (C.1): subspace iteration from the previous factor; heads it
         // cannot factor (or every head, without a previous state) take Jacobi
         if (warm)
-            launch_warm_factor(mat, warm->F_K, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d), FK, pl.RKp,
-                               nullptr, coldK, warm->valid, BH, d, st);
-        count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FK, pl.RKp, pl.rK_eff, nullptr,
-                                                          1.f / sqrtf((float)d), nullptr, 16, warm ? coldK : nullptr);
-        project_dispatch<T, false>(pl.RKp, K, FK, BH, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
+            launch_warm_factor(matK, warm->F_K, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d), FK, pl.RKp,
+                               nullptr, coldK, warm->valid, BHk, d, st);
+        count_launch(), jacobi<<<BHk, 1024, jac_smem, st>>>(matK, FK, pl.RKp, pl.rK_eff, nullptr,
+                                                           1.f / sqrtf((float)d), nullptr, 16, warm ? coldK : nullptr);
+        project_dispatch<T, false>(pl.RKp, K, FK, BHk, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
     }
     // 3. paired K/V groups
     WarmInit wiK{}, wiQ{};
@@ -853,12 +890,25 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
         wiK = WarmInit{warm->k_centroid, warm->n_groups, 1, FK, d, false, nullptr, 0.f, warm->valid};
         wiQ = WarmInit{warm->q_centroid, warm->n_groups, 0, FQ, d, !sem_q, rq, p.eps_rms, warm->valid};
     }
+    int32_t* raw = at<int32_t>(ws, pl.o_raw);
+    int32_t* rawK = G > 1 ? at<int32_t>(ws, pl.o_rawkv) : raw;
     kmeans_dispatch(pl.RKp, pl, p, ws, phiK, pl.Ck, 0, cenK, hnK, dbg ? out.debug_kv_scores : nullptr,
-                    dbg ? out.debug_kv_hist : nullptr, -1, warm ? &wiK : nullptr, st);
-    if (out.kv_centres) cudaMemcpyAsync(out.kv_centres, cenK, (size_t)BH * pl.Ck * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+                    dbg ? out.debug_kv_hist : nullptr, -1, warm ? &wiK : nullptr, BHk, rawK, st);
+    auto to_query_heads = [&](const void* src, void* dst, size_t words_per_head) {
+        const size_t tot = (size_t)BH * words_per_head;
+        count_launch(), broadcast_heads_kernel<<<grid_for(tot, 256), 256, 0, st>>>(
+            static_cast<const uint32_t*>(src), words_per_head, tot, G, static_cast<uint32_t*>(dst));
+    };
+    if (G > 1) {   // the K/V groups of each K/V head serve its G query heads
+        to_query_heads(rawK, raw, (size_t)N);
+        count_launch(), broadcast_iters_kernel<<<1, 1, 0, st>>>(ctl, BH, G);
+        if (out.kv_centres) to_query_heads(cenK, out.kv_centres, (size_t)pl.Ck * pl.RKp);
+    } else if (out.kv_centres) {
+        cudaMemcpyAsync(out.kv_centres, cenK, (size_t)BH * pl.Ck * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    }
     finalize_groups(pl, ws, pl.Ck, 1, out.kv_label, out.perm_kv, nullptr, out.kv_offsets, out.n_groups, st);
-    gather(K, out.perm_kv, pl, out.Kp, st);
-    gather(V, out.perm_kv, pl, out.Vp, st);
+    gather(K, out.perm_kv, pl, out.Kp, G, st);
+    gather(V, out.perm_kv, pl, out.Vp, G, st);
     // 4. centroids, query metric, factor, coordinates (§4.1, B.2)
     count_launch(), group_mean_kernel<T><<<dim3(pl.Ck, BH), d, 0, st>>>(static_cast<const T*>(out.Kp), out.kv_offsets,
                                                         out.n_groups, 1, N, pl.Ck, d, out.k_centroid);
@@ -881,11 +931,11 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     }
     // 5. query groups
     kmeans_dispatch(pl.RQp, pl, p, ws, phiQ, pl.Cq, 1, cenQ, hnQ, dbg ? out.debug_q_scores : nullptr,
-                    dbg ? out.debug_q_hist : nullptr, kCtlItersK, warm ? &wiQ : nullptr, st);
+                    dbg ? out.debug_q_hist : nullptr, kCtlItersK, warm ? &wiQ : nullptr, BH, raw, st);
     count_launch(), kmeans_reset_kernel<<<(BH + 127) / 128, 128, 0, st>>>(ctl, BH, kCtlItersQ);
     if (out.q_centres) cudaMemcpyAsync(out.q_centres, cenQ, (size_t)BH * pl.Cq * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
     finalize_groups(pl, ws, pl.Cq, 0, out.q_label, out.perm_q, out.pos_q, out.q_offsets, out.n_groups, st);
-    gather(Q, out.perm_q, pl, out.Qp, st);
+    gather(Q, out.perm_q, pl, out.Qp, 1, st);
     count_launch(), group_mean_kernel<T><<<dim3(pl.Cq, BH), d, 0, st>>>(static_cast<const T*>(out.Qp), out.q_offsets,
                                                         out.n_groups, 0, N, pl.Cq, d, out.q_centroid);
     // c_a (phi_Q space) into the query-centre buffer, then d_i (A.2)
@@ -895,9 +945,15 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), query_dist_kernel<<<grid_for((size_t)BH * N, 256), 256, 0, st>>>(phiQ, cenQ, out.q_label, BH, N,
                                                                      pl.Cq, pl.RQp, out.q_dist);
     count_launch(), iters_out_kernel<<<(BH + 127) / 128, 128, 0, st>>>(ctl, BH, out.kmeans_iters_run);
-    if (out.F_K) cudaMemcpyAsync(out.F_K, FK, (size_t)BH * d * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    if (out.F_K) {
+        if (G > 1) to_query_heads(FK, out.F_K, (size_t)d * pl.RKp);
+        else cudaMemcpyAsync(out.F_K, FK, (size_t)BH * d * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    }
     if (out.F_Q) cudaMemcpyAsync(out.F_Q, FQ, (size_t)BH * d * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
-    if (out.phi_K) cudaMemcpyAsync(out.phi_K, phiK, (size_t)BH * N * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    if (out.phi_K) {
+        if (G > 1) to_query_heads(phiK, out.phi_K, (size_t)N * pl.RKp);
+        else cudaMemcpyAsync(out.phi_K, phiK, (size_t)BH * N * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
+    }
     if (out.phi_Q) cudaMemcpyAsync(out.phi_Q, phiQ, (size_t)BH * N * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
     return cuda_status(cudaGetLastError());
 }

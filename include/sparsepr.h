@@ -22,7 +22,7 @@
  *   allocates no device memory: every intermediate lives in one caller-owned
  *   device workspace of sparsepr_workspace_size() bytes, 256-byte aligned.
  * - Q, K, V are [B, H, N, d] row-major, contiguous, in p->dtype (bf16 or
- *   fp32).  All float outputs are fp32.  Index outputs are int32 unless noted.
+ *   fp32); K and V are [B, Hkv, N, d] under GQA (p->Hkv, see below).  All float outputs are fp32.  Index outputs are int32 unless noted.
  *   "BH" below is B*H; per-head slices are contiguous.
  * - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *   NULL = legacy default stream) unless documented otherwise.  Group counts
@@ -124,6 +124,15 @@ typedef struct {
     int32_t correction;        /* sparsepr_correction (0 = full ridge, the paper's method) */
     int32_t residual_rank;     /* 0: no truncation (the paper's method); r in 1..d: B V_r V_r^T with
                                   V_r the leading r right singular vectors of W^1/2 Rbar (D.3) */
+    int32_t Hkv;               /* K/V heads: 0 or H (one per query head), else a divisor of H:
+                                  grouped-query attention with G = H/Hkv query heads per K/V head,
+                                  query head h using K/V head h/G.  The G heads share the key
+                                  metric (G*Ms evenly spaced rows of their stacked queries), F_K
+                                  and the K/V groups (§4.3 "Routing and GQA", C.1); query groups,
+                                  routing, probes and fit stay per query head.  K and V are then
+                                  [B,Hkv,N,d]; every output stays per query head (K/V-side
+                                  outputs repeated G times; the debug K/V arrays are indexed by
+                                  K/V head).  Not combinable with a warm start. */
 } sparsepr_params;
 
 /* Outputs of sparsepr_partition (paper §4.1).  Required unless marked

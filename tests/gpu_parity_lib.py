@@ -232,12 +232,13 @@ def _tf32(x):
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, semantic_queries=False):
+def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, semantic_queries=False, M_K=None):
     """Float outputs of the partition against fp64 recomputation from the
     GPU's own integer decisions.  ``warm`` (F_K, F_Q of the state a warm call
     started from, fp64) switches the factor references to the warm factor;
     a semantic side has the raw rows (TF32-rounded) as coordinates and the
-    identity as its factor."""
+    identity as its factor.  ``M_K`` overrides the key metric (GQA: the
+    metric the query heads of one K/V head share)."""
     kl, ql = h["kv_label"], h["q_label"]
     np.testing.assert_allclose(h["k_centroid"], O.group_means(k, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
     np.testing.assert_allclose(h["v_centroid"], O.group_means(v, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
@@ -258,7 +259,7 @@ def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, sema
     np.testing.assert_allclose(h["q_dist"], dist, rtol=1e-4, atol=1e-5)
     # metric factors: F F^T reproduces the (truncated) metric
     idx = O.sample_indices(cfg.N, cfg.Ms)
-    MK = O.key_metric(q, idx)
+    MK = O.key_metric(q, idx) if M_K is None else M_K
     w, U = O.eigh_desc(MK)
     r = min(cfg.rK, cfg.d, len(idx))
     ref = U[:, :r] @ np.diag(w[:r]) @ U[:, :r].T / cfg.d
