@@ -170,9 +170,16 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                 asm volatile("bar.sync 1, 256;" ::: "memory");
                 staged_bh = bh;
             }
-            // running first maximum over this half's columns, in column order
+            // running first maximum over this half's columns, in column order: the
+            // best value, the base column of the chunk holding it and a copy of
+            // that chunk's scores (predicated copies instead of a per-chunk index
+            // search, which every chunk would run: some lane of the warp almost
+            // always improves); the index is searched once per item
             float best = -INFINITY;
-            int bi = 0x7fffffff;
+            int bcb = 0;
+            float keep[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) keep[i] = -INFINITY;
             for (int blk = 0; blk < nblk; ++blk, ++gb) {
                 const int db = gb & 1;
                 const float* hb = hns + blk * NB;   // columns past C hold -inf and never win
@@ -211,19 +218,24 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                         const float m = fmaxf(fmax3(fmax3(m3[0], m3[1], m3[2]), fmax3(m3[3], m3[4], m3[5]),
                                                     fmax3(m3[6], m3[7], m3[8])),
                                               fmaxf(m3[9], m3[10]));
-                        if (m > best) {   // a later chunk only wins with a strictly larger score
-                            int idx = 31;
+                        const bool up = m > best;   // a later chunk only wins with a strictly larger score
+                        best = up ? m : best;
+                        bcb = up ? cb : bcb;
 #pragma unroll
-                            for (int i = 30; i >= 0; --i) idx = (sc[i] == m) ? i : idx;
-                            best = m;
-                            bi = cb + idx;
-                        }
+                        for (int i = 0; i < 32; ++i) keep[i] = up ? sc[i] : keep[i];
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(bar(B_DE + db));
             }
             if (!ok) break;
+            int bi = 0x7fffffff;
+            if (best > -INFINITY) {
+                int idx = 31;
+#pragma unroll
+                for (int i = 30; i >= 0; --i) idx = (keep[i] == best) ? i : idx;
+                bi = bcb + idx;
+            }
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (half == 1) {
                 red_s[row] = best;
