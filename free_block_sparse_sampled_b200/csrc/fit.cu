@@ -27,35 +27,57 @@ __global__ void fit_stats_kernel(const float* __restrict__ Xs, const float* __re
                                  int32_t* __restrict__ psum, int Cq, int Mp, int d, float eps_std,
                                  double* __restrict__ fstat, float* __restrict__ mu_x, float* __restrict__ sigma,
                                  float* __restrict__ mu_r) {
-    const int bh = blockIdx.x, j = threadIdx.x;
+    constexpr int kChunk = 1024;
+    __shared__ double alp[kChunk];     // alpha_p of the current chunk of probes
+    __shared__ int part[32];
     __shared__ int sum_w;
-    if (j == 0) {   // sum_p w_p = sum of |G_a| over groups holding probes
-        int s = 0;
-        const int Cqp = ng[bh * 2 + 0];
-        for (int a = 0; a < Cqp; ++a)
-            if (alloc[(size_t)bh * Cq + a] > 0) s += q_off[(size_t)bh * (Cq + 1) + a + 1] - q_off[(size_t)bh * (Cq + 1) + a];
-        sum_w = s;
-        psum[bh] = s;
-    }
-    __syncthreads();
-    const float* X = Xs + (size_t)bh * Mp * d;
-    const float* D = Xd + (size_t)bh * Mp * d;
+    const int bh = blockIdx.x, j = threadIdx.x, nt = blockDim.x;
     const int32_t* pg = probe_group + (size_t)bh * Mp;
     const int32_t* al = alloc + (size_t)bh * Cq;
     const int32_t* qo = q_off + (size_t)bh * (Cq + 1);
+    {   // sum_p w_p = sum of |G_a| over groups holding probes (fixed-order block sum)
+        int s = 0;
+        const int Cqp = ng[bh * 2 + 0];
+        for (int a = j; a < Cqp; a += nt)
+            if (al[a] > 0) s += qo[a + 1] - qo[a];
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if ((j & 31) == 0) part[j >> 5] = s;
+        __syncthreads();
+        if (j == 0) {
+            int t = 0;
+            for (int w = 0; w < nt / 32; ++w) t += part[w];
+            sum_w = t;
+            psum[bh] = t;
+        }
+        __syncthreads();
+    }
+    const float* X = Xs + (size_t)bh * Mp * d;
+    const float* D = Xd + (size_t)bh * Mp * d;
     const double sw = (double)sum_w;
     double mx = 0.0, mr = 0.0;
-    for (int p = 0; p < Mp; ++p) {
-        const double al_p = probe_alpha(p, pg, al, qo, sw);
-        const double x = X[(size_t)p * d + j];
-        mx += al_p * x;
-        mr += al_p * ((double)D[(size_t)p * d + j] - x);
+    for (int c0 = 0; c0 < Mp; c0 += kChunk) {
+        const int n = min(kChunk, Mp - c0);
+        __syncthreads();
+        for (int e = j; e < n; e += nt) alp[e] = probe_alpha(c0 + e, pg, al, qo, sw);
+        __syncthreads();
+#pragma unroll 4
+        for (int q = 0; q < n; ++q) {
+            const double x = X[(size_t)(c0 + q) * d + j];
+            mx += alp[q] * x;
+            mr += alp[q] * ((double)D[(size_t)(c0 + q) * d + j] - x);
+        }
     }
     double var = 0.0;
-    for (int p = 0; p < Mp; ++p) {
-        const double al_p = probe_alpha(p, pg, al, qo, sw);
-        const double c = (double)X[(size_t)p * d + j] - mx;
-        var += al_p * c * c;
+    for (int c0 = 0; c0 < Mp; c0 += kChunk) {
+        const int n = min(kChunk, Mp - c0);
+        __syncthreads();
+        for (int e = j; e < n; e += nt) alp[e] = probe_alpha(c0 + e, pg, al, qo, sw);
+        __syncthreads();
+#pragma unroll 4
+        for (int q = 0; q < n; ++q) {
+            const double c = (double)X[(size_t)(c0 + q) * d + j] - mx;
+            var += alp[q] * c * c;
+        }
     }
     const double sg = sqrt(var + (double)eps_std);
     double* fs = fstat + (size_t)bh * 3 * d;
@@ -238,19 +260,48 @@ __global__ void fit_solve_kernel(const double* __restrict__ G, double* __restric
         for (int e = tid; e < d * d; e += blockDim.x) Bout[(size_t)bh * d * d + e] = 0.f;
         return;
     }
-    double* R = rhs + (size_t)bh * d * d;
-    for (int j = tid; j < d; j += blockDim.x) {
-        for (int i = 0; i < d; ++i) {   // L y = rhs_j
-            double acc = R[(size_t)i * d + j];
-            for (int k = 0; k < i; ++k) acc -= Ls[i * ld + k] * R[(size_t)k * d + j];
-            R[(size_t)i * d + j] = acc / Ls[i * ld + i];
+    // Forward and back substitution for 64 right-hand-side columns at a time,
+    // staged in shared memory (Ys[i * 65 + c]); thread c < 64 solves column
+    // j0 + c on its own (four partial sums in a fixed order break the
+    // dependency chain), so no barrier is needed inside a solve.
+    const double* R = rhs + (size_t)bh * d * d;
+    double* Ys = Ls + d * ld;
+    constexpr int W = 64, LDY = W + 1;
+    for (int j0 = 0; j0 < d; j0 += W) {
+        __syncthreads();
+        for (int e = tid; e < d * W; e += blockDim.x) Ys[(e / W) * LDY + (e % W)] = R[(size_t)(e / W) * d + j0 + (e % W)];
+        __syncthreads();
+        if (tid < W) {
+            double* y = Ys + tid;
+            for (int i = 0; i < d; ++i) {   // L y = rhs
+                const double* li = Ls + i * ld;
+                double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+                int k = 0;
+                for (; k + 4 <= i; k += 4) {
+                    a0 += li[k] * y[k * LDY];
+                    a1 += li[k + 1] * y[(k + 1) * LDY];
+                    a2 += li[k + 2] * y[(k + 2) * LDY];
+                    a3 += li[k + 3] * y[(k + 3) * LDY];
+                }
+                for (; k < i; ++k) a0 += li[k] * y[k * LDY];
+                y[i * LDY] = (y[i * LDY] - ((a0 + a1) + (a2 + a3))) / li[i];
+            }
+            for (int i = d - 1; i >= 0; --i) {   // L^T b = y
+                double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+                int k = i + 1;
+                for (; k + 4 <= d; k += 4) {
+                    a0 += Ls[k * ld + i] * y[k * LDY];
+                    a1 += Ls[(k + 1) * ld + i] * y[(k + 1) * LDY];
+                    a2 += Ls[(k + 2) * ld + i] * y[(k + 2) * LDY];
+                    a3 += Ls[(k + 3) * ld + i] * y[(k + 3) * LDY];
+                }
+                for (; k < d; ++k) a0 += Ls[k * ld + i] * y[k * LDY];
+                y[i * LDY] = (y[i * LDY] - ((a0 + a1) + (a2 + a3))) / Ls[i * ld + i];
+            }
         }
-        for (int i = d - 1; i >= 0; --i) {   // L^T b = y
-            double acc = R[(size_t)i * d + j];
-            for (int k = i + 1; k < d; ++k) acc -= Ls[k * ld + i] * R[(size_t)k * d + j];
-            R[(size_t)i * d + j] = acc / Ls[i * ld + i];
-        }
-        for (int i = 0; i < d; ++i) Bout[((size_t)bh * d + i) * d + j] = (float)R[(size_t)i * d + j];
+        __syncthreads();
+        for (int e = tid; e < d * W; e += blockDim.x)
+            Bout[((size_t)bh * d + (e / W)) * d + j0 + (e % W)] = (float)Ys[(e / W) * LDY + (e % W)];
     }
 }
 
@@ -364,7 +415,7 @@ sparsepr_status run_fit(const sparsepr_params& p, const Plan& pl, const sparsepr
                                                                        part.q_offsets, psum, pl.Cq, Mp, d, p.lambda,
                                                                        fstat, G, rhs, S);
     if (p.correction == SPARSEPR_CORRECTION_FULL) {
-        const size_t smem = (size_t)d * (d + 1) * sizeof(double);
+        const size_t smem = (size_t)(d * (d + 1) + d * 65) * sizeof(double);
         cudaFuncSetAttribute(fit_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         count_launch(), fit_solve_kernel<<<BH, d, smem, st>>>(G, rhs, d, f.B, status);
     } else {
