@@ -65,6 +65,15 @@ def test_validation_codes(L):
     assert validate(_cfg(kmeans_iters=0)) == 1
     assert validate(_cfg(density=float("nan"))) == 1
     assert validate(_cfg(M=-1)) == 1
+    # probe / correction variants, rank truncation, GQA
+    assert validate(_cfg(probe_select="random")) == 0 and validate(_cfg(correction="mean")) == 0
+    assert validate(_cfg(residual_rank=8)) == 0 and validate(_cfg(residual_rank=65)) == 1
+    assert validate(_cfg(H=4, Hkv=2)) == 0
+    assert validate(_cfg(H=4, Hkv=3)) == 1                    # H not a multiple of Hkv
+    assert validate(_cfg(H=4, Hkv=-1)) == 1
+    from free_block_sparse_sampled_b200 import _abi
+    assert validate(_cfg(H=4, Hkv=2, flags=_abi.FLAG_WARM_START)) == 2   # warm state is per query head
+    assert validate(_cfg(H=4, Hkv=4, flags=_abi.FLAG_WARM_START)) == 0
 
 
 def test_workspace_size_and_host_errors(L):
@@ -89,7 +98,8 @@ def test_workspace_size_and_host_errors(L):
 def test_ctypes_layouts_match_c(L):
     from free_block_sparse_sampled_b200 import _abi
     structs = {"sparsepr_params": _abi.Params, "sparsepr_partition_out": _abi.PartitionOut,
-               "sparsepr_route_out": _abi.RouteOut, "sparsepr_fit_out": _abi.FitOut, "sparsepr_stats": _abi.Stats}
+               "sparsepr_route_out": _abi.RouteOut, "sparsepr_fit_out": _abi.FitOut, "sparsepr_stats": _abi.Stats,
+               "sparsepr_warm_state": _abi.WarmState}
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "sparsepr.h"', "int main(void) {"]
     for cname, py in structs.items():
         lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
