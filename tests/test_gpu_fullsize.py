@@ -37,3 +37,41 @@ def test_full_size_call(name):
     pairs = res["route"]["pairs"].cpu().numpy()
     rho = pairs[:, 1].sum() / (cfg.BH * cfg.N * cfg.N)
     assert rho >= w.density - 1e-9
+
+
+def test_full_size_warm_call():
+    """The wide call warm-started from the previous step's state (paper C.1,
+    2 k-means assignments), in the configuration the benchmark's warm call
+    times: integer chains for two heads and sampled output rows, each fed the
+    GPU's own upstream values."""
+    import free_block_sparse_sampled_b200 as S
+    from synthetic import drift_inputs
+    w = get_workload("wide")
+    cfg0 = S.SparsePRConfig.from_workload(w)
+    x0 = generate_inputs(w, bits=False)
+    x1 = drift_inputs(w, x0, step=1)
+    d0 = to_device(w, x0)
+    ws = S.alloc_workspace(cfg0)
+    p0 = S.partition(cfg0, *d0, ws, extras=True)
+    state = {n: p0[n].clone() for n in ("F_K", "F_Q", "k_centroid", "q_centroid", "n_groups")}
+    del p0, d0
+    torch.cuda.synchronize()
+    cfg = S.SparsePRConfig.from_workload(w, kmeans_iters=2)
+    d1 = to_device(w, x1)
+    part = S.partition(cfg, *d1, ws, warm=state)
+    rt = S.route(cfg, part, ws)
+    O_sp, pd, ps = S.attention(cfg, part, rt, ws)
+    fit = S.probe_fit(cfg, part, rt, ps, pd, ws)
+    out = S.apply(cfg, part, rt, O_sp, pd, fit, ws)
+    torch.cuda.synchronize()
+    res = {"part": part, "route": rt, "O_sp": O_sp, "probe_dense": pd, "probe_sparse": ps, "fit": fit, "out": out}
+    assert S.device_status(ws) == 0
+    assert (part["kmeans_iters_run"].cpu().numpy() <= 2).all()
+    for bh in (0, cfg.BH - 1):
+        hv = head_view(res, cfg, bh)
+        check_integer_chain(hv, cfg)
+        rows = sample_rows(hv, 48, seed=bh)
+        check_attention_rows(hv, cfg, rows, TOL_ATTN)
+        check_fit_and_apply_rows(hv, cfg, rows)
+    pairs = rt["pairs"].cpu().numpy()
+    assert pairs[:, 1].sum() / (cfg.BH * cfg.N * cfg.N) >= w.density - 1e-9
