@@ -649,22 +649,32 @@ __global__ void group_mean_indirect_kernel(const float* __restrict__ phi,
     out[((size_t)bh * C + g) * R + j] = acc / (float)(e - s);
 }
 
-// d_i = |phi_Q(q_i) - c_a|  (paper A.2), by original row.
+// d_i = |phi_Q(q_i) - c_a|  (paper A.2), by original row.  A power-of-two
+// group of lanes shares a row (one float4 each, coalesced); their partial
+// sums are combined by shuffles in a fixed order.
 __global__ void query_dist_kernel(const float* __restrict__ phi, const float* __restrict__ ca,
                                   const int32_t* __restrict__ qlab, int BH, int N, int C, int R,
                                   float* __restrict__ dist) {
+    const int nq = R / 4;                  // float4 per row (R a multiple of 16, at most 128)
+    int lpr = 4;                           // lanes per row: the power of two >= nq
+    while (lpr < nq) lpr <<= 1;
+    const int rpw = 32 / lpr;              // rows per warp step
+    const int lane = threadIdx.x & 31, part = lane % lpr, slot = lane / lpr;
     const size_t total = (size_t)BH * N;
-    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
-         e += (size_t)gridDim.x * blockDim.x) {
-        const int bh = (int)(e / N);
-        const float* x = phi + e * R;
-        const float* c = ca + ((size_t)bh * C + qlab[e]) * R;
+    const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
+    for (size_t base = (blockIdx.x * (size_t)(blockDim.x >> 5) + (threadIdx.x >> 5)) * rpw; base < total;
+         base += warps * rpw) {
+        const size_t e = base + slot;
         float ss = 0.f;
-        for (int t = 0; t < R; ++t) {
-            const float df = x[t] - c[t];
-            ss = fmaf(df, df, ss);
+        if (e < total && part < nq) {
+            const int bh = (int)(e / N);
+            const float4 x = reinterpret_cast<const float4*>(phi + e * R)[part];
+            const float4 c = reinterpret_cast<const float4*>(ca + ((size_t)bh * C + qlab[e]) * R)[part];
+            const float d0 = x.x - c.x, d1 = x.y - c.y, d2 = x.z - c.z, d3 = x.w - c.w;
+            ss = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, d3 * d3)));
         }
-        dist[e] = sqrtf(ss);
+        for (int o = lpr / 2; o > 0; o >>= 1) ss += __shfl_down_sync(0xffffffffu, ss, o, lpr);
+        if (part == 0 && e < total) dist[e] = sqrtf(ss);
     }
 }
 
