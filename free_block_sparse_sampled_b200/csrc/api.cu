@@ -231,7 +231,6 @@ sparsepr_status sparsepr_validate(const sparsepr_params* p) {
     if (p->probe_select < 0 || p->probe_select > 2 || p->correction < 0 || p->correction > 3) return SPARSEPR_INVALID_ARG;
     if (p->residual_rank < 0 || p->residual_rank > p->d) return SPARSEPR_INVALID_ARG;
     if (p->Hkv < 0 || (p->Hkv > 0 && p->H % p->Hkv != 0)) return SPARSEPR_INVALID_ARG;
-    if (p->Hkv > 0 && p->Hkv < p->H && (p->flags & SPARSEPR_FLAG_WARM_START)) return SPARSEPR_UNSUPPORTED;
     if (p->d != 64 && p->d != 128) return SPARSEPR_UNSUPPORTED;
     if (p->Cq > kMaxGroups || p->Ck > kMaxGroups) return SPARSEPR_UNSUPPORTED;
     if (p->rK > kMaxRank || p->rQ > kMaxRank) return SPARSEPR_UNSUPPORTED;
@@ -272,14 +271,14 @@ sparsepr_status sparsepr_partition_warm(const sparsepr_params* p, const void* Q,
     if (!Q || !K || !V || !partition_ok(part)) return SPARSEPR_INVALID_ARG;
     if (!prev || !prev->F_K || !prev->F_Q || !prev->k_centroid || !prev->q_centroid || !prev->n_groups)
         return SPARSEPR_INVALID_ARG;
-    if (pl.G > 1) return SPARSEPR_UNSUPPORTED;   // the warm state is per query head
     if ((p->flags & SPARSEPR_FLAG_DEBUG_EXPORT) &&
         !(part->debug_kv_scores && part->debug_q_scores && part->debug_kv_hist && part->debug_q_hist))
         return SPARSEPR_INVALID_ARG;
     cudaStream_t st = as_stream(stream);
     if (cudaMemsetAsync(at<void>(ws, pl.o_status), 0, 256, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
     if (cudaMemsetAsync(at<void>(ws, pl.o_warm), 0, 4, st) != cudaSuccess) return SPARSEPR_CUDA_ERROR;
-    const WarmSource src{prev->F_K, prev->F_Q, prev->k_centroid, prev->q_centroid, prev->n_groups, nullptr};
+    // F_K is per query head in the caller's outputs: K/V head h reads query head h * G
+    const WarmSource src{prev->F_K, prev->F_Q, prev->k_centroid, prev->q_centroid, prev->n_groups, nullptr, pl.G};
     return run_partition(*p, pl, Q, K, V, *part, ws, st, &src);
 }
 
@@ -350,8 +349,9 @@ sparsepr_status sparsepr_call(const sparsepr_params* p, const void* Q, const voi
     sparsepr_params q = *p;
     q.flags &= ~SPARSEPR_FLAG_DEBUG_EXPORT;
     int32_t* warm_word = at<int32_t>(ws, pl.o_warm);
+    // the workspace keeps F_K per K/V head (stride 1); centroids and counts are per query head
     const WarmSource src{at<float>(ws, pl.o_FK), at<float>(ws, pl.o_FQ), part.k_centroid, part.q_centroid,
-                         part.n_groups, warm_word};
+                         part.n_groups, warm_word, 1};
     const bool warm = (p->flags & SPARSEPR_FLAG_WARM_START) != 0;
     if ((s = run_partition(q, pl, Q, K, V, part, ws, st, warm ? &src : nullptr)) != SPARSEPR_OK) return s;
     launch_set_word(warm_word, kWarmMagic, st);

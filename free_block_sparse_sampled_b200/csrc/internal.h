@@ -10,6 +10,8 @@ namespace spr {
 
 // Warm start (paper C.1): where the previous call's state lives.  `valid`
 // (or nullptr) points at a word that must equal kWarmMagic for it to be used.
+// Under GQA the K/V-side state of K/V head h is read at head h * fk_stride
+// (F_K) and h * G (k_centroid and n_groups, which are per query head).
 struct WarmSource {
     const float* F_K;
     const float* F_Q;
@@ -17,6 +19,7 @@ struct WarmSource {
     const float* q_centroid;
     const int32_t* n_groups;
     const int32_t* valid;
+    int fk_stride;
 };
 sparsepr_status run_partition(const sparsepr_params& p, const Plan& pl, const void* Q, const void* K,
                               const void* V, const sparsepr_partition_out& out, void* ws, cudaStream_t st,
@@ -27,6 +30,7 @@ struct WarmInit {
     const float* cbar;
     const int32_t* ng_prev;
     int which;
+    int prev_stride;   // head of the previous state = this head * prev_stride
     const float* F;
     int d;
     bool rms;
@@ -42,9 +46,9 @@ void launch_jacobi_factor(const float* A, float* F, int Rp, int r, int BH, int d
 // *word = value, in stream order (one thread).
 void launch_set_word(int32_t* word, int32_t value, cudaStream_t st);
 // Warm metric factor; heads it cannot factor get cold[bh] = 1 (else 0).
-void launch_warm_factor(const float* M, const float* Fprev, int ld_prev, int r_req, const int32_t* ng, float scale,
-                        float* F, int Rp, int32_t* r_out, int32_t* cold, const int32_t* valid, int BH, int d,
-                        cudaStream_t st);
+void launch_warm_factor(const float* M, const float* Fprev, int ld_prev, int prev_stride, int r_req, const int32_t* ng,
+                        float scale, float* F, int Rp, int32_t* r_out, int32_t* cold, const int32_t* valid, int BH,
+                        int d, cudaStream_t st);
 sparsepr_status run_route(const sparsepr_params& p, const Plan& pl, const sparsepr_partition_out& part,
                           const sparsepr_route_out& r, void* ws, cudaStream_t st);
 bool attention_uses_tc(const sparsepr_params& p);

@@ -888,8 +888,8 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
         // warm start (C.1): subspace iteration from the previous factor; heads it
         // cannot factor (or every head, without a previous state) take Jacobi
         if (warm)
-            launch_warm_factor(matK, warm->F_K, pl.RKp, pl.rK_eff, nullptr, 1.f / sqrtf((float)d), FK, pl.RKp,
-                               nullptr, coldK, warm->valid, BHk, d, st);
+            launch_warm_factor(matK, warm->F_K, pl.RKp, warm->fk_stride, pl.rK_eff, nullptr, 1.f / sqrtf((float)d),
+                               FK, pl.RKp, nullptr, coldK, warm->valid, BHk, d, st);
         count_launch(), jacobi<<<BHk, 1024, jac_smem, st>>>(matK, FK, pl.RKp, pl.rK_eff, nullptr,
                                                            1.f / sqrtf((float)d), nullptr, 16, warm ? coldK : nullptr);
         project_dispatch<T, false>(pl.RKp, K, FK, BHk, N, d, nullptr, 0.f, phiK, at<DevStatus>(ws, pl.o_status), st);
@@ -897,8 +897,8 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     // 3. paired K/V groups
     WarmInit wiK{}, wiQ{};
     if (warm) {
-        wiK = WarmInit{warm->k_centroid, warm->n_groups, 1, FK, d, false, nullptr, 0.f, warm->valid};
-        wiQ = WarmInit{warm->q_centroid, warm->n_groups, 0, FQ, d, !sem_q, rq, p.eps_rms, warm->valid};
+        wiK = WarmInit{warm->k_centroid, warm->n_groups, 1, G, FK, d, false, nullptr, 0.f, warm->valid};
+        wiQ = WarmInit{warm->q_centroid, warm->n_groups, 0, 1, FQ, d, !sem_q, rq, p.eps_rms, warm->valid};
     }
     int32_t* raw = at<int32_t>(ws, pl.o_raw);
     int32_t* rawK = G > 1 ? at<int32_t>(ws, pl.o_rawkv) : raw;
@@ -933,8 +933,8 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
         count_launch(), centred_gram_kernel<<<dim3(d / 32, d / 32, BH), dim3(32, 8), 0, st>>>(out.k_centroid, muK,
                                                                               out.n_groups, pl.Ck, d, mat);
         if (warm)
-            launch_warm_factor(mat, warm->F_Q, pl.RQp, p.rQ, out.n_groups, 1.f, FQ, pl.RQp, rq, coldQ, warm->valid,
-                               BH, d, st);
+            launch_warm_factor(mat, warm->F_Q, pl.RQp, 1, p.rQ, out.n_groups, 1.f, FQ, pl.RQp, rq, coldQ,
+                               warm->valid, BH, d, st);
         count_launch(), jacobi<<<BH, 1024, jac_smem, st>>>(mat, FQ, pl.RQp, p.rQ, out.n_groups, 1.f, rq, 16,
                                                           warm ? coldQ : nullptr);
         project_dispatch<T, true>(pl.RQp, Q, FQ, BH, N, d, rq, p.eps_rms, phiQ, at<DevStatus>(ws, pl.o_status), st);

@@ -93,9 +93,9 @@ __device__ void metric_times_basis(const float* Ms, const float* Qs, double* Ys,
 
 template <int D>
 __global__ void __launch_bounds__(kWarmThreads) warm_factor_kernel(
-    const float* __restrict__ Min, const float* Fprev, int ld_prev, int r_req, const int32_t* __restrict__ ng,
-    float scale, float* F, int Rp, int32_t* __restrict__ r_out, int32_t* __restrict__ cold,
-    const int32_t* __restrict__ valid) {
+    const float* __restrict__ Min, const float* Fprev, int ld_prev, int prev_stride, int r_req,
+    const int32_t* __restrict__ ng, float scale, float* F, int Rp, int32_t* __restrict__ r_out,
+    int32_t* __restrict__ cold, const int32_t* __restrict__ valid) {
     using S = WarmSmem<D>;
     extern __shared__ __align__(16) unsigned char wsm[];
     float* Ms = reinterpret_cast<float*>(wsm);
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kWarmThreads) warm_factor_kernel(
     r = min(r, min(Rp, kWarmRW));
 
     const float* Mh = Min + (size_t)bh * D * D;
-    const float* Fp = Fprev + (size_t)bh * D * ld_prev;
+    const float* Fp = Fprev + (size_t)bh * prev_stride * D * ld_prev;   // previous factor of head bh * prev_stride
     for (int e = tid; e < D * D; e += nt) {
         const int i = e / D, j = e % D;
         Ms[i * S::ldM + j] = 0.5f * (Mh[i * D + j] + Mh[j * D + i]);
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kWarmThreads) warm_factor_kernel(
 template <int R, bool RMS>
 __global__ void __launch_bounds__(256) warm_init_kernel(
     const float* __restrict__ phi, int N, int C, uint64_t seed, int stage, const float* __restrict__ cbar,
-    const int32_t* __restrict__ ng_prev, int which, const float* __restrict__ F, int d,
+    const int32_t* __restrict__ ng_prev, int which, int prev_stride, const float* __restrict__ F, int d,
     const int32_t* __restrict__ r_eff, float eps, const int32_t* __restrict__ valid, float* __restrict__ cen,
     float* __restrict__ hn) {
     constexpr int J = (R + 31) / 32;
@@ -202,11 +202,12 @@ __global__ void __launch_bounds__(256) warm_init_kernel(
     const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (c >= C) return;
     int n_prev = 0;
-    if (valid == nullptr || *valid == kWarmMagic) n_prev = min(max(ng_prev[bh * 2 + which], 0), C);
+    const int ph = bh * prev_stride;   // the previous call's head holding this head's state
+    if (valid == nullptr || *valid == kWarmMagic) n_prev = min(max(ng_prev[ph * 2 + which], 0), C);
     float* dst = cen + ((size_t)bh * C + c) * R;
     float ss = 0.f;
     if (c < n_prev) {
-        const float* cb = cbar + ((size_t)bh * C + c) * d;
+        const float* cb = cbar + ((size_t)ph * C + c) * d;
         const float* Fh = F + (size_t)bh * d * R;
         float z[J];
 #pragma unroll
@@ -252,11 +253,11 @@ void warm_init_r(const WarmInit& w, const float* phi, int BH, int N, int C, uint
     const dim3 grid((C + 7) / 8, BH);
     if (w.rms)
         count_launch(), warm_init_kernel<R, true><<<grid, 256, 0, st>>>(phi, N, C, seed, stage, w.cbar, w.ng_prev,
-                                                                        w.which, w.F, w.d, w.r_eff, w.eps, w.valid,
+                                                                        w.which, w.prev_stride, w.F, w.d, w.r_eff, w.eps, w.valid,
                                                                         cen, hn);
     else
         count_launch(), warm_init_kernel<R, false><<<grid, 256, 0, st>>>(phi, N, C, seed, stage, w.cbar, w.ng_prev,
-                                                                         w.which, w.F, w.d, w.r_eff, w.eps, w.valid,
+                                                                         w.which, w.prev_stride, w.F, w.d, w.r_eff, w.eps, w.valid,
                                                                          cen, hn);
 }
 
@@ -270,18 +271,18 @@ void launch_set_word(int32_t* word, int32_t value, cudaStream_t st) {
 
 size_t warm_factor_smem(int d) { return d == 128 ? WarmSmem<128>::total : WarmSmem<64>::total; }
 
-void launch_warm_factor(const float* M, const float* Fprev, int ld_prev, int r_req, const int32_t* ng, float scale,
-                        float* F, int Rp, int32_t* r_out, int32_t* cold, const int32_t* valid, int BH, int d,
-                        cudaStream_t st) {
+void launch_warm_factor(const float* M, const float* Fprev, int ld_prev, int prev_stride, int r_req, const int32_t* ng,
+                        float scale, float* F, int Rp, int32_t* r_out, int32_t* cold, const int32_t* valid, int BH,
+                        int d, cudaStream_t st) {
     const size_t smem = warm_factor_smem(d);
     if (d == 128) {
         cudaFuncSetAttribute(warm_factor_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        count_launch(), warm_factor_kernel<128><<<BH, kWarmThreads, smem, st>>>(M, Fprev, ld_prev, r_req, ng, scale, F,
-                                                                                Rp, r_out, cold, valid);
+        count_launch(), warm_factor_kernel<128><<<BH, kWarmThreads, smem, st>>>(M, Fprev, ld_prev, prev_stride, r_req, ng,
+                                                                                scale, F, Rp, r_out, cold, valid);
     } else {
         cudaFuncSetAttribute(warm_factor_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        count_launch(), warm_factor_kernel<64><<<BH, kWarmThreads, smem, st>>>(M, Fprev, ld_prev, r_req, ng, scale, F,
-                                                                               Rp, r_out, cold, valid);
+        count_launch(), warm_factor_kernel<64><<<BH, kWarmThreads, smem, st>>>(M, Fprev, ld_prev, prev_stride, r_req, ng,
+                                                                               scale, F, Rp, r_out, cold, valid);
     }
 }
 

@@ -132,7 +132,7 @@ typedef struct {
                                   routing, probes and fit stay per query head.  K and V are then
                                   [B,Hkv,N,d]; every output stays per query head (K/V-side
                                   outputs repeated G times; the debug K/V arrays are indexed by
-                                  K/V head).  Not combinable with a warm start. */
+                                  K/V head). */
 } sparsepr_params;
 
 /* Outputs of sparsepr_partition (paper §4.1).  Required unless marked
@@ -246,7 +246,9 @@ typedef struct {
  *    first call).
  * Every other step, output and error is that of sparsepr_partition.  `prev`
  * may point into `part` of the previous call: each previous value is read
- * before this call overwrites it. */
+ * before this call overwrites it.  Under GQA (p->Hkv) the state is per query
+ * head, as the outputs are; K/V head h starts from query head h*G's F_K,
+ * k_centroid and C_k'. */
 sparsepr_status sparsepr_partition_warm(const sparsepr_params* p, const void* Q, const void* K,
                                         const void* V, const sparsepr_warm_state* prev,
                                         const sparsepr_partition_out* part, void* workspace,

@@ -663,12 +663,14 @@ def sparsepr_head(q, k, v, *, bh: int, seed: int, density: float, M: int, Ms: in
     return out
 
 
-def sparsepr_gqa(qs, k, v, *, kvh: int, Ms: int, **kw):
+def sparsepr_gqa(qs, k, v, *, kvh: int, Ms: int, warms=None, **kw):
     """R19: the G query heads qs[g] of K/V head ``kvh`` (query head indices
-    kvh G + g); returns one sparsepr_head result per query head."""
+    kvh G + g); returns one sparsepr_head result per query head.  ``warms``:
+    one warm state per query head (their F_K and kbar agree)."""
     G = len(qs)
     stacked = np.concatenate([np.asarray(x, dtype=np.float64) for x in qs], axis=0)
-    return [sparsepr_head(qs[g], k, v, bh=kvh * G + g, bh_kv=kvh, metric_rows=stacked, Ms=G * Ms, **kw)
+    return [sparsepr_head(qs[g], k, v, bh=kvh * G + g, bh_kv=kvh, metric_rows=stacked, Ms=G * Ms,
+                          warm=None if warms is None else warms[g], **kw)
             for g in range(G)]
 
 

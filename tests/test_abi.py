@@ -72,8 +72,7 @@ def test_validation_codes(L):
     assert validate(_cfg(H=4, Hkv=3)) == 1                    # H not a multiple of Hkv
     assert validate(_cfg(H=4, Hkv=-1)) == 1
     from free_block_sparse_sampled_b200 import _abi
-    assert validate(_cfg(H=4, Hkv=2, flags=_abi.FLAG_WARM_START)) == 2   # warm state is per query head
-    assert validate(_cfg(H=4, Hkv=4, flags=_abi.FLAG_WARM_START)) == 0
+    assert validate(_cfg(H=4, Hkv=2, flags=_abi.FLAG_WARM_START)) == 0
 
 
 def test_workspace_size_and_host_errors(L):

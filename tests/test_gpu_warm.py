@@ -185,3 +185,91 @@ def test_fused_warm_call_matches_staged_warm_partition():
     o_flag, _ = S.call(warm_cfg, *d1, ws2)
     torch.cuda.synchronize()
     assert torch.equal(o_flag, o_cold)
+
+
+WG = Workload("warm_gqa_bf16_d128", 1, 4, 128, (3, 20, 36), "bf16", 24, 128, 0.22, 256, 100, 1.0,
+              Cq=12, Ck=48, seed=23)
+G = 2
+
+
+def _gqa_inputs(step):
+    q, k, v = generate_inputs(WG)
+    x0 = (q, np.ascontiguousarray(k[:, ::G]), np.ascontiguousarray(v[:, ::G]))
+    return x0 if step == 0 else drift_inputs(WG, x0, step=step)
+
+
+def test_warm_call_under_gqa():
+    """GQA (G = 2) warm-started from the oracle's cold GQA call: K/V head h
+    starts from query head h*G's state; every stage checked as above, with
+    the shared key metric."""
+    from free_block_sparse_sampled_b200 import SparsePRConfig
+    x0, x1 = _gqa_inputs(0), _gqa_inputs(1)
+    cfg0 = SparsePRConfig.from_workload(WG, Hkv=WG.H // G)
+    kw = O.workload_kwargs(WG)
+    Ms = kw.pop("Ms")
+    BH, d = cfg0.BH, cfg0.d
+    st = {"F_K": np.zeros((BH, d, cfg0.RKp), np.float32), "F_Q": np.zeros((BH, d, cfg0.RQp), np.float32),
+          "k_centroid": np.zeros((BH, cfg0.Ck, d), np.float32), "q_centroid": np.zeros((BH, cfg0.Cq, d), np.float32),
+          "n_groups": np.zeros((BH, 2), np.int32)}
+    q0, k0, v0 = (a.astype(np.float64) for a in x0)
+    for b in range(WG.B):
+        for h in range(WG.H // G):
+            kvh = b * (WG.H // G) + h
+            res = O.sparsepr_gqa([q0[b, h * G + g] for g in range(G)], k0[b, h], v0[b, h], kvh=kvh, Ms=Ms, **kw)
+            for g, r in enumerate(res):
+                bh = kvh * G + g
+                st["F_K"][bh, :, :r["F_K"].shape[1]] = r["F_K"]
+                st["F_Q"][bh, :, :r["F_Q"].shape[1]] = r["F_Q"]
+                st["k_centroid"][bh, :r["Ck"]] = r["kbar"]
+                st["q_centroid"][bh, :r["Cq"]] = r["qbar"]
+                st["n_groups"][bh] = (r["Cq"], r["Ck"])
+    warm = {n: torch.from_numpy(a).cuda() for n, a in st.items()}
+    cfg = SparsePRConfig.from_workload(WG, Hkv=WG.H // G, kmeans_iters=2)
+    res = _run(cfg, *to_device(WG, x1), warm)
+    assert res["status"] == 0
+    q, k, v = (a.astype(np.float64) for a in x1)
+    p = res["part"]
+    for bh in range(cfg.BH):
+        b, h = divmod(bh, cfg.H)
+        kvh = bh // G
+        hv = head_view(res, cfg, bh)
+        hv["debug_kv_scores"] = p["debug_kv_scores"][kvh].cpu().numpy()
+        hv["debug_kv_hist"] = p["debug_kv_hist"][kvh].cpu().numpy().astype(np.int64)
+        assert (hv["iters"] <= 2).all()
+        check_kmeans_chain(hv, cfg, "kv")
+        check_kmeans_chain(hv, cfg, "q")
+        check_integer_chain(hv, cfg)
+        qs = [q[b, (h // G) * G + g] for g in range(G)]
+        MK = O.key_metric(np.concatenate(qs), O.sample_indices(G * cfg.N, G * cfg.Ms))
+        rq_prev = O.query_rank(cfg.rQ, cfg.d, int(st["n_groups"][bh][1]))
+        check_partition_floats(hv, cfg, q[b, h], k[b, h // G], v[b, h // G], M_K=MK,
+                               warm={"F_K": st["F_K"][kvh * G].astype(np.float64),
+                                     "F_Q": st["F_Q"][bh][:, :rq_prev].astype(np.float64)})
+        check_attention(hv, cfg, TOL_ATTN)
+        check_fit_and_apply(hv, cfg)
+
+
+def test_fused_warm_call_under_gqa_matches_staged():
+    """The fused call keeps F_K per K/V head in its workspace and reads the
+    centroids per query head: same output as the staged path with the state
+    of a staged cold partition."""
+    import free_block_sparse_sampled_b200 as S
+    from free_block_sparse_sampled_b200 import _abi
+    d0, d1 = to_device(WG, _gqa_inputs(0)), to_device(WG, _gqa_inputs(1))
+    cold_cfg = _cfg(WG, Hkv=WG.H // G)
+    warm_cfg = _cfg(WG, Hkv=WG.H // G, kmeans_iters=2, flags=_abi.FLAG_WARM_START)
+    plain_cfg = _cfg(WG, Hkv=WG.H // G, kmeans_iters=2)
+    ws = S.alloc_workspace(cold_cfg)
+    S.call(cold_cfg, *d0, ws)
+    o_warm, _ = S.call(warm_cfg, *d1, ws)
+    ws2 = S.alloc_workspace(cold_cfg)
+    p0 = S.partition(cold_cfg, *d0, ws2, extras=True)
+    state = {n: p0[n].clone() for n in ("F_K", "F_Q", "k_centroid", "q_centroid", "n_groups")}
+    part = S.partition(plain_cfg, *d1, ws2, warm=state)
+    rt = S.route(plain_cfg, part, ws2)
+    O_sp, pd, ps = S.attention(plain_cfg, part, rt, ws2)
+    fit = S.probe_fit(plain_cfg, part, rt, ps, pd, ws2)
+    o_staged = S.apply(plain_cfg, part, rt, O_sp, pd, fit, ws2)
+    torch.cuda.synchronize()
+    assert S.device_status(ws) == 0 and S.device_status(ws2) == 0
+    assert torch.equal(o_warm, o_staged)
