@@ -8,7 +8,9 @@
 //   O^_i = O^dense_i for probes,  O^sp_i + mu_R + Xbar_i B otherwise.
 //
 // The fit is small (M x d and d x d per head) and runs in fp64; B and the
-// statistics are stored in fp32 for the fp32 apply.
+// statistics are stored in fp32 for the fp32 apply.  Restricted families
+// (D.4: diagonal, scalar, mean-only) replace the solve, and a rank-r
+// truncation (D.3) projects B on the leading eigenvectors of Rbar^T W Rbar.
 #include "common.cuh"
 #include "internal.h"
 

@@ -7,6 +7,10 @@
 //   kbar, vbar, mu_K, M_Q = Ktilde^T Ktilde / (C_k' d), F_Q, phi_Q = RMSNorm(q F_Q)
 //   k-means with C_q requested centres -> query groups, qbar, c_a, d_i
 //
+// Variants: a warm start from the previous call's state (C.1; warm.cu), the
+// semantic partition on raw key / query rows (§3, Table 2), and GQA, where the
+// query heads of one K/V head share M_K, F_K and the K/V groups (§4.3, C.1).
+//
 // Every reduction that feeds an integer decision runs in a fixed order: the
 // k-means centre update sums members in the order of a stable counting sort,
 // never through floating-point atomics.

@@ -9,7 +9,9 @@
 //   Per query group: rank K/V groups by descending s (ties: lower index) and
 //   keep the shortest prefix whose key count reaches the budget beta.
 //   Probes: m_a by largest remainder on M|G_a|/N, the m_a rows of smallest
-//   (d_i, i) inside each group, coverage weights w~_p = M w_p / sum w.
+//   (d_i, i) inside each group, coverage weights w~_p = M w_p / sum w; or
+//   (Table 4) M random rows or M rows evenly spaced over the grid, with the
+//   coverage weights of the counts that fall in each group.
 #include "common.cuh"
 #include "internal.h"
 
