@@ -78,3 +78,30 @@ def test_gqa_with_one_group_is_the_plain_call():
     a = run_staged(S.SparsePRConfig.from_workload(W), *d)
     b = run_staged(S.SparsePRConfig.from_workload(W, Hkv=W.H), *d)
     assert torch.equal(a["out"], b["out"])
+
+
+def test_gqa_semantic_partition():
+    """GQA with the semantic partition: the K/V head's raw keys are
+    clustered once and the groups serve its G query heads."""
+    from free_block_sparse_sampled_b200 import SparsePRConfig, _abi
+    cfg = SparsePRConfig.from_workload(W, Hkv=W.H // G,
+                                       flags=_abi.FLAG_SEMANTIC_KEYS | _abi.FLAG_SEMANTIC_QUERIES)
+    q, k, v = _inputs()
+    res = run_staged(cfg, *to_device(W, (q, k, v)), debug=True)
+    assert res["status"] == 0
+    p = res["part"]
+    for bh in range(cfg.BH):
+        b, h = divmod(bh, cfg.H)
+        kvh = bh // G
+        hv = head_view(res, cfg, bh)
+        hv["debug_kv_scores"] = p["debug_kv_scores"][kvh].cpu().numpy()
+        hv["debug_kv_hist"] = p["debug_kv_hist"][kvh].cpu().numpy().astype(np.int64)
+        if bh % G:
+            assert np.array_equal(hv["kv_label"], head_view(res, cfg, bh - 1)["kv_label"])
+        check_kmeans_chain(hv, cfg, "kv")
+        check_kmeans_chain(hv, cfg, "q")
+        check_integer_chain(hv, cfg)
+        check_partition_floats(hv, cfg, q[b, h].astype(np.float64), k[b, h // G].astype(np.float64),
+                               v[b, h // G].astype(np.float64), semantic_keys=True, semantic_queries=True)
+        check_attention(hv, cfg, TOL_ATTN)
+        check_fit_and_apply(hv, cfg)
