@@ -814,3 +814,32 @@ def test_gqa_heads_share_the_kv_partition():
     one = O.sparsepr_gqa([q], k, v, kvh=0, Ms=w.Ms, **kw)[0]
     ref = O.sparsepr_head(q, k, v, bh=0, Ms=w.Ms, **kw)
     np.testing.assert_array_equal(one["O"], ref["O"])
+
+
+def test_gqa_warm_start_keeps_converged_shared_groups():
+    """Warm-starting a GQA call from its own converged state reproduces the
+    shared K/V groups (one assignment from the converged centres)."""
+    w, q, k, v = _tiny_head()
+    kw = O.workload_kwargs(w)
+    Ms = kw.pop("Ms")
+    kw.update(kmeans_iters=200, kmeans_tol=0.0)
+    qs = [q, q[::-1].copy()]
+    cold = O.sparsepr_gqa(qs, k, v, kvh=0, Ms=Ms, **kw)
+    kw["kmeans_iters"] = 2
+    warm = O.sparsepr_gqa(qs, k, v, kvh=0, Ms=Ms, warms=[O.warm_state(r) for r in cold], **kw)
+    for c, r in zip(cold, warm):
+        assert r["warm_factor_used"][0]
+        assert np.array_equal(r["kv_labels"], c["kv_labels"])
+    assert np.array_equal(warm[0]["kv_labels"], warm[1]["kv_labels"])
+
+
+def test_drift_inputs_are_seeded_and_small():
+    from synthetic import drift_inputs, generate_inputs
+    from synthetic import get_workload
+    w = get_workload("tiny", grid=(2, 8, 8))
+    x0 = generate_inputs(w)
+    a, b = drift_inputs(w, x0, step=1), drift_inputs(w, x0, step=1)
+    c = drift_inputs(w, x0, step=2)
+    for u, u2, u3, x in zip(a, b, c, x0):
+        assert np.array_equal(u, u2) and not np.array_equal(u, u3)
+        assert 0.02 < np.std(u - x) / np.std(x) < 0.08
