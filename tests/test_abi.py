@@ -90,6 +90,18 @@ def test_workspace_size_and_host_errors(L):
     assert L.sparsepr_call(ctypes.byref(p), q, q, q, q, None, ctypes.c_void_p((1 << 20) + 8), n, None) == 1
     assert L.sparsepr_call(ctypes.byref(bad), q, q, q, q, None, fake, n, None) == 1
     assert L.sparsepr_get_device_status(None, None, None) == 1
+    # the warm-started partition checks its previous state before anything runs
+    part = _abi.PartitionOut(*[q] * len(_abi.PARTITION_FIELDS))
+    assert L.sparsepr_partition_warm(ctypes.byref(p), q, q, q, None, ctypes.byref(part), fake, n, None) == 1
+    prev = _abi.WarmState(q, q, q, None, q)
+    assert L.sparsepr_partition_warm(ctypes.byref(p), q, q, q, ctypes.byref(prev), ctypes.byref(part), fake, n,
+                                     None) == 1
+    assert L.sparsepr_partition_warm(ctypes.byref(p), q, q, q, ctypes.byref(prev), ctypes.byref(part), fake, 16,
+                                     None) == 3
+    # variant parameters change the workspace plan only where they add buffers
+    n_rank = L.sparsepr_workspace_size(ctypes.byref(_cfg(residual_rank=8).c_params()))
+    n_sem = L.sparsepr_workspace_size(ctypes.byref(_cfg(flags=_abi.FLAG_SEMANTIC_KEYS).c_params()))
+    assert n_rank > n and n_sem >= n
     assert L.sparsepr_status_string(6) == b"ridge Gram matrix not positive definite"
     assert _abi.STATUS_NAMES[5] == "TIMEOUT"
 
