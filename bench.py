@@ -448,6 +448,22 @@ def run_ours(args, w):
         ms_dense = d0.elapsed_time(d1) / 3
         extras["dense_sdpa_ms"] = ms_dense
         extras["speedup_vs_dense_sdpa"] = ms_dense / ms_step
+        # our own attention kernel at full routed density (every cell selected):
+        # the dense reference of the same kernel, timed inside a whole call
+        try:
+            import dataclasses as _dc
+            dcfg = _dc.replace(cfg, density=1.0 + cfg.Mp / cfg.N)
+            wsd = S.alloc_workspace(dcfg, dev)
+            outd = torch.empty_like(out)
+            S.call(dcfg, q, k, v, wsd, outd)
+            _, dst = S.call(dcfg, q, k, v, wsd, outd, stats=True)
+            extras["own_kernel_full_density"] = {
+                "attention_ms": dst["ms_attention"], "call_ms": dst["ms_total"],
+                "attention_tflops": 4.0 * cfg.d * dst["pairs_exec"] / (dst["ms_attention"] * 1e-3) / 1e12,
+                "rho_exec": dst["rho_exec"]}
+            del wsd, outd
+        except Exception as exc:   # a reference measurement only: never lose the bench line over it
+            extras["own_kernel_full_density"] = {"error": repr(exc)[:200]}
         # accuracy on unprobed rows: 2048 evenly spaced rows per head vs fp32 dense
         S.call(cfg, q, k, v, ws, out)
         rows = torch.linspace(0, cfg.N - 1, 2048, device=dev).long()
@@ -534,6 +550,7 @@ def run_ours(args, w):
             "gpu_launches": launches * args.steps, "clocks": clocks,
             "exec_pair_tflops": 4.0 * cfg.d * pairs_exec / (ms_step * 1e-3) / 1e12,
             "attention_exec_pair_tflops": achieved, "attention_ms": ms_attn,
+            "attention_route_pair_tflops": 4.0 * cfg.d * pairs_route / (ms_attn * 1e-3) / 1e12,
             "rho_exec": st["rho_exec"], "pairs_route": pairs_route, "pairs_exec": pairs_exec,
             "pairs_visited": int(br[0]["pairs_visited"]),
             "breakdown_ms": {k_: st[k_] for k_ in ("ms_partition", "ms_route", "ms_attention", "ms_fit",
