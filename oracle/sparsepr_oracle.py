@@ -83,6 +83,12 @@ R19 GQA (§4.3 "Routing and GQA", C.1): the G query heads of one K/V head
     (all rows when fewer); the K/V k-means draws its initial rows from the
     K/V head's stream (head index = K/V head).  Query groups, routing,
     probes and the fit stay per query head, with the query head's streams.
+
+Parity unpinned: these functions carry only internal invariants, because no
+printed value or closed form fixes them -- routing_score (the prose around
+B.3 is lost; it is checked against its own definition), probe_allocation and
+probe_select (the A.2 rule is lost), the key_factor scale, kmeans_stop_count,
+the key_budget rounding and the mu_K definition.
 """
 
 from __future__ import annotations
