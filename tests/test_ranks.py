@@ -2,6 +2,8 @@
 torch.distributed.run would launch them, take the barrier and the maximum of
 their step times, and the job value counts one call per rank."""
 
+import hashlib
+import json
 import os
 import socket
 import sys
@@ -59,3 +61,20 @@ def test_single_rank_needs_no_process_group():
     ranks.barrier()
     ranks.close()
     assert bench.whole_job_ms_per_call(12.0, 1) == 12.0
+
+
+def test_profiled_traffic_only_for_the_captured_kernel_and_workload():
+    """The bench reports the ncu DRAM traffic only while the attention source
+    is the one captured, and only for the captured workload, scaled by heads."""
+    import bench
+    from synthetic import get_workload
+    w = get_workload("wide")
+    t = bench.profiled_traffic(w)
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "attention_tc_wide_h4.json")))
+    src = open(os.path.join(bench.ROOT, rec["source"]), "rb").read()
+    if hashlib.sha256(src).hexdigest() == rec["source_sha256"]:
+        assert t == (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * 40 / rec["heads"]
+        assert bench.profiled_traffic(w.replace(name="wide_h4", H=4)) == rec["dram_bytes_read"] + rec["dram_bytes_write"]
+    else:
+        assert t is None
+    assert bench.profiled_traffic(get_workload("large")) is None
