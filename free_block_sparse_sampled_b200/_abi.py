@@ -22,7 +22,7 @@ CORRECTIONS = {"full": 0, "diagonal": 1, "scalar": 2, "mean": 3}
 EXPORTED = ["sparsepr_status_string", "sparsepr_validate", "sparsepr_workspace_size",
             "sparsepr_partition", "sparsepr_route", "sparsepr_attention", "sparsepr_probe_fit",
             "sparsepr_apply", "sparsepr_call", "sparsepr_last_error_string", "sparsepr_get_device_status",
-            "sparsepr_probe_fit_static", "sparsepr_partition_warm"]
+            "sparsepr_probe_fit_static", "sparsepr_partition_warm", "sparsepr_debug_stall_attention"]
 
 # size of the static scratch array behind sparsepr_probe_fit_static
 FIT_STATIC_SCRATCH_BYTES = 8 << 20
@@ -126,6 +126,8 @@ def lib() -> ctypes.CDLL:
         L.sparsepr_probe_fit_static.restype = ctypes.c_int32
         L.sparsepr_probe_fit_static.argtypes = [ctypes.POINTER(Params), ctypes.POINTER(PartitionOut),
                                                 ctypes.POINTER(RouteOut), P, P, ctypes.POINTER(FitOut), P, P]
+        L.sparsepr_debug_stall_attention.restype = None
+        L.sparsepr_debug_stall_attention.argtypes = [ctypes.c_uint32]
         _LIB = L
     return _LIB
 

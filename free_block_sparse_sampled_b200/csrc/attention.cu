@@ -19,6 +19,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -261,7 +262,8 @@ constexpr int kSoftPairs = SPR_SOFT_PAIRS;
 static_assert(kSoftPairs >= 0 && kSoftPairs <= 16, "soft pairs per 16");
 enum { B_Q = 0, B_KF = 1, B_KE = B_KF + NS, B_VF = B_KE + NS, B_VE = B_VF + NS, B_SF = B_VE + NS,
        B_PF = B_SF + 2, B_OF = B_PF + 2, B_DR = B_OF + 1, B_MF = B_DR + 1, B_ME = B_MF + RING,
-       N_BAR = B_ME + RING };
+       B_ST = B_ME + RING,   // never signalled: the stall hook's wait (sparsepr_debug_stall_attention)
+       N_BAR = B_ST + 1 };
 
 template <int D>
 struct Layout {
@@ -322,7 +324,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
     int n_probe_items, int N, int Mp, int Cq, int Ck, int total_rows, const int32_t* __restrict__ kv_off,
     const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_groups, const float* __restrict__ vscale,
     float* __restrict__ O_sp, float* __restrict__ probe_dense, DevStatus* status,
-    unsigned long long* __restrict__ visited, float scale_log2) {
+    unsigned long long* __restrict__ visited, float scale_log2, uint32_t stall_polls) {
     using namespace tc;
     using namespace sm100;
     using L = Layout<D>;
@@ -357,6 +359,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
         }
         mbar_init(bar(B_OF), 1);
         mbar_init(bar(B_DR), 1);
+        mbar_init(bar(B_ST), 1);
         for (int s = 0; s < RING; ++s) {
             mbar_init(bar(B_MF + s), 1);
             mbar_init(bar(B_ME + s), 128 * nq);
@@ -543,7 +546,10 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
                         mma_f16_ts(tmem + 256 + D * t, tmem + 128 * t + kk * 8, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                     }
                 };
-                bool ok = mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
+                // Stall hook (testing the timeout path): a bounded wait on a
+                // barrier nothing signals runs out before any MMA is issued.
+                bool ok = stall_polls == 0 || mbar_wait(bar(B_ST), 0, abort_flag, stall_polls);
+                ok = ok && mbar_wait(bar(B_Q), 0, abort_flag, kSpin);
                 for (int j = 0; ok && j < n_tiles; ++j) {
                     const int stage = j % NS;
                     if (!mbar_wait(bar(B_KF + stage), (j / NS) & 1, abort_flag, kSpin)) { ok = false; break; }
@@ -814,6 +820,8 @@ bool tc_register_split_ok(int d) {
     return true;
 }
 
+std::atomic<uint32_t> g_stall_polls{0};
+
 inline int grid_for(size_t total, int threads) {
     size_t g = (total + threads - 1) / threads;
     return (int)(g > 148 * 64 ? 148 * 64 : (g == 0 ? 1 : g));
@@ -882,14 +890,16 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
             count_launch(), k<<<grid2, tc::kThreads, tc::Layout<128>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
                                                                        pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
                                                                        r.sel_count, r.sel_groups, vscale, O_sp,
-                                                                       probe_dense, status, visited, scale_log2);
+                                                                       probe_dense, status, visited, scale_log2,
+                                                                       g_stall_polls.load());
         } else {
             auto k = attention_tc_kernel<64>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<64>::smem);
             count_launch(), k<<<grid2, tc::kThreads, tc::Layout<64>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
                                                                       pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
                                                                       r.sel_count, r.sel_groups, vscale, O_sp,
-                                                                      probe_dense, status, visited, scale_log2);
+                                                                      probe_dense, status, visited, scale_log2,
+                                                                      g_stall_polls.load());
         }
     } else {
         const int threads = 2 * pl.BM;
@@ -914,3 +924,5 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
 }
 
 }  // namespace spr
+
+extern "C" void sparsepr_debug_stall_attention(uint32_t polls) { spr::g_stall_polls.store(polls); }

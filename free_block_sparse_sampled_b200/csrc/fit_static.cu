@@ -53,7 +53,9 @@ StaticLayout static_layout(size_t BH, size_t d) {
 
 // Device address of the scratch array on the current device, looked up once
 // per device.  The lookup may load the module, so the first call on a device
-// should come before any stream capture.
+// should come before any stream capture.  The cached address belongs to the
+// context current at that lookup and is not refreshed: it does not survive a
+// cudaDeviceReset of the device.
 sparsepr_status scratch_address(void** out) {
     int dev = 0;
     sparsepr_status s = cuda_status(cudaGetDevice(&dev));

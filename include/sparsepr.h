@@ -309,7 +309,13 @@ sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const sparsepr_part
  * before anything is launched; sparsepr_last_error_string() then gives the
  * bytes needed and the limit.  Other checks as sparsepr_probe_fit.
  * The first call on a device looks up the array's device address (which can
- * load the module); make that first call before any stream capture.
+ * load the module); make that first call before any stream capture.  The
+ * address is kept per device index for the life of the process and belongs
+ * to the device context that was current at that first call: after
+ * cudaDeviceReset, or anything else that destroys and re-creates the
+ * device's primary context, the module may load at another address, so a
+ * process that resets a device must not call this entry point on that
+ * device again.
  * Every call on a device shares the array and finds the previous call's
  * contents there; each call clears the status word it needs zeroed, and the
  * rest is fully rewritten before it is read.  Calls whose work overlaps on
@@ -342,6 +348,19 @@ const char* sparsepr_last_error_string(void);
 /* Reads (synchronously on `stream`) and clears the device status word of
  * `workspace`: *out = SPARSEPR_OK or the first device-side failure. */
 sparsepr_status sparsepr_get_device_status(void* workspace, void* stream, int32_t* out);
+
+/* Testing hook for the device-timeout path (no counterpart in the paper).
+ * While polls > 0, every block of the tensor-core attention kernel launched
+ * afterwards (by sparsepr_attention or sparsepr_call, from any host thread)
+ * first waits at most `polls` polls on an mbarrier that nothing signals.  The
+ * wait runs out like any bounded wait that gives up: the kernel records
+ * SPARSEPR_TIMEOUT in the workspace status word, stops its other warps, lets
+ * the copies and MMAs it issued finish, frees its tensor memory and returns,
+ * and the blocks that start later return at once.  O_sp and the probe rows of
+ * such a call are undefined.  polls = 0 (the default) turns the hook off.
+ * Nothing else uses it; it exists so that tests can check that a timed-out
+ * kernel leaves the context usable and the status readable. */
+void sparsepr_debug_stall_attention(uint32_t polls);
 
 #ifdef __cplusplus
 }

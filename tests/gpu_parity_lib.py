@@ -232,13 +232,17 @@ def _tf32(x):
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
-def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, semantic_queries=False, M_K=None):
+def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, semantic_queries=False, M_K=None,
+                           score_rows=None):
     """Float outputs of the partition against fp64 recomputation from the
     GPU's own integer decisions.  ``warm`` (F_K, F_Q of the state a warm call
     started from, fp64) switches the factor references to the warm factor;
     a semantic side has the raw rows (TF32-rounded) as coordinates and the
     identity as its factor.  ``M_K`` overrides the key metric (GQA: the
-    metric the query heads of one K/V head share)."""
+    metric the query heads of one K/V head share).  ``score_rows`` limits the
+    routing-score comparison to those query groups (default: all).
+    Returns which cold factors were compared: a factor whose metric has no
+    spectral gap at the truncation rank is not unique and is skipped."""
     kl, ql = h["kv_label"], h["q_label"]
     np.testing.assert_allclose(h["k_centroid"], O.group_means(k, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
     np.testing.assert_allclose(h["v_centroid"], O.group_means(v, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
@@ -266,11 +270,13 @@ def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, sema
     FK = h["F_K"]
     gap_ok = (r == cfg.d or (w[r - 1] - w[r]) > 1e-2 * w[0]) and not semantic_keys
     Fw = None if warm is None else O.warm_factor(MK, warm["F_K"], r, 1.0 / math.sqrt(cfg.d))
+    compared = {"F_K": False, "F_Q": False}
     if Fw is not None:
         ref = Fw @ Fw.T
         assert np.abs(FK @ FK.T - ref).max() <= 2e-4 * np.abs(ref).max(), "warm F_K"
     elif gap_ok:
         assert np.abs(FK @ FK.T - ref).max() <= 2e-4 * np.abs(ref).max()
+        compared["F_K"] = True
     MQ = O.query_metric(h["k_centroid"])
     wq, Uq = O.eigh_desc(MQ)
     refq = Uq[:, :rq] @ np.diag(wq[:rq]) @ Uq[:, :rq].T
@@ -281,10 +287,13 @@ def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, sema
         assert np.abs(FQ @ FQ.T - refq).max() <= 2e-4 * np.abs(refq).max(), "warm F_Q"
     elif not semantic_queries and (rq >= int((wq > 1e-9 * wq[0]).sum()) or (wq[rq - 1] - wq[rq]) > 1e-2 * wq[0]):
         assert np.abs(FQ @ FQ.T - refq).max() <= 2e-4 * np.abs(refq).max()
+        compared["F_Q"] = True
     # routing scores vs the direct sum on the GPU's groups and centroids
-    s_ref = O.routing_score(h["q_centroid"], k, v, h["k_centroid"], h["v_centroid"], kl)
+    rows = np.arange(h["Cq"]) if score_rows is None else np.asarray(score_rows)
+    s_ref = O.routing_score(h["q_centroid"][rows], k, v, h["k_centroid"], h["v_centroid"], kl)
     scale = np.abs(s_ref).max(axis=1, keepdims=True)
-    assert np.all(np.abs(h["score"] - s_ref) <= 2e-4 * scale + 1e-30)
+    assert np.all(np.abs(h["score"][rows] - s_ref) <= 2e-4 * scale + 1e-30)
+    return compared
 
 
 def sample_rows(h, n, seed=0):

@@ -24,7 +24,7 @@ def L():
 
 def _declared_functions():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:const char\*|sparsepr_status|size_t)\s+(sparsepr_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const char\*|sparsepr_status|size_t|void)\s+(sparsepr_\w+)\s*\(", text, re.M)))
 
 
 def test_header_declares_the_boundary():

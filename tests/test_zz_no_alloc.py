@@ -5,8 +5,8 @@ device memory where they run the fit: their framework's caching allocator
 owns all free HBM, or they must not take the device-wide synchronisation of
 cudaMalloc/cudaFree.  This entry point keeps the fit's scratch in a static
 device array instead.  These tests call it through the C ABI and compare it
-with sparsepr_probe_fit on the same inputs, on two calls in a row (the array
-keeps the previous call's contents), and check that a call whose scratch
+with sparsepr_probe_fit, on two calls in a row on different inputs (the
+array keeps the previous call's contents), and check that a call whose scratch
 would exceed the array is refused before anything runs.
 
 The file is named so that pytest collects it after every other test file.
@@ -60,18 +60,28 @@ def test_static_fit_refuses_oversized_call():
     assert "sparsepr_probe_fit_static" in msg and str(limit) in msg
 
 
-@pytest.mark.gpu
-def test_static_fit_matches_workspace_fit_twice():
-    if not torch.cuda.is_available():
-        pytest.skip("needs a CUDA GPU")
+def test_static_fit_limit_matches_header():
+    """The binding's copy of the array size is the header's."""
+    import os
+    import re
+    _, A = _lib_and_abi()
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                            "sparsepr.h")).read()
+    m = re.search(r"#define SPARSEPR_FIT_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
+    assert m is not None
+    assert A.FIT_STATIC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def _fit_inputs(w):
+    """Partition, routing and probe rows of workload ``w`` on the GPU, and the
+    workspace fit of the same inputs as the reference."""
     import free_block_sparse_sampled_b200 as S
     from free_block_sparse_sampled_b200 import SparsePRConfig
-    from free_block_sparse_sampled_b200.api import _p, _stream
-    lib, A = _lib_and_abi()
-    cfg = SparsePRConfig.from_workload(CASE)
-    assert _static_scratch_bytes(cfg.BH, cfg.d) <= A.FIT_STATIC_SCRATCH_BYTES
-    q, k, v = generate_inputs(CASE)
     from synthetic.video_grid import bf16_bits
+    _, A = _lib_and_abi()
+    cfg = SparsePRConfig.from_workload(w)
+    assert _static_scratch_bytes(cfg.BH, cfg.d) <= A.FIT_STATIC_SCRATCH_BYTES
+    q, k, v = generate_inputs(w)
     dev = [torch.from_numpy(bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda() for a in (q, k, v)]
     ws = S.alloc_workspace(cfg)
     part = S.partition(cfg, *dev, ws)
@@ -80,8 +90,22 @@ def test_static_fit_matches_workspace_fit_twice():
     ref = S.probe_fit(cfg, part, rt, ps, pd, ws)
     torch.cuda.synchronize()
     assert S.device_status(ws) == 0
+    return cfg, part, rt, ps, pd, ref
+
+
+@pytest.mark.gpu
+def test_static_fit_matches_workspace_fit_twice():
+    """Two calls in a row on different inputs: three heads, then two heads of
+    another seed.  Scratch the second call failed to rewrite would still hold
+    the first call's values, which belong to other inputs, so each call is
+    compared with the workspace fit of its own inputs."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from free_block_sparse_sampled_b200.api import _p, _stream
+    lib, A = _lib_and_abi()
     names = ["B", "mu_x", "sigma", "mu_r"]
-    for call in range(2):
+    for call, w in enumerate([CASE.replace(H=3), CASE.replace(name="no_alloc_fit_2", seed=22)]):
+        cfg, part, rt, ps, pd, ref = _fit_inputs(w)
         # outputs start as NaN so that anything left unwritten shows
         out = {n: torch.full_like(ref[n], float("nan")) for n in names}
         st = torch.full((1,), -1, dtype=torch.int32, device="cuda")
