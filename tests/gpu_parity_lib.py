@@ -232,6 +232,25 @@ def _tf32(x):
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+def check_factor_spectral(F, M, r, scale):
+    """A metric factor F = U_r sqrt(Lambda_r) * scale checked without needing a
+    spectral gap at r: its columns are orthogonal, each column f is an
+    eigenvector of M with eigenvalue |f|^2 / scale^2, and those eigenvalues are
+    the r largest of M.  Where eigenvalues cluster around the truncation rank,
+    F F^T is not unique but these properties still hold (Weyl's bound)."""
+    Fr = F[:, :r]
+    lam = (Fr * Fr).sum(0) / scale ** 2
+    w, _ = O.eigh_desc(M)
+    top = w[0]
+    assert np.all(np.abs(np.sort(lam)[::-1] - w[:r]) <= 2e-4 * top), "factor eigenvalues"
+    G = Fr.T @ Fr
+    off = G - np.diag(np.diag(G))
+    assert np.abs(off).max() <= 2e-4 * top * scale ** 2, "factor columns not orthogonal"
+    res = M @ Fr - Fr * lam[None, :]
+    assert np.all(np.linalg.norm(res, axis=0) <= 1e-3 * top * np.linalg.norm(Fr, axis=0) + 1e-12), "eigen residual"
+    assert np.all(F[:, r:] == 0.0)
+
+
 def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, semantic_queries=False, M_K=None,
                            score_rows=None):
     """Float outputs of the partition against fp64 recomputation from the
@@ -241,8 +260,10 @@ def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, sema
     identity as its factor.  ``M_K`` overrides the key metric (GQA: the
     metric the query heads of one K/V head share).  ``score_rows`` limits the
     routing-score comparison to those query groups (default: all).
-    Returns which cold factors were compared: a factor whose metric has no
-    spectral gap at the truncation rank is not unique and is skipped."""
+    Returns which cold factors were compared.  Every cold factor gets the
+    gap-free spectral check; F F^T is also compared with the truncated metric
+    where the metric has a spectral gap at the truncation rank (without one,
+    F F^T is not unique)."""
     kl, ql = h["kv_label"], h["q_label"]
     np.testing.assert_allclose(h["k_centroid"], O.group_means(k, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
     np.testing.assert_allclose(h["v_centroid"], O.group_means(v, kl, h["Ck"]), rtol=1e-4, atol=1e-5)
@@ -271,6 +292,9 @@ def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, sema
     gap_ok = (r == cfg.d or (w[r - 1] - w[r]) > 1e-2 * w[0]) and not semantic_keys
     Fw = None if warm is None else O.warm_factor(MK, warm["F_K"], r, 1.0 / math.sqrt(cfg.d))
     compared = {"F_K": False, "F_Q": False}
+    if Fw is None and not semantic_keys:
+        check_factor_spectral(FK, MK, r, 1.0 / math.sqrt(cfg.d))
+        compared["F_K"] = True
     if Fw is not None:
         ref = Fw @ Fw.T
         assert np.abs(FK @ FK.T - ref).max() <= 2e-4 * np.abs(ref).max(), "warm F_K"
@@ -282,6 +306,9 @@ def check_partition_floats(h, cfg, q, k, v, warm=None, semantic_keys=False, sema
     refq = Uq[:, :rq] @ np.diag(wq[:rq]) @ Uq[:, :rq].T
     FQ = h["F_Q"]
     Fwq = None if warm is None else O.warm_factor(MQ, warm["F_Q"], rq, 1.0)
+    if Fwq is None and not semantic_queries:
+        check_factor_spectral(FQ, MQ, rq, 1.0)
+        compared["F_Q"] = True
     if Fwq is not None:
         refq = Fwq @ Fwq.T
         assert np.abs(FQ @ FQ.T - refq).max() <= 2e-4 * np.abs(refq).max(), "warm F_Q"
