@@ -532,19 +532,29 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
             if (lane == 0) {
                 constexpr uint32_t idesc_qk = idesc_f32acc(128, 128, kFmtBF16, false);
                 constexpr uint32_t idesc_pv = idesc_f32acc(128, D, kFmtF16, true);
+                // Descriptors are built once; every MMA adds a compile-time offset
+                // (its start address, >> 4, sits in the low bits and never carries
+                // out: shared addresses are below 2^18).  Rebuilding them per MMA
+                // costs more issue cycles than the 64 an M=128, N=128, K=16 MMA takes.
+                const uint64_t dq = smem_desc(sQ, 16, 1024), dk = smem_desc(sK, 16, 1024);
+                const uint64_t dv = smem_desc(sV, BN * 128, 1024);
                 auto issue_s = [&](int t, int stage) {
+                    const uint64_t a0 = dq + (uint64_t)((t * L::QB) >> 4), b0 = dk + (uint64_t)((stage * L::KB) >> 4);
+                    const uint32_t d = tmem + 128 * t;
+#pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t a = smem_desc(sQ + t * L::QB + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
-                        const uint64_t b = smem_desc(sK + stage * L::KB + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
-                        mma_f16_ss(tmem + 128 * t, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                        const uint64_t off = (uint64_t)((((kk / 4) * BM * 128) + (kk % 4) * 32) >> 4);
+                        const uint64_t offb = (uint64_t)((((kk / 4) * BN * 128) + (kk % 4) * 32) >> 4);
+                        mma_f16_ss(d, a0 + off, b0 + offb, idesc_qk, kk > 0 ? 1u : 0u);
                     }
                 };
                 auto issue_pv = [&](int t, int jj) {
-                    const int stage = jj % NS;
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint64_t b = smem_desc(sV + stage * L::KB + kk * 2048, BN * 128, 1024);
-                        mma_f16_ts(tmem + 256 + D * t, tmem + 128 * t + kk * 8, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    const uint64_t b0 = dv + (uint64_t)(((jj % NS) * L::KB) >> 4);
+                    const uint32_t d = tmem + 256 + D * t, a = tmem + 128 * t;
+                    const uint32_t acc0 = jj > 0 ? 1u : 0u;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_f16_ts(d, a + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
                 };
                 // Stall hook (testing the timeout path): a bounded wait on a
                 // barrier nothing signals runs out before any MMA is issued.
