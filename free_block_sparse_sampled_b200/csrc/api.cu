@@ -63,6 +63,7 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_hnK = bump(c, BH * Ck * 4);
     pl.o_cenQ = bump(c, BH * Cq * pl.RQp * 4);
     pl.o_hnQ = bump(c, BH * Cq * 4);
+    pl.o_hs = bump(c, BH * Cm * 8 * 4);
     pl.o_raw = bump(c, BH * N * 4);
     pl.o_hist = bump(c, BH * pl.n_sort_tiles * Cm * 4);
     pl.o_sorted = bump(c, BH * N * 4);

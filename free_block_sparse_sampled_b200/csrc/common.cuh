@@ -107,7 +107,7 @@ struct Plan {
     int64_t beta;        // key budget per query group
     int stop_changed;    // k-means stop threshold on changed labels
     // internal buffers (byte offsets into the workspace)
-    size_t o_status, o_ctl, o_mat, o_FK, o_FQ, o_rq, o_phiK, o_phiQ, o_cenK, o_hnK, o_cenQ, o_hnQ,
+    size_t o_status, o_ctl, o_mat, o_FK, o_FQ, o_rq, o_phiK, o_phiQ, o_cenK, o_hnK, o_cenQ, o_hnQ, o_hs,
         o_raw, o_hist, o_sorted, o_offs, o_newid, o_muK, o_t1, o_t2, o_mloc, o_pslot, o_palloc,
         o_poff, o_psum, o_qprobe, o_work, o_fstat, o_G, o_rhs, o_vh, o_vmax, o_vscale, o_qsplit, o_uw, o_lbar, o_vv,
         o_warm,   // [0]: kWarmMagic when the fused call's state is complete; [1 + bh], [1 + BH + bh]: cold K / Q factor

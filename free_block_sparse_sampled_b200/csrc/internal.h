@@ -57,8 +57,9 @@ bool route_uses_tc(const sparsepr_params& p);
 bool launch_route_tc(const Plan& pl, const sparsepr_partition_out& part, void* ws, float* t1, float* t2, float* ml,
                      cudaStream_t st);
 // Tensor-core k-means assignment; false if its tensor maps could not be built.
-bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, int BH, int N, int C, int R,
-                             int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
+// hs: scratch of BH * C * 8 floats for the split half-norms of the centres.
+bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, float* hs, int BH, int N, int C,
+                             int R, int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
                              int max_iter, DevStatus* status, cudaStream_t st);
 // 2-D tensor map over [rows, cols] row-major elements (4-byte fp32, or 2-byte
 // fp16 / bf16 chosen by is_float), boxes of box_cols x box_rows, 128-byte swizzle.

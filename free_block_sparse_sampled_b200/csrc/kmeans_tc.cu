@@ -4,11 +4,14 @@
 //
 // Coordinates and centres are stored TF32-rounded (round to nearest even),
 // so the tcgen05 kind::tf32 products are exact and the scores carry only fp32
-// accumulation error.  Centres stream through shared memory in blocks of up
-// to 256 (TMA, 128-byte swizzle, two stages); the scores of a block land in
-// TMEM (two buffers) and eight epilogue warps (two per TMEM lane quadrant,
-// each owning half of the columns) take the running argmax while the next
-// block multiplies.  All waits are bounded.
+// accumulation error.  The -|c|^2/2 term joins the product as one more K step:
+// a constant tile of ones (two columns) against each centre's -|c|^2/2 split
+// into TF32 hi and lo parts, so the tensor core returns the score itself.
+// Centres stream through shared memory in blocks of up to 256 (TMA, 128-byte
+// swizzle, two stages, with their split half-norms 32-byte swizzled); the
+// scores of a block land in TMEM (two buffers) and eight epilogue warps (two
+// per TMEM lane quadrant, each owning half of the columns) take the running
+// argmax while the next block multiplies.  All waits are bounded.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -23,23 +26,43 @@ constexpr uint32_t kSpin = 1u << 20;
 enum { B_AF = 0, B_AE = 2, B_BF = 4, B_BE = 6, B_DF = 8, B_DE = 10, B_DR = 12, N_BAR = 13 };
 constexpr int oA = 0;                                   // 2 buffers x 2 chunks x 128 rows x 128 B
 constexpr int oB = oA + 2 * 2 * BP * 128;               // 2 stages x 2 chunks x 256 rows x 128 B
-constexpr int oBar = oB + 2 * 2 * NBMAX * 128;
-constexpr int oRed = oBar + N_BAR * 8;                  // 128 x (score, index) of the upper half
-constexpr int oHn = oRed + BP * 8;                      // negated half-norms of the head's centres
-constexpr int oMisc = oHn + kMaxGroups * 4;
+constexpr int oOnes = oB + 2 * 2 * NBMAX * 128;        // 128 rows x 8 TF32: ones in columns 0 and 1
+constexpr int oH = oOnes + BP * 32;                     // 2 stages x NBMAX x 8 TF32: (hi, lo, 0 ...) of -|c|^2/2
+constexpr int oBar2 = oH + 2 * NBMAX * 32;
+constexpr int oRed = oBar2 + N_BAR * 8;                 // 128 x (score, index) of the upper half
+constexpr int oMisc = oRed + BP * 8;
 constexpr int kSmem = oMisc + 64 + 1024;
+static_assert(oOnes % 256 == 0 && oH % 256 == 0, "32-byte swizzled tiles need 256-byte alignment");
 
 struct Maps {
     CUtensorMap pts;       // [BH*N, R] fp32, box 32 x 128
     CUtensorMap cen;       // [BH*C, R] fp32, box 32 x NB
+    CUtensorMap hs;        // [BH*C, 8] fp32, box 8 x NB, 32-byte swizzle
 };
+
+// Byte offset of element (row, k) of a [rows x 8] fp32 tile in the 32-byte
+// swizzled K-major layout (16-byte unit index XOR bit 2 of the row).
+__device__ __forceinline__ uint32_t sw32(int row, int k) {
+    return (uint32_t)(row * 32 + ((((k >> 2) ^ (row >> 2)) & 1) << 4) + (k & 3) * 4);
+}
+
+// -|c|^2/2 of every centre as (hi, lo, 0, 0, 0, 0, 0, 0) with hi the TF32
+// rounding and lo the TF32 rounding of the remainder.
+__global__ void half_norm_split_kernel(const float* __restrict__ hn, size_t n, float* __restrict__ hs) {
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+        const float h = -hn[e], hi = tf32_round(h), lo = tf32_round(h - hi);
+        float4* o = reinterpret_cast<float4*>(hs + e * 8);
+        o[0] = make_float4(hi, lo, 0.f, 0.f);
+        o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
 }  // namespace kmtc
 
 // Persistent: block k handles items k, k + grid, ... where an item is 128
 // points of one head; heads whose k-means has stopped are skipped by every role.
 template <bool DBG>
 __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
-    const __grid_constant__ kmtc::Maps maps, const float* __restrict__ hn, int BH, int N, int C, int R, int NB,
+    const __grid_constant__ kmtc::Maps maps, int BH, int N, int C, int R, int NB,
     int nblk, int32_t* __restrict__ labels, int32_t* __restrict__ ctl, int first, float* __restrict__ dbg_scores,
     int32_t* __restrict__ dbg_hist, int max_iter, DevStatus* status) {
     using namespace kmtc;
@@ -51,7 +74,7 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
     const int n_items = BH * tiles_per_head;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_u32(sm);
-    auto bar = [&](int i) -> uint32_t { return s_base + oBar + 8 * i; };
+    auto bar = [&](int i) -> uint32_t { return s_base + oBar2 + 8 * i; };
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + oMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     const int nchunk = (R + 31) / 32;           // 32 fp32 per 128-byte row chunk
@@ -71,6 +94,14 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         fence_barrier_init();
         misc[1] = 0;
     }
+    {   // the ones tile of the half-norm K step: columns 0 and 1 of every row
+        float* ones = reinterpret_cast<float*>(sm + oOnes);
+        for (int e = tid; e < BP * 8; e += blockDim.x) {
+            const int row = e >> 3, k = e & 7;
+            ones[sw32(row, k) >> 2] = k < 2 ? 1.f : 0.f;
+        }
+        fence_proxy_async_smem();
+    }
     if (warp == 9) {
         tmem_alloc(smem_u32(misc), 512);
         tmem_relinquish();
@@ -84,6 +115,7 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         if (lane == 0) {   // TMA producer
             prefetch_tmap(&maps.pts);
             prefetch_tmap(&maps.cen);
+            prefetch_tmap(&maps.hs);
             int li = 0, gb = 0;           // local item count, global centre-block count
             bool ok = true;
             for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
@@ -96,10 +128,11 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                 for (int blk = 0; blk < nblk; ++blk, ++gb) {
                     const int stage = gb & 1;
                     if (gb >= 2 && !mbar_wait(bar(B_BE + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
-                    mbar_arrive_expect_tx(bar(B_BF + stage), nchunk * NB * 128);
+                    mbar_arrive_expect_tx(bar(B_BF + stage), nchunk * NB * 128 + NB * 32);
                     for (int ch = 0; ch < nchunk; ++ch)
                         tma_load_2d(s_base + oB + (stage * 2 + ch) * NBMAX * 128, &maps.cen, bar(B_BF + stage),
                                     ch * 32, bh * C + blk * NB);
+                    tma_load_2d(s_base + oH + stage * NBMAX * 32, &maps.hs, bar(B_BF + stage), 0, bh * C + blk * NB);
                 }
                 ++li;
             }
@@ -114,26 +147,31 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         if (lane == 0) {   // MMA issuer
             const uint32_t idesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NB >> 3) << 17) |
                                    ((uint32_t)(BP >> 4) << 24);   // F32 <- TF32 x TF32, K-major both
+            // descriptors built once; each MMA adds its offset (>> 4) to the
+            // start-address field, which never carries out (shared < 2^18)
+            const uint64_t dA = smem_desc(s_base + oA, 16, 1024), dB = smem_desc(s_base + oB, 16, 1024);
+            const uint64_t dOnes = smem_desc_sw32(s_base + oOnes), dH = smem_desc_sw32(s_base + oH);
             int li = 0, gb = 0;
             bool ok = true;
             for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
                 if (!item_live(w)) continue;
                 const int ab = li & 1;
                 if (!mbar_wait(bar(B_AF + ab), (li >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                const uint64_t a0 = dA + (uint64_t)((ab * 2 * BP * 128) >> 4);
                 for (int blk = 0; blk < nblk; ++blk, ++gb) {
                     const int stage = gb & 1;
                     if (!mbar_wait(bar(B_BF + stage), (gb >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
                     if (gb >= 2 && !mbar_wait(bar(B_DE + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
                     tc_fence_after();
+                    const uint64_t b0 = dB + (uint64_t)((stage * 2 * NBMAX * 128) >> 4);
+                    const uint32_t d = tmem + stage * NB;
                     for (int kk = 0; kk < ksteps; ++kk) {
-                        const uint64_t a = smem_desc(s_base + oA + (ab * 2 + kk / 4) * BP * 128 + (kk % 4) * 32, 16, 1024);
-                        const uint64_t b = smem_desc(s_base + oB + (stage * 2 + kk / 4) * NBMAX * 128 + (kk % 4) * 32, 16, 1024);
-                        asm volatile(
-                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                            "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem + stage * NB),
-                            "l"(a), "l"(b), "r"(idesc), "r"(kk > 0 ? 1u : 0u)
-                            : "memory");
+                        const uint64_t off = (uint64_t)(((kk >> 2) * BP * 128 + (kk & 3) * 32) >> 4);
+                        const uint64_t offb = (uint64_t)(((kk >> 2) * NBMAX * 128 + (kk & 3) * 32) >> 4);
+                        mma_tf32_ss(d, a0 + off, b0 + offb, idesc, kk > 0 ? 1u : 0u);
                     }
+                    // + 1 * hi + 1 * lo: the -|c|^2/2 term of every score
+                    mma_tf32_ss(d, dOnes, dH + (uint64_t)((stage * NBMAX * 32) >> 4), idesc, 1u);
                     mma_commit(bar(B_DF + stage));
                     mma_commit(bar(B_BE + stage));
                 }
@@ -154,8 +192,7 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         const int hw = NB / 2;
         float* red_s = reinterpret_cast<float*>(sm + oRed);
         int* red_i = reinterpret_cast<int*>(sm + oRed + BP * 4);
-        float* hns = reinterpret_cast<float*>(sm + oHn);
-        int gb = 0, staged_bh = -1;
+        int gb = 0;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
             if (!item_live(w)) continue;
@@ -164,12 +201,6 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
             int32_t* hc = ctl + bh * kCtlStride;
             // previous label, read now and used after the last centre block
             const int old_label = (valid && !first) ? labels[(size_t)bh * N + p] : 0;
-            if (bh != staged_bh) {   // a persistent block's items mostly share a head: stage its centres' -|c|^2/2 once
-                asm volatile("bar.sync 1, 256;" ::: "memory");   // the previous head's table is no longer read
-                for (int c = tid; c < nblk * NB; c += 256) hns[c] = (c < C) ? -hn[(size_t)bh * C + c] : -INFINITY;
-                asm volatile("bar.sync 1, 256;" ::: "memory");
-                staged_bh = bh;
-            }
             // running first maximum over this half's columns, in column order: the
             // best value, the base column of the chunk holding it and a copy of
             // that chunk's scores (predicated copies instead of a per-chunk index
@@ -182,7 +213,6 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
             for (int i = 0; i < 32; ++i) keep[i] = -INFINITY;
             for (int blk = 0; blk < nblk; ++blk, ++gb) {
                 const int db = gb & 1;
-                const float* hb = hns + blk * NB;   // columns past C hold -inf and never win
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + db), (gb >> 1) & 1, abort_flag, kSpin));
                 if (!ok) break;
                 tc_fence_after();
@@ -197,13 +227,12 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                     for (int q = 0; q < 2; ++q) {
                         if (q == 1 && !two) break;
                         const int cb = blk * NB + half * hw + c0 + 32 * q;
-                        const float2* hr = reinterpret_cast<const float2*>(hb + half * hw + c0 + 32 * q);
                         float sc[32];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float2 x = fadd2(make_float2(v[q][2 * i], v[q][2 * i + 1]), hr[i]);
-                            sc[2 * i] = x.x;
-                            sc[2 * i + 1] = x.y;
+                        for (int i = 0; i < 32; ++i) sc[i] = v[q][i];
+                        if (cb + 32 > C) {   // columns past C (another head's centres or zero fill) never win
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) sc[i] = (cb + i < C) ? sc[i] : -INFINITY;
                         }
                         if (DBG) {
 #pragma unroll
@@ -290,15 +319,16 @@ EncodeTiledFn encode_fn_km() {
     }
     return fn;
 }
-bool make_f32_map(CUtensorMap* m, const void* base, uint64_t rows, int R, int box_rows) {
+bool make_f32_map(CUtensorMap* m, const void* base, uint64_t rows, int R, int box_rows, int box_cols = 32,
+                  CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn_km();
     if (fn == nullptr) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)R, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)R * 4};
-    const cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     const cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 }  // namespace
@@ -309,8 +339,8 @@ void kmeans_centre_blocks(int C, int& NB, int& nblk) {
     if (NB > kmtc::NBMAX) NB = kmtc::NBMAX;
 }
 
-bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, int BH, int N, int C, int R,
-                             int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
+bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, float* hs, int BH, int N, int C,
+                             int R, int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
                              int max_iter, DevStatus* status, cudaStream_t st) {
     if (R > kMaxRank) return false;              // shared-memory tiles hold rows of up to 64 floats
     int NB, nblk;
@@ -318,16 +348,22 @@ bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn
     kmtc::Maps maps;
     if (!make_f32_map(&maps.pts, phi, (uint64_t)BH * N, R, kmtc::BP)) return false;
     if (!make_f32_map(&maps.cen, cen, (uint64_t)BH * C, R, NB)) return false;
+    if (!make_f32_map(&maps.hs, hs, (uint64_t)BH * C, 8, NB, 8, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
+    {
+        const size_t n = (size_t)BH * C;
+        const int g = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+        count_launch(), kmtc::half_norm_split_kernel<<<g, 256, 0, st>>>(hn, n, hs);
+    }
     const int items = BH * ((N + kmtc::BP - 1) / kmtc::BP);
     const int grid = items < sm_count() ? items : sm_count();
     if (dbg_scores != nullptr) {
         cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
         count_launch(), kmeans_assign_tc_kernel<true><<<grid, 320, kmtc::kSmem, st>>>(
-            maps, hn, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
+            maps, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
     } else {
         cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
         count_launch(), kmeans_assign_tc_kernel<false><<<grid, 320, kmtc::kSmem, st>>>(
-            maps, hn, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
+            maps, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
     }
     return true;
 }

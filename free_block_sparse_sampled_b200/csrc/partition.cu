@@ -779,7 +779,7 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
                                                                               sorted, ctl);
             count_launch(), centre_update_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, sorted, offs, N, C, cen, hn, ctl);
         }
-        if (!launch_kmeans_assign_tc(phi, cen, hn, BH, N, C, R, raw, ctl, first, dbg_scores, dbg_hist,
+        if (!launch_kmeans_assign_tc(phi, cen, hn, at<float>(ws, pl.o_hs), BH, N, C, R, raw, ctl, first, dbg_scores, dbg_hist,
                                      p.kmeans_iters, at<DevStatus>(ws, pl.o_status), st))
             count_launch(), kmeans_assign_kernel<R><<<agrid, 128, 0, st>>>(phi, cen, hn, N, C, raw, ctl, first,
                                                                           dbg_scores, dbg_hist, p.kmeans_iters);

@@ -171,6 +171,18 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
     return desc;
 }
 
+// The same for a K-major tile of 32-byte rows (8 TF32) in the 32-byte swizzle
+// (swizzle mode 6): 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t addr) {
+    uint64_t desc = 0;
+    desc |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    desc |= (uint64_t)1 << 16;                     // leading byte offset 16 (unused: one swizzle atom along K)
+    desc |= (uint64_t)(256 >> 4) << 32;            // stride byte offset: 8 rows x 32 bytes
+    desc |= (uint64_t)1 << 46;
+    desc |= (uint64_t)6 << 61;                     // 32-byte swizzle
+    return desc;
+}
+
 // Instruction descriptor for kind::f16 with FP32 accumulation; A and B share
 // one format: 0 = F16, 1 = BF16 (kind::f16), 2 = TF32 (kind::tf32).
 constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1, kFmtTF32 = 2;
