@@ -255,6 +255,298 @@ __global__ void __maxnreg__(168) apply_tc_kernel(
     }
 }
 
+// ---------------------------------------------------------------- transposed form (d = 128)
+// The same output computed as D^T = B'^T Xbar^T with B' = B + diag(sigma), so
+//   O_out[perm_q[p]] = (mu_X + mu_R) + (Xbar B')_p
+// (Xbar sigma + mu_X gives back O^sp).  B'^T, split into TF32 hi and lo, sits
+// in TMEM as the MMA's A operand (lanes = output channels); each 128-row tile
+// of O^sp streams in once through a TMA ring of 32-channel chunks, which the
+// transform warps standardise and split in place (hi) and beside it (lo); the
+// accumulator holds one output channel per lane and one tile row per column,
+// so every warp of the epilogue writes a row's 32 channels as one coalesced
+// 128-byte store.
+//   warp 0: TMA producer; warp 1: MMA issuer; warps 2-5: transform (one tile
+//   row each); warps 6-13: epilogue (channels = TMEM lane quadrant, rows =
+//   half of the tile) and the per-head staging of B'^T.
+// TMEM: B'^T hi [0,128), lo [128,256); accumulators [256,384), [384,512).
+namespace aptt {
+constexpr int D = 128, BM = 128, NCH = 4, NST = 4;
+constexpr int kThreads = 448;
+constexpr uint32_t kSpin = 1u << 20;
+enum { B_RF = 0, B_XF = NST, B_XE = 2 * NST, B_DF = 3 * NST, B_DE = 3 * NST + 2, B_AF = 3 * NST + 4,
+       B_AE = 3 * NST + 5, B_DR = 3 * NST + 6, B_SS = 3 * NST + 7, N_BAR = 3 * NST + 9 };
+constexpr int CHB = BM * 128;                 // one chunk: 128 rows x 32 fp32
+constexpr int oHi = 0;                        // NST chunks: raw O^sp, then Xbar hi in place
+constexpr int oLo = oHi + NST * CHB;          // NST chunks: Xbar lo
+constexpr int oStat = oLo + NST * CHB;        // 2 x (mu_X, 1 / sigma) of the last two heads (transform warps)
+constexpr int oBar = oStat + 2 * 2 * D * 4;
+constexpr int oMisc = oBar + N_BAR * 8;
+constexpr int kSmem = oMisc + 16 + 1024;
+static_assert(oLo % 1024 == 0 && oStat % 16 == 0, "alignment");
+}  // namespace aptt
+
+__global__ void __maxnreg__(144) apply_t_kernel(
+    const __grid_constant__ CUtensorMap osp_map, const float* __restrict__ Bm, const float* __restrict__ mu_x,
+    const float* __restrict__ sigma, const float* __restrict__ mu_r, const int32_t* __restrict__ pslot,
+    const float* __restrict__ probe_dense, const int32_t* __restrict__ perm_q, int BH, int N, int Mp,
+    float* __restrict__ O_out, DevStatus* status) {
+    using namespace aptt;
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    if (*reinterpret_cast<volatile const int32_t*>(&status->code) != 0) return;
+    const int tiles_per_head = (N + BM - 1) / BM;
+    const long long total = (long long)BH * tiles_per_head;
+    const int w_begin = (int)(total * blockIdx.x / gridDim.x), w_end = (int)(total * (blockIdx.x + 1) / gridDim.x);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t s_base = smem_u32(sm);
+    auto bar = [&](int i) -> uint32_t { return s_base + oBar + 8 * i; };
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + oMisc);   // [0] tmem, [1] abort
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bar(B_RF + s), 1);
+            mbar_init(bar(B_XF + s), 128);
+            mbar_init(bar(B_XE + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_DF + s), 1);
+            mbar_init(bar(B_DE + s), 256);
+        }
+        mbar_init(bar(B_AF), 256);
+        mbar_init(bar(B_AE), 1);
+        mbar_init(bar(B_DR), 1);
+        mbar_init(bar(B_SS), 128);
+        mbar_init(bar(B_SS + 1), 128);
+        fence_barrier_init();
+        misc[1] = 0;
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(misc), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer: raw O^sp chunks
+            prefetch_tmap(&osp_map);
+            bool ok = true;
+            int g = 0;
+            for (int w = w_begin; ok && w < w_end; ++w) {
+                const int bh = w / tiles_per_head, p0 = (w % tiles_per_head) * BM;
+                for (int c = 0; c < NCH; ++c, ++g) {
+                    const int s = g % NST;
+                    if (g >= NST && !mbar_wait(bar(B_XE + s), ((g / NST) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar(B_RF + s), CHB);
+                    tma_load_2d(s_base + oHi + s * CHB, &osp_map, bar(B_RF + s), 32 * c, bh * N + p0);
+                }
+            }
+            if (!ok) {
+                record_status(status, SPARSEPR_TIMEOUT, 73);
+                *abort_flag = 1;
+            }
+            // every copy issued above lands before the CTA can exit
+            for (int t = max(0, g - NST); t < g; ++t) mbar_wait(bar(B_RF + t % NST), (t / NST) & 1, nullptr, kSpin);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_f32acc(128, BM, kFmtTF32, false);
+            const uint64_t dHi = smem_desc(s_base + oHi, 16, 1024), dLo = smem_desc(s_base + oLo, 16, 1024);
+            bool ok = true;
+            int g = 0, heads = 0, cur_bh = -1, i = 0;
+            for (int w = w_begin; ok && w < w_end; ++w, ++i) {
+                const int bh = w / tiles_per_head;
+                if (bh != cur_bh) {
+                    if (!mbar_wait(bar(B_AF), heads & 1, abort_flag, kSpin)) { ok = false; break; }
+                    cur_bh = bh;
+                    ++heads;
+                }
+                const int d = i & 1;
+                if (i >= 2 && !mbar_wait(bar(B_DE + d), ((i >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                const uint32_t acc = tmem + 256 + BM * d;
+                for (int c = 0; c < NCH; ++c, ++g) {
+                    const int s = g % NST;
+                    if (!mbar_wait(bar(B_XF + s), (g / NST) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t bh_d = dHi + (uint64_t)((s * CHB) >> 4), bl_d = dLo + (uint64_t)((s * CHB) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {   // K = 8 per instruction, 32-byte steps inside the 128-byte rows
+                        const uint32_t ahi = tmem + 32 * c + 8 * kk, alo = tmem + 128 + 32 * c + 8 * kk;
+                        const uint64_t bo = (uint64_t)((kk * 32) >> 4);
+                        mma_tf32_ts(acc, ahi, bh_d + bo, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                        mma_tf32_ts(acc, ahi, bl_d + bo, idesc, 1u);
+                        mma_tf32_ts(acc, alo, bh_d + bo, idesc, 1u);
+                    }
+                    mma_commit(bar(B_XE + s));
+                }
+                if (!ok) break;
+                mma_commit(bar(B_DF + d));
+                // the last tile of a head releases B'^T for the next head's staging
+                if (w + 1 == w_end || (w + 1) / tiles_per_head != bh) mma_commit(bar(B_AE));
+            }
+            if (!ok) {
+                record_status(status, SPARSEPR_TIMEOUT, 74);
+                *abort_flag = 1;
+            }
+            mma_commit(bar(B_DR));
+            mbar_wait(bar(B_DR), 0, nullptr, kSpin);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ transform: Xbar = (O^sp - mu_X) / sigma, hi and lo
+        const int t = tid - 64;   // tile row
+        float* stat = nullptr;
+        bool ok = true;
+        int g = 0, cur_bh = -1, heads = 0;
+        for (int w = w_begin; ok && w < w_end; ++w) {
+            const int bh = w / tiles_per_head, p0 = (w % tiles_per_head) * BM;
+            if (bh != cur_bh) {
+                // the head's mu_X and 1 / sigma, in the buffer of its parity: the
+                // other buffer may still be read by a thread on the previous head;
+                // this one was last read for head - 2, which every thread left
+                // before it passed the previous head's exchange
+                const int hp = heads & 1;
+                stat = reinterpret_cast<float*>(sm + oStat) + hp * 2 * D;
+                stat[t] = mu_x[(size_t)bh * D + t];
+                stat[D + t] = 1.f / sigma[(size_t)bh * D + t];
+                mbar_arrive(bar(B_SS + hp));
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SS + hp), (heads >> 1) & 1, abort_flag, kSpin));
+                if (!ok) break;
+                cur_bh = bh;
+                ++heads;
+            }
+            const bool live = p0 + t < N;
+            for (int c = 0; c < NCH; ++c, ++g) {
+                const int s = g % NST;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_RF + s), (g / NST) & 1, abort_flag, kSpin));
+                if (!ok) break;
+                uint8_t* hi = sm + oHi + s * CHB + t * 128;
+                uint8_t* lo = sm + oLo + s * CHB + t * 128;
+                const float4* m4 = reinterpret_cast<const float4*>(stat) + 8 * c;
+                const float4* i4 = reinterpret_cast<const float4*>(stat + D) + 8 * c;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {   // 16-byte unit u of the row sits at (u ^ row % 8) (128-byte swizzle)
+                    const int pu = (u ^ t) & 7;
+                    float4 x = *reinterpret_cast<const float4*>(hi + pu * 16);
+                    const float4 m = m4[u], iv = i4[u];
+                    x.x = live ? (x.x - m.x) * iv.x : 0.f;
+                    x.y = live ? (x.y - m.y) * iv.y : 0.f;
+                    x.z = live ? (x.z - m.z) * iv.z : 0.f;
+                    x.w = live ? (x.w - m.w) * iv.w : 0.f;
+                    const float4 h = make_float4(tf32_round(x.x), tf32_round(x.y), tf32_round(x.z), tf32_round(x.w));
+                    *reinterpret_cast<float4*>(hi + pu * 16) = h;
+                    *reinterpret_cast<float4*>(lo + pu * 16) =
+                        make_float4(tf32_round(x.x - h.x), tf32_round(x.y - h.y), tf32_round(x.z - h.z),
+                                    tf32_round(x.w - h.w));
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(bar(B_XF + s));
+            }
+        }
+        if (!ok) {
+            record_status(status, SPARSEPR_TIMEOUT, 75);
+            *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------ epilogue (and B'^T staging)
+        const int q = warp & 3, hrow = (warp - 6) >> 2;   // lane quadrant = output channels, half of the tile rows
+        const int n = q * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+        bool ok = true;
+        int heads = 0, cur_bh = -1, i = 0;
+        float bias = 0.f;
+        for (int w = w_begin; ok && w < w_end; ++w, ++i) {
+            const int bh = w / tiles_per_head, p0 = (w % tiles_per_head) * BM;
+            if (bh != cur_bh) {
+                // B'^T of this head into TMEM, once the previous head's MMAs are done:
+                // lane n, column k holds B[k][n] (+ sigma[n] on the diagonal), hi and lo
+                if (heads > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar(B_AE), (heads - 1) & 1, abort_flag, kSpin));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const float* Bh = Bm + (size_t)bh * D * D;
+                const float sg = sigma[(size_t)bh * D + n];
+                for (int c2 = 0; c2 < 4; ++c2) {   // 32 columns at a time: hi (c2 even), then lo
+                    const int k0 = 64 * hrow + 32 * (c2 >> 1);
+                    float vb[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int k = k0 + e;
+                        const float b = Bh[(size_t)k * D + n] + (k == n ? sg : 0.f);
+                        const float h = tf32_round(b);
+                        vb[e] = (c2 & 1) ? tf32_round(b - h) : h;
+                    }
+                    tmem_st32(t_lane + 128 * (c2 & 1) + k0, vb);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(bar(B_AF));
+                bias = mu_x[(size_t)bh * D + n] + mu_r[(size_t)bh * D + n];
+                cur_bh = bh;
+                ++heads;
+            }
+            const int d = i & 1;
+            // the row indices of this half of the tile: lane l holds rows 64 hrow + l and + 32
+            const int r0 = p0 + 64 * hrow + lane, r1 = r0 + 32;
+            const size_t hb = (size_t)bh * N;
+            const int sl0 = r0 < N ? pslot[hb + r0] : -2, sl1 = r1 < N ? pslot[hb + r1] : -2;
+            const int dq0 = r0 < N ? perm_q[hb + r0] : 0, dq1 = r1 < N ? perm_q[hb + r1] : 0;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + d), (i >> 1) & 1, abort_flag, kSpin));
+            if (!ok) break;
+            tc_fence_after();
+            float v[2][32];
+            tmem_ld32(t_lane + 256 + BM * d + 64 * hrow, v[0]);
+            tmem_ld32(t_lane + 256 + BM * d + 64 * hrow + 32, v[1]);
+            tmem_wait_ld(v[0]);
+            tmem_wait_ld(v[1]);
+            tc_fence_before();
+            mbar_arrive(bar(B_DE + d));   // the accumulator is free for tile i + 2
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int sl = h ? sl1 : sl0, dq = h ? dq1 : dq0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int slot = __shfl_sync(0xffffffffu, sl, j);   // uniform: the warp writes one row
+                    const int dst = __shfl_sync(0xffffffffu, dq, j);
+                    if (slot == -2) continue;                            // past the head's last row
+                    float* orow = O_out + (hb + dst) * D;
+                    orow[n] = slot < 0 ? v[h][j] + bias : probe_dense[((size_t)bh * Mp + slot) * D + n];
+                }
+            }
+        }
+        if (!ok) {
+            record_status(status, SPARSEPR_TIMEOUT, 76);
+            *abort_flag = 1;
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// O_out[perm_q[p]] = O^sp[p]: the output of a call without probes (one warp per row).
+__global__ void unpermute_rows_kernel(const float* __restrict__ O_sp, const int32_t* __restrict__ perm_q, int BH,
+                                      int N, int d, float* __restrict__ O_out) {
+    const size_t rows = (size_t)BH * N;
+    const int lane = threadIdx.x & 31, n4 = d / 4;
+    for (size_t r = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5; r < rows;
+         r += ((size_t)gridDim.x * blockDim.x) >> 5) {
+        const size_t bh = r / N;
+        const float4* src = reinterpret_cast<const float4*>(O_sp + r * d);
+        float4* dst = reinterpret_cast<float4*>(O_out + (bh * N + perm_q[r]) * d);
+        for (int c = lane; c < n4; c += 32) dst[c] = src[c];
+    }
+}
+
 bool launch_apply_tc(const Plan& pl, const sparsepr_partition_out& part, const float* O_sp, const float* probe_dense,
                      const sparsepr_fit_out& f, const int32_t* pslot, float* O_out, DevStatus* status,
                      cudaStream_t st) {
@@ -263,6 +555,21 @@ bool launch_apply_tc(const Plan& pl, const sparsepr_partition_out& part, const f
     const long long tiles = (long long)pl.BH * ((pl.N + aptc::BM - 1) / aptc::BM);
     const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
     if (grid == 0) return true;
+    if (pl.Mp == 0) {   // no probes, no correction: the sparse output restored to the original order, bit for bit
+        const size_t rows = (size_t)pl.BH * pl.N;
+        const int g = (int)((rows * 32 + 255) / 256 < (size_t)sm_count() * 16 ? (rows * 32 + 255) / 256
+                                                                                 : (size_t)sm_count() * 16);
+        count_launch(), unpermute_rows_kernel<<<g, 256, 0, st>>>(O_sp, part.perm_q, pl.BH, pl.N, d, O_out);
+        return true;
+    }
+    if (d == 128) {
+        CUtensorMap m;
+        if (!encode_rows_map(&m, O_sp, (uint64_t)pl.BH * pl.N, 128, 4, true, 32, aptt::BM)) return false;
+        cudaFuncSetAttribute(apply_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, aptt::kSmem);
+        count_launch(), apply_t_kernel<<<grid, aptt::kThreads, aptt::kSmem, st>>>(
+            m, f.B, f.mu_x, f.sigma, f.mu_r, pslot, probe_dense, part.perm_q, pl.BH, pl.N, pl.Mp, O_out, status);
+        return true;
+    }
     if (d == 128) {
         auto k = apply_tc_kernel<128>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, aptc::Layout<128>::smem);
