@@ -140,7 +140,8 @@ def partition(cfg: SparsePRConfig, q, k, v, ws: torch.Tensor, debug: bool = Fals
     i32 = dict(dtype=torch.int32, device=dev)
     f32 = dict(dtype=torch.float32, device=dev)
     o = {
-        "Qp": torch.empty_like(q), "Kp": torch.empty_like(q), "Vp": torch.empty_like(q),
+        # permuted K/V: one per K/V head (the G query heads of a K/V head share its groups)
+        "Qp": torch.empty_like(q), "Kp": torch.empty_like(k), "Vp": torch.empty_like(v),
         "q_label": torch.empty(BH, N, **i32), "kv_label": torch.empty(BH, N, **i32),
         "perm_q": torch.empty(BH, N, **i32), "perm_kv": torch.empty(BH, N, **i32),
         "pos_q": torch.empty(BH, N, **i32), "q_offsets": torch.empty(BH, Cq + 1, **i32),

@@ -82,7 +82,8 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_fstat = bump(c, BH * 3 * d * 8);
     pl.o_G = bump(c, BH * d * d * 8);
     pl.o_rhs = bump(c, BH * d * d * 8);
-    pl.o_vh = bump(c, p.dtype == SPARSEPR_BF16 ? BH * N * d * 2 : 256);
+    const size_t BHk = BH / pl.G;   // K/V heads: the permuted K/V and their fp16 copy are per K/V head
+    pl.o_vh = bump(c, p.dtype == SPARSEPR_BF16 ? BHk * N * d * 2 : 256);
     pl.o_vmax = bump(c, BH * 4);
     pl.o_vscale = bump(c, BH * 4);
     pl.o_qsplit = bump(c, BH * 3 * (size_t)round_up(p.Cq, 128) * d * 2);
@@ -95,8 +96,8 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_rawkv = bump(c, pl.G > 1 ? BH / pl.G * N * 4 : 256);
     // outputs owned by the workspace (fused call)
     pl.o_Qp = bump(c, BH * N * d * es);
-    pl.o_Kp = bump(c, BH * N * d * es);
-    pl.o_Vp = bump(c, BH * N * d * es);
+    pl.o_Kp = bump(c, BHk * N * d * es);
+    pl.o_Vp = bump(c, BHk * N * d * es);
     pl.o_qlab = bump(c, BH * N * 4);
     pl.o_kvlab = bump(c, BH * N * 4);
     pl.o_permq = bump(c, BH * N * 4);

@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(256) attention_simt_kernel(
     int n_probe_items, int BM, int N, int Mp, int Cq, int Ck, const int32_t* __restrict__ kv_off,
     const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_groups,
     float* __restrict__ O_sp, float* __restrict__ probe_dense, unsigned long long* __restrict__ visited,
-    float scale_log2) {
+    float scale_log2, int G) {
     constexpr int H = D / 2, KC = 32;
     __shared__ float ks[KC][D];
     __shared__ float vs[KC][D];
@@ -189,8 +189,9 @@ __global__ void __launch_bounds__(256) attention_simt_kernel(
             for (int x = threadIdx.x; x < KC * D; x += blockDim.x) {
                 const int j = x / D, t = x % D;
                 const bool ok = j < n;
-                ks[j][t] = ok ? ldf(Kp + ((size_t)it.bh * N + c0 + j) * D + t) : 0.f;
-                vs[j][t] = ok ? ldf(Vp + ((size_t)it.bh * N + c0 + j) * D + t) : 0.f;
+                const size_t kr = (size_t)(it.bh / G) * N + c0 + j;   // the K/V head under GQA
+                ks[j][t] = ok ? ldf(Kp + kr * D + t) : 0.f;
+                vs[j][t] = ok ? ldf(Vp + kr * D + t) : 0.f;
             }
             __syncthreads();
             float sc[KC];
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
     int n_probe_items, int N, int Mp, int Cq, int Ck, int total_rows, const int32_t* __restrict__ kv_off,
     const int32_t* __restrict__ sel_count, const int32_t* __restrict__ sel_groups, const float* __restrict__ vscale,
     float* __restrict__ O_sp, float* __restrict__ probe_dense, DevStatus* status,
-    unsigned long long* __restrict__ visited, float scale_log2, uint32_t stall_polls) {
+    unsigned long long* __restrict__ visited, float scale_log2, uint32_t stall_polls, int G) {
     using namespace tc;
     using namespace sm100;
     using L = Layout<D>;
@@ -425,6 +426,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
                         tma_load_2d(sQ + t * L::QB + hh * BM * 128, tq, bar(B_Q), hh * 64, qrow + t * BM);
             }
             const bool probe = it.a < 0;
+            const int kv_head = it.bh / G;   // permuted K/V rows of the K/V head (GQA)
             const int32_t* sg = sel_groups + ((size_t)it.bh * Cq + (probe ? 0 : it.a)) * Ck;
             const int32_t* ko = kv_off + (size_t)it.bh * (Ck + 1);
             const int n_groups = probe ? 1 : sel_count[(size_t)it.bh * Cq + it.a];
@@ -493,7 +495,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
                     const int lo = max(my_sb, T0), hi = min(my_se, T0 + 16);
                     if (lo < hi) {
                         const int o = lo - my_sb;
-                        runs[lo - T0] = make_int2(it.bh * N + my_rs + 8 * o, hi - lo);
+                        runs[lo - T0] = make_int2(kv_head * N + my_rs + 8 * o, hi - lo);
                         for (int t = lo; t < hi; ++t) vm[t - T0] = (uint8_t)min(8, my_len - 8 * (t - my_sb));
                     }
                     if (w_end >= T0 + 16 || gbase + 32 >= n_groups) break;
@@ -706,7 +708,7 @@ __global__ void __launch_bounds__(384, 1) attention_tc_kernel(
                     const int row = it.row0 + BM * t + r;
                     float* out = (it.a < 0) ? probe_dense + ((size_t)it.bh * Mp + row) * D
                                             : O_sp + ((size_t)it.bh * N + row) * D;
-                    const float inv = vscale[it.bh] / (l2.x + l2.y);
+                    const float inv = vscale[it.bh / G] / (l2.x + l2.y);
     #pragma unroll
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         float v[32];
@@ -877,17 +879,18 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
         unsigned* vmax = at<unsigned>(ws, pl.o_vmax);
         float* vscale = at<float>(ws, pl.o_vscale);
         const size_t per_head = (size_t)N * d;
-        cudaMemsetAsync(vmax, 0, (size_t)BH * sizeof(unsigned), st);
-        const dim3 vgrid((unsigned)std::min<size_t>((per_head / 8 + 255) / 256, 148), BH);
+        const int BHk = BH / pl.G;   // V is per K/V head
+        cudaMemsetAsync(vmax, 0, (size_t)BHk * sizeof(unsigned), st);
+        const dim3 vgrid((unsigned)std::min<size_t>((per_head / 8 + 255) / 256, 148), BHk);
         count_launch(), vmax_kernel<<<vgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(part.Vp), per_head, vmax);
         count_launch(), vconvert_kernel<<<vgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(part.Vp), per_head,
                                                               vmax, VH, vscale);
         tc::Maps maps;
-        const uint64_t rows = (uint64_t)BH * N;
+        const uint64_t rows = (uint64_t)BH * N, kv_rows = (uint64_t)BHk * N;
         bool ok = true;
         for (int k = 0; k < tc::NBOX; ++k) {
-            ok = ok && make_rows_map(&maps.k[k], part.Kp, rows, d, 8 << k, false);
-            ok = ok && make_rows_map(&maps.v[k], VH, rows, d, 8 << k, true);
+            ok = ok && make_rows_map(&maps.k[k], part.Kp, kv_rows, d, 8 << k, false);
+            ok = ok && make_rows_map(&maps.v[k], VH, kv_rows, d, 8 << k, true);
         }
         ok = ok && make_rows_map(&maps.q, part.Qp, rows, d, 128, false);
         if (Mp > 0) ok = ok && make_rows_map(&maps.qp, qprobe, (uint64_t)BH * Mp, d, 128, false);
@@ -898,18 +901,18 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
             auto k = attention_tc_kernel<128>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<128>::smem);
             count_launch(), k<<<grid2, tc::kThreads, tc::Layout<128>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
-                                                                       pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
+                                                                       pl.Cq, pl.Ck, (int)kv_rows, part.kv_offsets,
                                                                        r.sel_count, r.sel_groups, vscale, O_sp,
                                                                        probe_dense, status, visited, scale_log2,
-                                                                       g_stall_polls.load());
+                                                                       g_stall_polls.load(), pl.G);
         } else {
             auto k = attention_tc_kernel<64>;
             cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Layout<64>::smem);
             count_launch(), k<<<grid2, tc::kThreads, tc::Layout<64>::smem, st>>>(maps, items, counter, n_probe2, N, Mp,
-                                                                      pl.Cq, pl.Ck, (int)rows, part.kv_offsets,
+                                                                      pl.Cq, pl.Ck, (int)kv_rows, part.kv_offsets,
                                                                       r.sel_count, r.sel_groups, vscale, O_sp,
                                                                       probe_dense, status, visited, scale_log2,
-                                                                      g_stall_polls.load());
+                                                                      g_stall_polls.load(), pl.G);
         }
     } else {
         const int threads = 2 * pl.BM;
@@ -917,7 +920,7 @@ sparsepr_status run_attention(const sparsepr_params& p, const Plan& pl, const sp
     count_launch(), attention_simt_kernel<T, D><<<grid, threads, 0, st>>>(                                                    \
         static_cast<const T*>(part.Qp), static_cast<const T*>(part.Kp), static_cast<const T*>(part.Vp),     \
         static_cast<const T*>(qprobe), items, counter, pl.n_probe_items, pl.BM, N, Mp, pl.Cq, pl.Ck,        \
-        part.kv_offsets, r.sel_count, r.sel_groups, O_sp, probe_dense, visited, scale_log2)
+        part.kv_offsets, r.sel_count, r.sel_groups, O_sp, probe_dense, visited, scale_log2, pl.G)
         if (p.dtype == SPARSEPR_BF16) {
             if (d == 128) SPR_SIMT(__nv_bfloat16, 128); else SPR_SIMT(__nv_bfloat16, 64);
         } else {

@@ -610,29 +610,32 @@ __global__ void relabel_kernel(const int32_t* __restrict__ raw, const int32_t* _
     }
 }
 
-// Xp[r] = X[perm[r]] in 16-byte chunks (group-major gather, paper §4.3).
+// Xp[h, r] = X[h, perm[h * perm_mul, r]] in 16-byte chunks (group-major
+// gather, paper §4.3).  perm_mul = G gathers each K/V head once, in the order
+// of its first query head (all G share the K/V groups under GQA).
 __global__ void gather_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ perm,
-                                   int BH, int N, int chunks, int G, uint4* __restrict__ Xp) {
+                                   int BH, int N, int chunks, int perm_mul, uint4* __restrict__ Xp) {
     const size_t total = (size_t)BH * N * chunks;
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
          e += (size_t)gridDim.x * blockDim.x) {
         const size_t row = e / chunks;
         const int ch = (int)(e - row * chunks);
-        const size_t bh = row / N;
-        const size_t src = (bh / G) * N + perm[row];   // source head: K/V head bh / G under GQA
+        const size_t bh = row / N, r = row - bh * N;
+        const size_t src = bh * N + perm[(bh * perm_mul) * N + r];
         Xp[e] = X[src * chunks + ch];
     }
 }
 
 // Mean of the rows of each group in group-major storage (fixed row order).
+// The rows of head bh live at head bh / src_div of Xp (the K/V head under GQA).
 template <typename T>
 __global__ void group_mean_kernel(const T* __restrict__ Xp, const int32_t* __restrict__ offs,
-                                  const int32_t* __restrict__ ng, int which, int N, int C, int d,
+                                  const int32_t* __restrict__ ng, int which, int N, int C, int d, int src_div,
                                   float* __restrict__ out) {
     const int bh = blockIdx.y, g = blockIdx.x, j = threadIdx.x;
     if (g >= ng[bh * 2 + which]) return;
     const int s = offs[(size_t)bh * (C + 1) + g], e = offs[(size_t)bh * (C + 1) + g + 1];
-    const T* base = Xp + (size_t)bh * N * d + j;
+    const T* base = Xp + (size_t)(bh / src_div) * N * d + j;
     float acc = 0.f;
     for (int r = s; r < e; ++r) acc += ldf(base + (size_t)r * d);
     out[((size_t)bh * C + g) * d + j] = acc / (float)(e - s);
@@ -835,11 +838,12 @@ void finalize_groups(const Plan& pl, void* ws, int C, int which, int32_t* label_
                                                                   label_out, perm_out, pos_out);
 }
 
-void gather(const void* X, const int32_t* perm, const Plan& pl, void* Xp, int G, cudaStream_t st) {
+// heads: output heads; perm_mul: output head h takes the permutation of head h * perm_mul.
+void gather(const void* X, const int32_t* perm, const Plan& pl, int heads, int perm_mul, void* Xp, cudaStream_t st) {
     const int chunks = pl.d * pl.esz / 16;
-    const size_t total = (size_t)pl.BH * pl.N * chunks;
+    const size_t total = (size_t)heads * pl.N * chunks;
     count_launch(), gather_rows_kernel<<<grid_for(total, 256), 256, 0, st>>>(
-        static_cast<const uint4*>(X), perm, pl.BH, pl.N, chunks, G, static_cast<uint4*>(Xp));
+        static_cast<const uint4*>(X), perm, heads, pl.N, chunks, perm_mul, static_cast<uint4*>(Xp));
 }
 
 template <typename T>
@@ -921,13 +925,14 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
         cudaMemcpyAsync(out.kv_centres, cenK, (size_t)BH * pl.Ck * pl.RKp * 4, cudaMemcpyDeviceToDevice, st);
     }
     finalize_groups(pl, ws, pl.Ck, 1, out.kv_label, out.perm_kv, nullptr, out.kv_offsets, out.n_groups, st);
-    gather(K, out.perm_kv, pl, out.Kp, G, st);
-    gather(V, out.perm_kv, pl, out.Vp, G, st);
+    // one permuted K/V per K/V head, in the group order its query heads share (GQA)
+    gather(K, out.perm_kv, pl, BHk, G, out.Kp, st);
+    gather(V, out.perm_kv, pl, BHk, G, out.Vp, st);
     // 4. centroids, query metric, factor, coordinates (§4.1, B.2)
     count_launch(), group_mean_kernel<T><<<dim3(pl.Ck, BH), d, 0, st>>>(static_cast<const T*>(out.Kp), out.kv_offsets,
-                                                        out.n_groups, 1, N, pl.Ck, d, out.k_centroid);
+                                                        out.n_groups, 1, N, pl.Ck, d, G, out.k_centroid);
     count_launch(), group_mean_kernel<T><<<dim3(pl.Ck, BH), d, 0, st>>>(static_cast<const T*>(out.Vp), out.kv_offsets,
-                                                        out.n_groups, 1, N, pl.Ck, d, out.v_centroid);
+                                                        out.n_groups, 1, N, pl.Ck, d, G, out.v_centroid);
     if (sem_q) {
         // semantic query groups: k-means on the raw query rows (RQp = d)
         count_launch(), identity_factor_kernel<<<BH, 256, 0, st>>>(FQ, d, pl.RQp, rq);
@@ -949,9 +954,9 @@ sparsepr_status partition_typed(const sparsepr_params& p, const Plan& pl, const 
     count_launch(), kmeans_reset_kernel<<<(BH + 127) / 128, 128, 0, st>>>(ctl, BH, kCtlItersQ);
     if (out.q_centres) cudaMemcpyAsync(out.q_centres, cenQ, (size_t)BH * pl.Cq * pl.RQp * 4, cudaMemcpyDeviceToDevice, st);
     finalize_groups(pl, ws, pl.Cq, 0, out.q_label, out.perm_q, out.pos_q, out.q_offsets, out.n_groups, st);
-    gather(Q, out.perm_q, pl, out.Qp, 1, st);
+    gather(Q, out.perm_q, pl, BH, 1, out.Qp, st);
     count_launch(), group_mean_kernel<T><<<dim3(pl.Cq, BH), d, 0, st>>>(static_cast<const T*>(out.Qp), out.q_offsets,
-                                                        out.n_groups, 0, N, pl.Cq, d, out.q_centroid);
+                                                        out.n_groups, 0, N, pl.Cq, d, 1, out.q_centroid);
     // c_a (phi_Q space) into the query-centre buffer, then d_i (A.2)
     count_launch(), group_mean_indirect_kernel<<<dim3(pl.Cq, BH), pl.RQp > 64 ? pl.RQp : 64, 0, st>>>(
                                                               phiQ, out.perm_q, out.q_offsets,

@@ -24,7 +24,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) route_partial_kernel(
     const T* __restrict__ Kp, const T* __restrict__ Vp, const int32_t* __restrict__ kv_off,
     const int32_t* __restrict__ ng, const float* __restrict__ vbar, const float* __restrict__ qbar,
-    int N, int Cq, int Ck, int d, float* __restrict__ t1o, float* __restrict__ t2o,
+    int N, int Cq, int Ck, int d, int G, float* __restrict__ t1o, float* __restrict__ t2o,
     float* __restrict__ mloc) {
     constexpr int RB = 64;
     extern __shared__ float sm[];
@@ -51,8 +51,8 @@ __global__ void __launch_bounds__(256) route_partial_kernel(
         const int n = min(RB, e - r0);
         __syncthreads();
         for (int rr = warp; rr < n; rr += 8) {
-            const T* kr = Kp + ((size_t)bh * N + r0 + rr) * d;
-            const T* vr = Vp + ((size_t)bh * N + r0 + rr) * d;
+            const T* kr = Kp + ((size_t)(bh / G) * N + r0 + rr) * d;   // the K/V head under GQA
+            const T* vr = Vp + ((size_t)(bh / G) * N + r0 + rr) * d;
             float uu = 0.f, ww = 0.f;
             for (int t = lane; t < d; t += 32) {
                 ks[rr * ld + t] = ldf(kr + t);
@@ -460,7 +460,7 @@ void route_partial(const Plan& pl, const sparsepr_partition_out& part, float* t1
     cudaFuncSetAttribute(route_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     count_launch(), route_partial_kernel<T><<<dim3(pl.Ck, (pl.Cq + 7) / 8, pl.BH), 256, smem, st>>>(
         static_cast<const T*>(part.Kp), static_cast<const T*>(part.Vp), part.kv_offsets,
-        part.n_groups, part.v_centroid, part.q_centroid, pl.N, pl.Cq, pl.Ck, d, t1, t2, ml);
+        part.n_groups, part.v_centroid, part.q_centroid, pl.N, pl.Cq, pl.Ck, d, pl.G, t1, t2, ml);
 }
 
 }  // namespace

@@ -64,18 +64,20 @@ __global__ void route_qsplit_kernel(const float* __restrict__ qbar, const int32_
     }
 }
 
-// u_j = vbar_b . v_j and w_j = |v_j|^2 for every permuted key row j (b its group).
+// u_j = vbar_b . v_j and w_j = |v_j|^2 for every permuted key row j (b its
+// group), once per K/V head: under GQA the G query heads of a K/V head share
+// its groups, centroids and rows, so head kh reads query head kh * G's.
 template <typename T>
 __global__ void route_uw_kernel(const T* __restrict__ Vp, const float* __restrict__ vbar,
-                                const int32_t* __restrict__ kv_label, const int32_t* __restrict__ perm_kv, int BH, int N,
-                                int Ck, int d, float2* __restrict__ uw) {
+                                const int32_t* __restrict__ kv_label, const int32_t* __restrict__ perm_kv, int BHk,
+                                int N, int Ck, int d, int G, float2* __restrict__ uw) {
     const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
     const int lane = threadIdx.x & 31;
-    for (size_t row = blockIdx.x * (size_t)(blockDim.x >> 5) + (threadIdx.x >> 5); row < (size_t)BH * N; row += warps) {
-        const size_t bh = row / N;
-        const int b = kv_label[bh * N + perm_kv[row]];
+    for (size_t row = blockIdx.x * (size_t)(blockDim.x >> 5) + (threadIdx.x >> 5); row < (size_t)BHk * N; row += warps) {
+        const size_t kh = row / N, qh = kh * G, r = row - kh * N;
+        const int b = kv_label[qh * N + perm_kv[qh * N + r]];
         const T* v = Vp + row * d;
-        const float* vb = vbar + (bh * Ck + b) * d;
+        const float* vb = vbar + (qh * Ck + b) * d;
         float u = 0.f, w = 0.f;
         for (int t = lane; t < d; t += 32) {
             const float x = ldf(v + t);
@@ -91,7 +93,7 @@ __global__ void route_uw_kernel(const T* __restrict__ Vp, const float* __restric
 template <int D>
 __global__ void __launch_bounds__(192, 1) route_tc_kernel(
     const __grid_constant__ rtc::Maps maps, const float2* __restrict__ uw, const int32_t* __restrict__ kv_off,
-    const int32_t* __restrict__ ng, int N, int Cq, int Ck, int CqPad, float* __restrict__ t1o,
+    const int32_t* __restrict__ ng, int N, int Cq, int Ck, int CqPad, int G, float* __restrict__ t1o,
     float* __restrict__ t2o, float* __restrict__ mloc, DevStatus* status) {
     using namespace rtc;
     using namespace sm100;
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
             __syncwarp();
             for (int c = lane; c < BK; c += 32) {
                 const int j = j0 + c;
-                const float2 v = (j < j_end) ? uw[(size_t)bh * N + j] : make_float2(0.f, 0.f);
+                const float2 v = (j < j_end) ? uw[(size_t)(bh / G) * N + j] : make_float2(0.f, 0.f);
                 meta[c] = v.x;
                 meta[BK + c] = v.y;
             }
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
                 mbar_arrive_expect_tx(bar(B_BF + stage), L::KB);
                 for (int hh = 0; hh < D / 64; ++hh)
                     tma_load_2d(s_base + L::oK + stage * L::KB + hh * BK * 128, &maps.k, bar(B_BF + stage), hh * 64,
-                                bh * N + j0);
+                                (bh / G) * N + j0);
             }
             issued = t + 1;
         }
@@ -337,20 +339,22 @@ bool launch_route_tc(const Plan& pl, const sparsepr_partition_out& part, void* w
     float2* uw = at<float2>(ws, pl.o_uw);
     DevStatus* status = at<DevStatus>(ws, pl.o_status);
     count_launch(), route_qsplit_kernel<<<dim3(64, BH), 256, 0, st>>>(part.q_centroid, part.n_groups, pl.Cq, CqPad, d, qs);
+    const int G = pl.G, BHk = BH / G;
     count_launch(), route_uw_kernel<__nv_bfloat16><<<148 * 8, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(part.Vp), part.v_centroid, part.kv_label, part.perm_kv, BH, N, pl.Ck, d, uw);
+        static_cast<const __nv_bfloat16*>(part.Vp), part.v_centroid, part.kv_label, part.perm_kv, BHk, N, pl.Ck, d, G,
+        uw);
     rtc::Maps maps;
     if (!make_bf16_rows(&maps.a, qs, (uint64_t)BH * 3 * CqPad, d)) return false;
-    if (!make_bf16_rows(&maps.k, part.Kp, (uint64_t)BH * N, d)) return false;
+    if (!make_bf16_rows(&maps.k, part.Kp, (uint64_t)BHk * N, d)) return false;
     const dim3 grid((pl.Ck + rtc::GPB - 1) / rtc::GPB, CqPad / rtc::BA, BH);
     if (d == 128) {
         cudaFuncSetAttribute(route_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, rtc::Layout<128>::smem);
         count_launch(), route_tc_kernel<128><<<grid, 192, rtc::Layout<128>::smem, st>>>(
-            maps, uw, part.kv_offsets, part.n_groups, N, pl.Cq, pl.Ck, CqPad, t1, t2, ml, status);
+            maps, uw, part.kv_offsets, part.n_groups, N, pl.Cq, pl.Ck, CqPad, G, t1, t2, ml, status);
     } else {
         cudaFuncSetAttribute(route_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, rtc::Layout<64>::smem);
         count_launch(), route_tc_kernel<64><<<grid, 192, rtc::Layout<64>::smem, st>>>(
-            maps, uw, part.kv_offsets, part.n_groups, N, pl.Cq, pl.Ck, CqPad, t1, t2, ml, status);
+            maps, uw, part.kv_offsets, part.n_groups, N, pl.Cq, pl.Ck, CqPad, G, t1, t2, ml, status);
     }
     return true;
 }

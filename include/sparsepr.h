@@ -138,8 +138,10 @@ typedef struct {
 /* Outputs of sparsepr_partition (paper §4.1).  Required unless marked
  * optional (NULL = not written).  Sizes: BH*N int32 for per-row arrays. */
 typedef struct {
-    void* Qp; void* Kp; void* Vp; /* [BH,N,d] p->dtype: rows in group-major order,
-                                     stable by original index (§4.3); V keeps its key's row */
+    void* Qp;             /* [BH,N,d] p->dtype: rows in group-major order, stable by original index (§4.3) */
+    void* Kp; void* Vp;   /* [B*Hkv,N,d] p->dtype: the same for the keys (V keeps its key's row), one per
+                             K/V head: under GQA the G query heads of a K/V head share its groups, so
+                             its rows are stored once (without GQA, Hkv = H) */
     int32_t* q_label;     /* [BH,N] query group of each ORIGINAL row (0..C_q'-1) */
     int32_t* kv_label;    /* [BH,N] K/V group of each original key row */
     int32_t* perm_q;      /* [BH,N] permuted row -> original row */

@@ -65,7 +65,9 @@ def head_view(res, cfg, bh):
     h["q_offsets"] = npi(p["q_offsets"][bh])[: Cq2 + 1]
     h["kv_offsets"] = npi(p["kv_offsets"][bh])[: Ck2 + 1]
     b, hh = divmod(bh, cfg.H)
-    h["Qp"], h["Kp"], h["Vp"] = (np64(p[n][b, hh]) for n in ("Qp", "Kp", "Vp"))
+    hk = hh // (cfg.H // cfg.Hk)   # permuted K/V live per K/V head
+    h["Qp"] = np64(p["Qp"][b, hh])
+    h["Kp"], h["Vp"] = (np64(p[n][b, hk]) for n in ("Kp", "Vp"))
     h["q_centroid"] = np64(p["q_centroid"][bh])[:Cq2]
     h["k_centroid"] = np64(p["k_centroid"][bh])[:Ck2]
     h["v_centroid"] = np64(p["v_centroid"][bh])[:Ck2]

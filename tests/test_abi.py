@@ -106,6 +106,19 @@ def test_workspace_size_and_host_errors(L):
     assert _abi.STATUS_NAMES[5] == "TIMEOUT"
 
 
+def test_gqa_keeps_one_permuted_kv_per_kv_head(L):
+    """Under GQA the permuted K and V and the fp16 copy of V are stored once
+    per K/V head: the workspace of G = 4 query heads per K/V head is smaller
+    by at least (G - 1)/G of those buffers (bf16 K, V and the fp16 V copy)."""
+    H, G = 8, 4
+    base = _cfg(H=H, dtype="bf16", d=128, block=128)
+    n_mha = L.sparsepr_workspace_size(ctypes.byref(base.c_params()))
+    n_gqa = L.sparsepr_workspace_size(ctypes.byref(_cfg(H=H, dtype="bf16", d=128, block=128, Hkv=H // G).c_params()))
+    kv_bytes = 3 * base.B * H * base.N * base.d * 2   # Kp, Vp and the fp16 V copy per query head
+    gqa_only = base.B * (H // G) * base.N * 4 + 256      # raw labels of the K/V heads' k-means
+    assert 0 < n_gqa <= n_mha - kv_bytes * (G - 1) // G + gqa_only
+
+
 def test_ctypes_layouts_match_c(L):
     from free_block_sparse_sampled_b200 import _abi
     structs = {"sparsepr_params": _abi.Params, "sparsepr_partition_out": _abi.PartitionOut,
