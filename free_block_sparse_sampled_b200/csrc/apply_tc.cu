@@ -460,8 +460,20 @@ __global__ void __maxnreg__(144) apply_t_kernel(
         bool ok = true;
         int heads = 0, cur_bh = -1, i = 0;
         float bias = 0.f;
+        // row indices of a tile (probe slot, destination row) for this half of
+        // its rows: lane l holds rows 64 hrow + l and + 32; loaded one tile ahead
+        auto load_rows = [&](int w, int& sl0, int& sl1, int& dq0, int& dq1) {
+            const int bhw = w / tiles_per_head, r0 = (w % tiles_per_head) * BM + 64 * hrow + lane, r1 = r0 + 32;
+            const size_t hb = (size_t)bhw * N;
+            sl0 = r0 < N ? pslot[hb + r0] : -2;
+            sl1 = r1 < N ? pslot[hb + r1] : -2;
+            dq0 = r0 < N ? perm_q[hb + r0] : 0;
+            dq1 = r1 < N ? perm_q[hb + r1] : 0;
+        };
+        int nsl0 = -2, nsl1 = -2, ndq0 = 0, ndq1 = 0;
+        if (w_begin < w_end) load_rows(w_begin, nsl0, nsl1, ndq0, ndq1);
         for (int w = w_begin; ok && w < w_end; ++w, ++i) {
-            const int bh = w / tiles_per_head, p0 = (w % tiles_per_head) * BM;
+            const int bh = w / tiles_per_head;
             if (bh != cur_bh) {
                 // B'^T of this head into TMEM, once the previous head's MMAs are done:
                 // lane n, column k holds B[k][n] (+ sigma[n] on the diagonal), hi and lo
@@ -492,11 +504,9 @@ __global__ void __maxnreg__(144) apply_t_kernel(
                 ++heads;
             }
             const int d = i & 1;
-            // the row indices of this half of the tile: lane l holds rows 64 hrow + l and + 32
-            const int r0 = p0 + 64 * hrow + lane, r1 = r0 + 32;
             const size_t hb = (size_t)bh * N;
-            const int sl0 = r0 < N ? pslot[hb + r0] : -2, sl1 = r1 < N ? pslot[hb + r1] : -2;
-            const int dq0 = r0 < N ? perm_q[hb + r0] : 0, dq1 = r1 < N ? perm_q[hb + r1] : 0;
+            const int sl0 = nsl0, sl1 = nsl1, dq0 = ndq0, dq1 = ndq1;
+            if (w + 1 < w_end) load_rows(w + 1, nsl0, nsl1, ndq0, ndq1);
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + d), (i >> 1) & 1, abort_flag, kSpin));
             if (!ok) break;
             tc_fence_after();
