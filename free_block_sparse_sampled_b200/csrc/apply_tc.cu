@@ -272,6 +272,10 @@ __global__ void __maxnreg__(168) apply_tc_kernel(
 namespace aptt {
 constexpr int D = 128, BM = 128, NCH = 4, NST = 4;
 constexpr int kThreads = 448;
+// each SM sub-partition holds 16384 registers and takes every fourth warp of
+// the block: ceil(14 / 4) = 4 warps of 32 threads at kRegs registers must fit
+constexpr int kRegs = 128;
+static_assert((kThreads / 32 + 3) / 4 * 32 * kRegs <= 16384, "registers per sub-partition");
 constexpr uint32_t kSpin = 1u << 20;
 enum { B_RF = 0, B_XF = NST, B_XE = 2 * NST, B_DF = 3 * NST, B_DE = 3 * NST + 2, B_AF = 3 * NST + 4,
        B_AE = 3 * NST + 5, B_DR = 3 * NST + 6, B_SS = 3 * NST + 7, N_BAR = 3 * NST + 9 };
@@ -285,7 +289,7 @@ constexpr int kSmem = oMisc + 16 + 1024;
 static_assert(oLo % 1024 == 0 && oStat % 16 == 0, "alignment");
 }  // namespace aptt
 
-__global__ void __maxnreg__(144) apply_t_kernel(
+__global__ void __maxnreg__(aptt::kRegs) apply_t_kernel(
     const __grid_constant__ CUtensorMap osp_map, const float* __restrict__ Bm, const float* __restrict__ mu_x,
     const float* __restrict__ sigma, const float* __restrict__ mu_r, const int32_t* __restrict__ pslot,
     const float* __restrict__ probe_dense, const int32_t* __restrict__ perm_q, int BH, int N, int Mp,
