@@ -7,11 +7,13 @@
 // accumulation error.  The -|c|^2/2 term joins the product as one more K step:
 // a constant tile of ones (two columns) against each centre's -|c|^2/2 split
 // into TF32 hi and lo parts, so the tensor core returns the score itself.
-// Centres stream through shared memory in blocks of up to 256 (TMA, 128-byte
-// swizzle, two stages, with their split half-norms 32-byte swizzled); the
-// scores of a block land in TMEM (two buffers) and eight epilogue warps (two
-// per TMEM lane quadrant, each owning half of the columns) take the running
-// argmax while the next block multiplies.  All waits are bounded.
+// Coordinates and centres move through shared memory as 16-float column
+// chunks (TMA, 64-byte swizzle, sized to the rank): the points of an item in
+// two buffers, the centres in blocks of up to 256 in two stages, with their
+// split half-norms 32-byte swizzled.  The scores of a block land in TMEM (two
+// buffers) and eight epilogue warps (two per TMEM lane quadrant, each owning
+// half of the columns) take the running argmax while the next block
+// multiplies.  All waits are bounded.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -21,22 +23,36 @@
 namespace spr {
 namespace kmtc {
 constexpr int BP = 128;                 // points per item (TMEM lanes)
-constexpr int NBMAX = 256;              // centres per MMA block
 constexpr uint32_t kSpin = 1u << 20;
 enum { B_AF = 0, B_AE = 2, B_BF = 4, B_BE = 6, B_DF = 8, B_DE = 10, B_DR = 12, N_BAR = 13 };
-constexpr int oA = 0;                                   // 2 buffers x 2 chunks x 128 rows x 128 B
-constexpr int oB = oA + 2 * 2 * BP * 128;               // 2 stages x 2 chunks x 256 rows x 128 B
-constexpr int oOnes = oB + 2 * 2 * NBMAX * 128;        // 128 rows x 8 TF32: ones in columns 0 and 1
-constexpr int oH = oOnes + BP * 32;                     // 2 stages x NBMAX x 8 TF32: (hi, lo, 0 ...) of -|c|^2/2
-constexpr int oBar2 = oH + 2 * NBMAX * 32;
-constexpr int oRed = oBar2 + N_BAR * 8;                 // 128 x (score, index) of the upper half
-constexpr int oMisc = oRed + BP * 8;
-constexpr int kSmem = oMisc + 64 + 1024;
-static_assert(oOnes % 256 == 0 && oH % 256 == 0, "32-byte swizzled tiles need 256-byte alignment");
+constexpr int kKeepStride = 144;        // bytes per lane of the best-chunk copy (32 floats + 16: no bank conflicts)
+
+// Shared-memory plan for rank R and centre blocks of NB (every tile 1024-aligned):
+//   A: 2 buffers x R/16 chunks x 128 rows x 64 B; B: 2 stages x R/16 chunks x NB rows x 64 B;
+//   a 128 x 8 TF32 ones tile and 2 stages x NB x 8 TF32 split half-norms (32-byte swizzle);
+//   per epilogue lane a copy of its best 32-score chunk; barriers; the half merge.
+struct Layout {
+    int a_buf, b_stage, oA, oB, oOnes, oH, oKeep, oBar, oRed, oMisc, bytes;
+    __host__ __device__ Layout(int R, int NB) {
+        a_buf = BP * R * 4;
+        b_stage = NB * R * 4;
+        oA = 0;
+        oB = oA + 2 * a_buf;
+        oOnes = oB + 2 * b_stage;
+        oH = oOnes + BP * 32;
+        oKeep = oH + 2 * NB * 32;
+        oBar = oKeep + 8 * 32 * kKeepStride;
+        oRed = oBar + N_BAR * 8;
+        oMisc = oRed + BP * 8;
+        bytes = oMisc + 64 + 1024;
+    }
+};
+// largest centre block for rank R that keeps the plan within 227 KB
+__host__ __device__ constexpr int nb_max(int R) { return R > 48 ? 192 : 256; }
 
 struct Maps {
-    CUtensorMap pts;       // [BH*N, R] fp32, box 32 x 128
-    CUtensorMap cen;       // [BH*C, R] fp32, box 32 x NB
+    CUtensorMap pts;       // [BH*N, R] fp32, box 16 x 128, 64-byte swizzle
+    CUtensorMap cen;       // [BH*C, R] fp32, box 16 x NB, 64-byte swizzle
     CUtensorMap hs;        // [BH*C, 8] fp32, box 8 x NB, 32-byte swizzle
 };
 
@@ -56,6 +72,74 @@ __global__ void half_norm_split_kernel(const float* __restrict__ hn, size_t n, f
         o[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
+// Maximum of 32 scores as a tree of three-way maxima.
+__device__ __forceinline__ float max32(const float (&s)[32]) {
+    using sm100::fmax3;
+    float m3[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) m3[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+    m3[10] = fmaxf(s[30], s[31]);
+    return fmaxf(fmax3(fmax3(m3[0], m3[1], m3[2]), fmax3(m3[3], m3[4], m3[5]), fmax3(m3[6], m3[7], m3[8])),
+                 fmaxf(m3[9], m3[10]));
+}
+
+// Stores 16 scores at a shared-window address when p holds (predicated, no branch).
+__device__ __forceinline__ void st_shared_16_if(uint32_t a, bool p, const float* s) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+        "@q st.shared.v4.f32 [%0], {%2, %3, %4, %5};\n\t"
+        "@q st.shared.v4.f32 [%0+16], {%6, %7, %8, %9};\n\t"
+        "@q st.shared.v4.f32 [%0+32], {%10, %11, %12, %13};\n\t"
+        "@q st.shared.v4.f32 [%0+48], {%14, %15, %16, %17};\n\t}" ::"r"(a),
+        "r"((int)p), "f"(s[0]), "f"(s[1]), "f"(s[2]), "f"(s[3]), "f"(s[4]), "f"(s[5]), "f"(s[6]), "f"(s[7]),
+        "f"(s[8]), "f"(s[9]), "f"(s[10]), "f"(s[11]), "f"(s[12]), "f"(s[13]), "f"(s[14]), "f"(s[15])
+        : "memory");
+}
+
+// One 64-column pair of an epilogue lane: the chunks of 32 scores at columns
+// cb0 and cb0 + 32, of which the columns below lim take part.  MODE 0: both
+// chunks whole; 1: the first whole and the second past lim; 2: columns at or
+// past lim masked to -inf.  Both chunk maxima are taken before either updates
+// the running first maximum (best, the base column bcb of its chunk), and the
+// lane's copy of its best chunk at `keep` is rewritten by predicated stores,
+// so a pair is one branch-free stretch of code.
+template <int MODE, bool DBG>
+__device__ __forceinline__ void pair_update(float (&v)[2][32], int cb0, int lim, float& best, int& bcb, uint32_t keep,
+                                            float* dbg_row) {
+    if (MODE == 2) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[q][i] = (cb0 + 32 * q + i < lim) ? v[q][i] : -INFINITY;
+    }
+    if (DBG && dbg_row != nullptr) {
+#pragma unroll
+        for (int q = 0; q < (MODE == 1 ? 1 : 2); ++q)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (cb0 + 32 * q + i < lim) dbg_row[cb0 + 32 * q + i] = v[q][i];
+    }
+    const float m0 = max32(v[0]);
+    if (MODE == 1) {
+        const bool up0 = m0 > best;   // a later chunk only wins with a strictly larger score
+        best = up0 ? m0 : best;
+        bcb = up0 ? cb0 : bcb;
+        st_shared_16_if(keep, up0, v[0]);
+        st_shared_16_if(keep + 64, up0, v[0] + 16);
+        return;
+    }
+    const float m1 = max32(v[1]);
+    const bool up0 = m0 > best;
+    const float b0 = up0 ? m0 : best;
+    const bool up1 = m1 > b0;
+    best = up1 ? m1 : b0;
+    bcb = up1 ? cb0 + 32 : (up0 ? cb0 : bcb);
+    const bool s0 = up0 && !up1;
+    st_shared_16_if(keep, s0, v[0]);
+    st_shared_16_if(keep + 64, s0, v[0] + 16);
+    st_shared_16_if(keep, up1, v[1]);
+    st_shared_16_if(keep + 64, up1, v[1] + 16);
+}
 }  // namespace kmtc
 
 // Persistent: block k handles items k, k + grid, ... where an item is 128
@@ -74,12 +158,23 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
     const int n_items = BH * tiles_per_head;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_u32(sm);
-    auto bar = [&](int i) -> uint32_t { return s_base + oBar2 + 8 * i; };
-    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + oMisc);
+    const Layout L(R, NB);
+    auto bar = [&](int i) -> uint32_t { return s_base + L.oBar + 8 * i; };
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L.oMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-    const int nchunk = (R + 31) / 32;           // 32 fp32 per 128-byte row chunk
+    const int nchunk = R / 16;                  // 16 fp32 per 64-byte row chunk
     const int ksteps = R / 8;                   // kind::tf32 K = 8 per instruction
-    auto item_live = [&](int w) -> bool { return ctl[(w / tiles_per_head) * kCtlStride + kCtlDone] == 0; };
+    // a head's stop flag is set between launches: each role reads it once per head
+    int live_bh = -1;
+    bool live = false;
+    auto item_live = [&](int w) -> bool {
+        const int bh = w / tiles_per_head;
+        if (bh != live_bh) {
+            live_bh = bh;
+            live = ctl[bh * kCtlStride + kCtlDone] == 0;
+        }
+        return live;
+    };
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -95,7 +190,7 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         misc[1] = 0;
     }
     {   // the ones tile of the half-norm K step: columns 0 and 1 of every row
-        float* ones = reinterpret_cast<float*>(sm + oOnes);
+        float* ones = reinterpret_cast<float*>(sm + L.oOnes);
         for (int e = tid; e < BP * 8; e += blockDim.x) {
             const int row = e >> 3, k = e & 7;
             ones[sw32(row, k) >> 2] = k < 2 ? 1.f : 0.f;
@@ -122,17 +217,18 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                 if (!item_live(w)) continue;
                 const int bh = w / tiles_per_head, p0 = (w % tiles_per_head) * BP, ab = li & 1;
                 if (li >= 2 && !mbar_wait(bar(B_AE + ab), ((li >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
-                mbar_arrive_expect_tx(bar(B_AF + ab), nchunk * BP * 128);
+                mbar_arrive_expect_tx(bar(B_AF + ab), L.a_buf);
                 for (int ch = 0; ch < nchunk; ++ch)
-                    tma_load_2d(s_base + oA + (ab * 2 + ch) * BP * 128, &maps.pts, bar(B_AF + ab), ch * 32, bh * N + p0);
+                    tma_load_2d(s_base + L.oA + ab * L.a_buf + ch * BP * 64, &maps.pts, bar(B_AF + ab), ch * 16,
+                                bh * N + p0);
                 for (int blk = 0; blk < nblk; ++blk, ++gb) {
                     const int stage = gb & 1;
                     if (gb >= 2 && !mbar_wait(bar(B_BE + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
-                    mbar_arrive_expect_tx(bar(B_BF + stage), nchunk * NB * 128 + NB * 32);
+                    mbar_arrive_expect_tx(bar(B_BF + stage), L.b_stage + NB * 32);
                     for (int ch = 0; ch < nchunk; ++ch)
-                        tma_load_2d(s_base + oB + (stage * 2 + ch) * NBMAX * 128, &maps.cen, bar(B_BF + stage),
-                                    ch * 32, bh * C + blk * NB);
-                    tma_load_2d(s_base + oH + stage * NBMAX * 32, &maps.hs, bar(B_BF + stage), 0, bh * C + blk * NB);
+                        tma_load_2d(s_base + L.oB + stage * L.b_stage + ch * NB * 64, &maps.cen, bar(B_BF + stage),
+                                    ch * 16, bh * C + blk * NB);
+                    tma_load_2d(s_base + L.oH + stage * NB * 32, &maps.hs, bar(B_BF + stage), 0, bh * C + blk * NB);
                 }
                 ++li;
             }
@@ -149,29 +245,30 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                                    ((uint32_t)(BP >> 4) << 24);   // F32 <- TF32 x TF32, K-major both
             // descriptors built once; each MMA adds its offset (>> 4) to the
             // start-address field, which never carries out (shared < 2^18)
-            const uint64_t dA = smem_desc(s_base + oA, 16, 1024), dB = smem_desc(s_base + oB, 16, 1024);
-            const uint64_t dOnes = smem_desc_sw32(s_base + oOnes), dH = smem_desc_sw32(s_base + oH);
+            const uint64_t dA = smem_desc_sw64(s_base + L.oA), dB = smem_desc_sw64(s_base + L.oB);
+            const uint64_t dOnes = smem_desc_sw32(s_base + L.oOnes), dH = smem_desc_sw32(s_base + L.oH);
             int li = 0, gb = 0;
             bool ok = true;
             for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
                 if (!item_live(w)) continue;
                 const int ab = li & 1;
                 if (!mbar_wait(bar(B_AF + ab), (li >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
-                const uint64_t a0 = dA + (uint64_t)((ab * 2 * BP * 128) >> 4);
+                const uint64_t a0 = dA + (uint64_t)((ab * L.a_buf) >> 4);
                 for (int blk = 0; blk < nblk; ++blk, ++gb) {
                     const int stage = gb & 1;
                     if (!mbar_wait(bar(B_BF + stage), (gb >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
                     if (gb >= 2 && !mbar_wait(bar(B_DE + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t b0 = dB + (uint64_t)((stage * 2 * NBMAX * 128) >> 4);
+                    const uint64_t b0 = dB + (uint64_t)((stage * L.b_stage) >> 4);
                     const uint32_t d = tmem + stage * NB;
                     for (int kk = 0; kk < ksteps; ++kk) {
-                        const uint64_t off = (uint64_t)(((kk >> 2) * BP * 128 + (kk & 3) * 32) >> 4);
-                        const uint64_t offb = (uint64_t)(((kk >> 2) * NBMAX * 128 + (kk & 3) * 32) >> 4);
+                        // K step kk: chunk kk / 2, 32 bytes further inside the 64-byte row for odd kk
+                        const uint64_t off = (uint64_t)(((kk >> 1) * BP * 64 + (kk & 1) * 32) >> 4);
+                        const uint64_t offb = (uint64_t)(((kk >> 1) * NB * 64 + (kk & 1) * 32) >> 4);
                         mma_tf32_ss(d, a0 + off, b0 + offb, idesc, kk > 0 ? 1u : 0u);
                     }
                     // + 1 * hi + 1 * lo: the -|c|^2/2 term of every score
-                    mma_tf32_ss(d, dOnes, dH + (uint64_t)((stage * NBMAX * 32) >> 4), idesc, 1u);
+                    mma_tf32_ss(d, dOnes, dH + (uint64_t)((stage * NB * 32) >> 4), idesc, 1u);
                     mma_commit(bar(B_DF + stage));
                     mma_commit(bar(B_BE + stage));
                 }
@@ -190,8 +287,10 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
         const int half = warp >> 2, row = (warp & 3) * 32 + lane;
         const uint32_t t_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const int hw = NB / 2;
-        float* red_s = reinterpret_cast<float*>(sm + oRed);
-        int* red_i = reinterpret_cast<int*>(sm + oRed + BP * 4);
+        float* red_s = reinterpret_cast<float*>(sm + L.oRed);
+        int* red_i = reinterpret_cast<int*>(sm + L.oRed + BP * 4);
+        // this lane's copy of its best chunk
+        const uint32_t keep = s_base + L.oKeep + (uint32_t)(warp * 32 + lane) * kKeepStride;
         int gb = 0;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
@@ -202,57 +301,33 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
             // previous label, read now and used after the last centre block
             const int old_label = (valid && !first) ? labels[(size_t)bh * N + p] : 0;
             // running first maximum over this half's columns, in column order: the
-            // best value, the base column of the chunk holding it and a copy of
-            // that chunk's scores (predicated copies instead of a per-chunk index
-            // search, which every chunk would run: some lane of the warp almost
-            // always improves); the index is searched once per item
+            // best value, the base column of the chunk holding it and, in shared
+            // memory, a copy of that chunk's scores (eight predicated vector
+            // stores instead of a per-chunk index search, which every chunk would
+            // run: some lane of the warp almost always improves); the index is
+            // searched once per item
             float best = -INFINITY;
             int bcb = 0;
-            float keep[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) keep[i] = -INFINITY;
+            float* dbg_row = (DBG && valid) ? dbg_scores + ((size_t)bh * N + p) * C : nullptr;
             for (int blk = 0; blk < nblk; ++blk, ++gb) {
                 const int db = gb & 1;
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + db), (gb >> 1) & 1, abort_flag, kSpin));
                 if (!ok) break;
                 tc_fence_after();
+                // the columns of this half that hold centres of this head
+                const int lim = min(C, blk * NB + (half + 1) * hw);
                 for (int c0 = 0; c0 < hw; c0 += 64) {
-                    const bool two = c0 + 32 < hw;   // warp-uniform
+                    const int cb0 = blk * NB + half * hw + c0;   // warp-uniform
+                    if (cb0 >= lim) break;
+                    // 64 columns (those past the half stay inside the allocation and are masked)
                     float v[2][32];
                     tmem_ld32(t_row + db * NB + half * hw + c0, v[0]);
-                    if (two) tmem_ld32(t_row + db * NB + half * hw + c0 + 32, v[1]);
+                    tmem_ld32(t_row + db * NB + half * hw + c0 + 32, v[1]);
                     tmem_wait_ld(v[0]);
-                    if (two) tmem_wait_ld(v[1]);
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        if (q == 1 && !two) break;
-                        const int cb = blk * NB + half * hw + c0 + 32 * q;
-                        float sc[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) sc[i] = v[q][i];
-                        if (cb + 32 > C) {   // columns past C (another head's centres or zero fill) never win
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) sc[i] = (cb + i < C) ? sc[i] : -INFINITY;
-                        }
-                        if (DBG) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (valid && cb + i < C) dbg_scores[((size_t)bh * N + p) * C + cb + i] = sc[i];
-                        }
-                        // chunk maximum as a tree of three-way maxima
-                        float m3[11];
-#pragma unroll
-                        for (int i = 0; i < 10; ++i) m3[i] = fmax3(sc[3 * i], sc[3 * i + 1], sc[3 * i + 2]);
-                        m3[10] = fmaxf(sc[30], sc[31]);
-                        const float m = fmaxf(fmax3(fmax3(m3[0], m3[1], m3[2]), fmax3(m3[3], m3[4], m3[5]),
-                                                    fmax3(m3[6], m3[7], m3[8])),
-                                              fmaxf(m3[9], m3[10]));
-                        const bool up = m > best;   // a later chunk only wins with a strictly larger score
-                        best = up ? m : best;
-                        bcb = up ? cb : bcb;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) keep[i] = up ? sc[i] : keep[i];
-                    }
+                    tmem_wait_ld(v[1]);
+                    if (cb0 + 64 <= lim) pair_update<0, DBG>(v, cb0, lim, best, bcb, keep, dbg_row);
+                    else if (cb0 + 32 == lim) pair_update<1, DBG>(v, cb0, lim, best, bcb, keep, dbg_row);
+                    else pair_update<2, DBG>(v, cb0, lim, best, bcb, keep, dbg_row);
                 }
                 tc_fence_before();
                 mbar_arrive(bar(B_DE + db));
@@ -260,9 +335,12 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
             if (!ok) break;
             int bi = 0x7fffffff;
             if (best > -INFINITY) {
+                float kv[32];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ld_shared_v4(keep + 16 * j, kv[4 * j], kv[4 * j + 1], kv[4 * j + 2], kv[4 * j + 3]);
                 int idx = 31;
 #pragma unroll
-                for (int i = 30; i >= 0; --i) idx = (keep[i] == best) ? i : idx;
+                for (int i = 30; i >= 0; --i) idx = (kv[i] == best) ? i : idx;
                 bi = bcb + idx;
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -333,21 +411,23 @@ bool make_f32_map(CUtensorMap* m, const void* base, uint64_t rows, int R, int bo
 }
 }  // namespace
 
-void kmeans_centre_blocks(int C, int& NB, int& nblk) {
-    nblk = (C + kmtc::NBMAX - 1) / kmtc::NBMAX;
+void kmeans_centre_blocks(int C, int R, int& NB, int& nblk) {
+    const int nbm = kmtc::nb_max(R);
+    nblk = (C + nbm - 1) / nbm;
     NB = round_up((C + nblk - 1) / nblk, 64);
-    if (NB > kmtc::NBMAX) NB = kmtc::NBMAX;
+    if (NB > nbm) NB = nbm;
 }
 
 bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn, float* hs, int BH, int N, int C,
                              int R, int32_t* labels, int32_t* ctl, int first, float* dbg_scores, int32_t* dbg_hist,
                              int max_iter, DevStatus* status, cudaStream_t st) {
-    if (R > kMaxRank) return false;              // shared-memory tiles hold rows of up to 64 floats
+    if (R > kMaxRank || R % 16 != 0) return false;   // 16-float chunks of rows of up to 64 floats
     int NB, nblk;
-    kmeans_centre_blocks(C, NB, nblk);
+    kmeans_centre_blocks(C, R, NB, nblk);
+    const kmtc::Layout L(R, NB);
     kmtc::Maps maps;
-    if (!make_f32_map(&maps.pts, phi, (uint64_t)BH * N, R, kmtc::BP)) return false;
-    if (!make_f32_map(&maps.cen, cen, (uint64_t)BH * C, R, NB)) return false;
+    if (!make_f32_map(&maps.pts, phi, (uint64_t)BH * N, R, kmtc::BP, 16, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
+    if (!make_f32_map(&maps.cen, cen, (uint64_t)BH * C, R, NB, 16, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
     if (!make_f32_map(&maps.hs, hs, (uint64_t)BH * C, 8, NB, 8, CU_TENSOR_MAP_SWIZZLE_32B)) return false;
     {
         const size_t n = (size_t)BH * C;
@@ -357,12 +437,12 @@ bool launch_kmeans_assign_tc(const float* phi, const float* cen, const float* hn
     const int items = BH * ((N + kmtc::BP - 1) / kmtc::BP);
     const int grid = items < sm_count() ? items : sm_count();
     if (dbg_scores != nullptr) {
-        cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
-        count_launch(), kmeans_assign_tc_kernel<true><<<grid, 320, kmtc::kSmem, st>>>(
+        cudaFuncSetAttribute(kmeans_assign_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, L.bytes);
+        count_launch(), kmeans_assign_tc_kernel<true><<<grid, 320, L.bytes, st>>>(
             maps, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
     } else {
-        cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kmtc::kSmem);
-        count_launch(), kmeans_assign_tc_kernel<false><<<grid, 320, kmtc::kSmem, st>>>(
+        cudaFuncSetAttribute(kmeans_assign_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, L.bytes);
+        count_launch(), kmeans_assign_tc_kernel<false><<<grid, 320, L.bytes, st>>>(
             maps, BH, N, C, R, NB, nblk, labels, ctl, first, dbg_scores, dbg_hist, max_iter, status);
     }
     return true;

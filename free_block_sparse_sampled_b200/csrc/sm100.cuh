@@ -183,6 +183,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t addr) {
     return desc;
 }
 
+// The same for a K-major tile of 64-byte rows (16 fp32 / TF32) in the 64-byte
+// swizzle (swizzle mode 4): 8-row groups 512 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t addr) {
+    uint64_t desc = 0;
+    desc |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    desc |= (uint64_t)1 << 16;                     // leading byte offset 16 (unused: one swizzle atom along K)
+    desc |= (uint64_t)(512 >> 4) << 32;            // stride byte offset: 8 rows x 64 bytes
+    desc |= (uint64_t)1 << 46;
+    desc |= (uint64_t)4 << 61;                     // 64-byte swizzle
+    return desc;
+}
+
 // Instruction descriptor for kind::f16 with FP32 accumulation; A and B share
 // one format: 0 = F16, 1 = BF16 (kind::f16), 2 = TF32 (kind::tf32).
 constexpr uint32_t kFmtF16 = 0, kFmtBF16 = 1, kFmtTF32 = 2;
@@ -213,6 +225,14 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     return d;
 }
 // max of three (one instruction on sm_100)
+// 16-byte shared-memory store and load at a shared-window address.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, float& a, float& b, float& c, float& d) {
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(a), "=f"(b), "=f"(c), "=f"(d) : "r"(addr) : "memory");
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
