@@ -24,7 +24,7 @@ namespace spr {
 namespace kmtc {
 constexpr int BP = 128;                 // points per item (TMEM lanes)
 constexpr uint32_t kSpin = 1u << 20;
-enum { B_AF = 0, B_AE = 2, B_BF = 4, B_BE = 6, B_DF = 8, B_DE = 10, B_DR = 12, N_BAR = 13 };
+enum { B_AF = 0, B_AE = 2, B_BF = 4, B_DF = 6, B_DE = 8, B_DR = 10, N_BAR = 11 };
 constexpr int kKeepStride = 144;        // bytes per lane of the best-chunk copy (32 floats + 16: no bank conflicts)
 
 // Shared-memory plan for rank R and centre blocks of NB (every tile 1024-aligned):
@@ -140,6 +140,21 @@ __device__ __forceinline__ void pair_update(float (&v)[2][32], int cb0, int lim,
     st_shared_16_if(keep, up1, v[1]);
     st_shared_16_if(keep + 64, up1, v[1] + 16);
 }
+// The K steps of one centre block: D = A B^T over R/8 TF32 steps of 8, then
+// + ones x (hi, lo) for the -|c|^2/2 term.  Descriptors advance by the
+// 64-byte chunk stride (512 units for the points, cb for the centres) every
+// second step and by 32 bytes inside a chunk.
+template <int KS>
+__device__ __forceinline__ void mma_block(uint32_t d, uint64_t a0, uint64_t b0, uint32_t cb, uint64_t ones, uint64_t h,
+                                          uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+        const uint64_t oa = (uint64_t)((kk >> 1) * ((BP * 64) >> 4) + (kk & 1) * 2);
+        const uint64_t ob = (uint64_t)((kk >> 1) * cb + (kk & 1) * 2);
+        sm100::mma_tf32_ss(d, a0 + oa, b0 + ob, idesc, kk > 0 ? 1u : 0u);
+    }
+    sm100::mma_tf32_ss(d, ones, h, idesc, 1u);
+}
 }  // namespace kmtc
 
 // Persistent: block k handles items k, k + grid, ... where an item is 128
@@ -181,7 +196,6 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
             mbar_init(bar(B_AF + s), 1);
             mbar_init(bar(B_AE + s), 1);
             mbar_init(bar(B_BF + s), 1);
-            mbar_init(bar(B_BE + s), 1);
             mbar_init(bar(B_DF + s), 1);
             mbar_init(bar(B_DE + s), 256);
         }
@@ -223,7 +237,9 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                                 bh * N + p0);
                 for (int blk = 0; blk < nblk; ++blk, ++gb) {
                     const int stage = gb & 1;
-                    if (gb >= 2 && !mbar_wait(bar(B_BE + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
+                    // the stage is free once the products of block gb - 2 are done (the
+                    // commit that also hands their scores to the epilogue)
+                    if (gb >= 2 && !mbar_wait(bar(B_DF + stage), ((gb >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar(B_BF + stage), L.b_stage + NB * 32);
                     for (int ch = 0; ch < nchunk; ++ch)
                         tma_load_2d(s_base + L.oB + stage * L.b_stage + ch * NB * 64, &maps.cen, bar(B_BF + stage),
@@ -261,16 +277,13 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
                     tc_fence_after();
                     const uint64_t b0 = dB + (uint64_t)((stage * L.b_stage) >> 4);
                     const uint32_t d = tmem + stage * NB;
-                    for (int kk = 0; kk < ksteps; ++kk) {
-                        // K step kk: chunk kk / 2, 32 bytes further inside the 64-byte row for odd kk
-                        const uint64_t off = (uint64_t)(((kk >> 1) * BP * 64 + (kk & 1) * 32) >> 4);
-                        const uint64_t offb = (uint64_t)(((kk >> 1) * NB * 64 + (kk & 1) * 32) >> 4);
-                        mma_tf32_ss(d, a0 + off, b0 + offb, idesc, kk > 0 ? 1u : 0u);
+                    const uint64_t h0 = dH + (uint64_t)((stage * NB * 32) >> 4);
+                    switch (ksteps) {
+                        case 4: mma_block<4>(d, a0, b0, (uint32_t)((NB * 64) >> 4), dOnes, h0, idesc); break;
+                        case 6: mma_block<6>(d, a0, b0, (uint32_t)((NB * 64) >> 4), dOnes, h0, idesc); break;
+                        default: mma_block<8>(d, a0, b0, (uint32_t)((NB * 64) >> 4), dOnes, h0, idesc); break;
                     }
-                    // + 1 * hi + 1 * lo: the -|c|^2/2 term of every score
-                    mma_tf32_ss(d, dOnes, dH + (uint64_t)((stage * NB * 32) >> 4), idesc, 1u);
                     mma_commit(bar(B_DF + stage));
-                    mma_commit(bar(B_BE + stage));
                 }
                 mma_commit(bar(B_AE + ab));
                 ++li;
