@@ -278,15 +278,18 @@ constexpr int kRegs = 128;
 static_assert((kThreads / 32 + 3) / 4 * 32 * kRegs <= 16384, "registers per sub-partition");
 constexpr uint32_t kSpin = 1u << 20;
 enum { B_RF = 0, B_XF = NST, B_XE = 2 * NST, B_DF = 3 * NST, B_DE = 3 * NST + 2, B_AF = 3 * NST + 4,
-       B_AE = 3 * NST + 5, B_DR = 3 * NST + 6, B_SS = 3 * NST + 7, N_BAR = 3 * NST + 9 };
+       B_AE = 3 * NST + 5, B_DR = 3 * NST + 6, B_SS = 3 * NST + 7, B_OF = 3 * NST + 9, B_OE = 3 * NST + 11,
+       N_BAR = 3 * NST + 13 };
 constexpr int CHB = BM * 128;                 // one chunk: 128 rows x 32 fp32
 constexpr int oHi = 0;                        // NST chunks: raw O^sp, then Xbar hi in place
 constexpr int oLo = oHi + NST * CHB;          // NST chunks: Xbar lo
 constexpr int oStat = oLo + NST * CHB;        // 2 x (mu_X, 1 / sigma) of the last two heads (transform warps)
-constexpr int oBar = oStat + 2 * 2 * D * 4;
+constexpr int oOut = oStat + 2 * 2 * D * 4;    // 2 row halves x 64 rows x 128 fp32: the restored rows
+constexpr int oBar = oOut + 2 * 64 * D * 4;
 constexpr int oMisc = oBar + N_BAR * 8;
 constexpr int kSmem = oMisc + 16 + 1024;
-static_assert(oLo % 1024 == 0 && oStat % 16 == 0, "alignment");
+static_assert(oLo % 1024 == 0 && oStat % 16 == 0 && oOut % 16 == 0, "alignment");
+static_assert(kSmem <= 232448, "shared memory");
 }  // namespace aptt
 
 __global__ void __maxnreg__(aptt::kRegs) apply_t_kernel(
@@ -323,6 +326,10 @@ __global__ void __maxnreg__(aptt::kRegs) apply_t_kernel(
         mbar_init(bar(B_DR), 1);
         mbar_init(bar(B_SS), 128);
         mbar_init(bar(B_SS + 1), 128);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(bar(B_OF + h), 4);   // the four channel warps of a row half staged their columns
+            mbar_init(bar(B_OE + h), 4);   // ... and wrote their rows out
+        }
         fence_barrier_init();
         misc[1] = 0;
     }
@@ -463,19 +470,21 @@ __global__ void __maxnreg__(aptt::kRegs) apply_t_kernel(
         const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
         bool ok = true;
         int heads = 0, cur_bh = -1, i = 0;
-        float bias = 0.f;
-        // row indices of a tile (probe slot, destination row) for this half of
-        // its rows: lane l holds rows 64 hrow + l and + 32; loaded one tile ahead
-        auto load_rows = [&](int w, int& sl0, int& sl1, int& dq0, int& dq1) {
-            const int bhw = w / tiles_per_head, r0 = (w % tiles_per_head) * BM + 64 * hrow + lane, r1 = r0 + 32;
+        float4 bias4 = make_float4(0.f, 0.f, 0.f, 0.f);   // mu_X + mu_R of channels 4 lane .. 4 lane + 3
+        // The four channel warps of a row half stage their 32 channels of its 64
+        // rows in shared memory; then each writes 16 whole rows (512 bytes, one
+        // 16-byte vector per lane) to their restored positions.  Row indices
+        // (probe slot, destination) of this warp's 16 rows: lane l holds row
+        // 16 q + (l & 15) of the half; loaded one tile ahead.
+        float* out_s = reinterpret_cast<float*>(sm + oOut) + hrow * 64 * D;
+        auto load_rows = [&](int w, int& sl, int& dq) {
+            const int bhw = w / tiles_per_head, r = (w % tiles_per_head) * BM + 64 * hrow + 16 * q + (lane & 15);
             const size_t hb = (size_t)bhw * N;
-            sl0 = r0 < N ? pslot[hb + r0] : -2;
-            sl1 = r1 < N ? pslot[hb + r1] : -2;
-            dq0 = r0 < N ? perm_q[hb + r0] : 0;
-            dq1 = r1 < N ? perm_q[hb + r1] : 0;
+            sl = r < N ? pslot[hb + r] : -2;
+            dq = r < N ? perm_q[hb + r] : 0;
         };
-        int nsl0 = -2, nsl1 = -2, ndq0 = 0, ndq1 = 0;
-        if (w_begin < w_end) load_rows(w_begin, nsl0, nsl1, ndq0, ndq1);
+        int nsl = -2, ndq = 0;
+        if (w_begin < w_end) load_rows(w_begin, nsl, ndq);
         for (int w = w_begin; ok && w < w_end; ++w, ++i) {
             const int bh = w / tiles_per_head;
             if (bh != cur_bh) {
@@ -503,14 +512,16 @@ __global__ void __maxnreg__(aptt::kRegs) apply_t_kernel(
                 }
                 tc_fence_before();
                 mbar_arrive(bar(B_AF));
-                bias = mu_x[(size_t)bh * D + n] + mu_r[(size_t)bh * D + n];
+                const float4 mx = reinterpret_cast<const float4*>(mu_x + (size_t)bh * D)[lane];
+                const float4 mr = reinterpret_cast<const float4*>(mu_r + (size_t)bh * D)[lane];
+                bias4 = make_float4(mx.x + mr.x, mx.y + mr.y, mx.z + mr.z, mx.w + mr.w);
                 cur_bh = bh;
                 ++heads;
             }
             const int d = i & 1;
             const size_t hb = (size_t)bh * N;
-            const int sl0 = nsl0, sl1 = nsl1, dq0 = ndq0, dq1 = ndq1;
-            if (w + 1 < w_end) load_rows(w + 1, nsl0, nsl1, ndq0, ndq1);
+            const int sl = nsl, dq = ndq;
+            if (w + 1 < w_end) load_rows(w + 1, nsl, ndq);
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DF + d), (i >> 1) & 1, abort_flag, kSpin));
             if (!ok) break;
             tc_fence_after();
@@ -521,18 +532,38 @@ __global__ void __maxnreg__(aptt::kRegs) apply_t_kernel(
             tmem_wait_ld(v[1]);
             tc_fence_before();
             mbar_arrive(bar(B_DE + d));   // the accumulator is free for tile i + 2
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int sl = h ? sl1 : sl0, dq = h ? dq1 : dq0;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int slot = __shfl_sync(0xffffffffu, sl, j);   // uniform: the warp writes one row
-                    const int dst = __shfl_sync(0xffffffffu, dq, j);
-                    if (slot == -2) continue;                            // past the head's last row
-                    float* orow = O_out + (hb + dst) * D;
-                    orow[n] = slot < 0 ? v[h][j] + bias : probe_dense[((size_t)bh * Mp + slot) * D + n];
-                }
+            // the staging half is free once its rows of the previous tile are written out
+            if (i >= 1) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OE + hrow), (i - 1) & 1, abort_flag, kSpin));
+                if (!ok) break;
             }
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int j = 0; j < 32; ++j) out_s[(32 * h + j) * D + n] = v[h][j];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_OF + hrow));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF + hrow), i & 1, abort_flag, kSpin));
+            if (!ok) break;
+#pragma unroll 4
+            for (int r = 0; r < 16; ++r) {
+                const int slot = __shfl_sync(0xffffffffu, sl, r);   // uniform: the warp writes one row
+                const int dst = __shfl_sync(0xffffffffu, dq, r);
+                if (slot == -2) continue;                            // past the head's last row
+                float4 x;
+                if (slot < 0) {
+                    x = reinterpret_cast<const float4*>(out_s + (16 * q + r) * D)[lane];
+                    x.x += bias4.x;
+                    x.y += bias4.y;
+                    x.z += bias4.z;
+                    x.w += bias4.w;
+                } else {
+                    x = reinterpret_cast<const float4*>(probe_dense + ((size_t)bh * Mp + slot) * D)[lane];
+                }
+                reinterpret_cast<float4*>(O_out + (hb + dst) * D)[lane] = x;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_OE + hrow));
         }
         if (!ok) {
             record_status(status, SPARSEPR_TIMEOUT, 76);
