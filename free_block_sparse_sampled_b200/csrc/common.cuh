@@ -13,7 +13,7 @@ namespace spr {
 
 constexpr int kMaxGroups = 2048;   // C_q, C_k upper limit (one sort of 2048 keys per block)
 constexpr int kMaxRank = 64;       // r_K, r_Q upper limit (register-resident coordinates)
-constexpr int kSortTile = 256;     // points per histogram/scatter tile of the group sort
+constexpr int kSortTile = 1024;    // points per histogram/scatter tile of the group sort
 constexpr int kMaxN = (1 << 20) - 1;
 
 // Device status word (first 256 bytes of the workspace).  The first failure

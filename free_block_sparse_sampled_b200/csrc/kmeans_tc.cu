@@ -83,26 +83,18 @@ __device__ __forceinline__ float max32(const float (&s)[32]) {
                  fmaxf(m3[9], m3[10]));
 }
 
-// Stores 16 scores at a shared-window address when p holds (predicated, no branch).
-__device__ __forceinline__ void st_shared_16_if(uint32_t a, bool p, const float* s) {
-    asm volatile(
-        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
-        "@q st.shared.v4.f32 [%0], {%2, %3, %4, %5};\n\t"
-        "@q st.shared.v4.f32 [%0+16], {%6, %7, %8, %9};\n\t"
-        "@q st.shared.v4.f32 [%0+32], {%10, %11, %12, %13};\n\t"
-        "@q st.shared.v4.f32 [%0+48], {%14, %15, %16, %17};\n\t}" ::"r"(a),
-        "r"((int)p), "f"(s[0]), "f"(s[1]), "f"(s[2]), "f"(s[3]), "f"(s[4]), "f"(s[5]), "f"(s[6]), "f"(s[7]),
-        "f"(s[8]), "f"(s[9]), "f"(s[10]), "f"(s[11]), "f"(s[12]), "f"(s[13]), "f"(s[14]), "f"(s[15])
-        : "memory");
+// Stores a chunk of 32 scores at a shared-window address.
+__device__ __forceinline__ void st_chunk(uint32_t a, const float (&v)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sm100::st_shared_v4(a + 16 * j, v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
 // One 64-column pair of an epilogue lane: the chunks of 32 scores at columns
 // cb0 and cb0 + 32, of which the columns below lim take part.  MODE 0: both
 // chunks whole; 1: the first whole and the second past lim; 2: columns at or
 // past lim masked to -inf.  Both chunk maxima are taken before either updates
-// the running first maximum (best, the base column bcb of its chunk), and the
-// lane's copy of its best chunk at `keep` is rewritten by predicated stores,
-// so a pair is one branch-free stretch of code.
+// the running first maximum (best, the base column bcb of its chunk); a lane
+// whose maximum moved then rewrites its copy of the best chunk at `keep`.
 template <int MODE, bool DBG>
 __device__ __forceinline__ void pair_update(float (&v)[2][32], int cb0, int lim, float& best, int& bcb, uint32_t keep,
                                             float* dbg_row) {
@@ -124,8 +116,7 @@ __device__ __forceinline__ void pair_update(float (&v)[2][32], int cb0, int lim,
         const bool up0 = m0 > best;   // a later chunk only wins with a strictly larger score
         best = up0 ? m0 : best;
         bcb = up0 ? cb0 : bcb;
-        st_shared_16_if(keep, up0, v[0]);
-        st_shared_16_if(keep + 64, up0, v[0] + 16);
+        if (up0) st_chunk(keep, v[0]);
         return;
     }
     const float m1 = max32(v[1]);
@@ -134,11 +125,10 @@ __device__ __forceinline__ void pair_update(float (&v)[2][32], int cb0, int lim,
     const bool up1 = m1 > b0;
     best = up1 ? m1 : b0;
     bcb = up1 ? cb0 + 32 : (up0 ? cb0 : bcb);
-    const bool s0 = up0 && !up1;
-    st_shared_16_if(keep, s0, v[0]);
-    st_shared_16_if(keep + 64, s0, v[0] + 16);
-    st_shared_16_if(keep, up1, v[1]);
-    st_shared_16_if(keep + 64, up1, v[1] + 16);
+    // divergent branches after both maxima: only the lanes that move store
+    // (predicated stores cost shared-memory bandwidth for every lane)
+    if (up1) st_chunk(keep, v[1]);
+    else if (up0) st_chunk(keep, v[0]);
 }
 // The K steps of one centre block: D = A B^T over R/8 TF32 steps of 8, then
 // + ones x (hi, lo) for the -|c|^2/2 term.  Descriptors advance by the
@@ -315,10 +305,10 @@ __global__ void __launch_bounds__(320, 1) kmeans_assign_tc_kernel(
             const int old_label = (valid && !first) ? labels[(size_t)bh * N + p] : 0;
             // running first maximum over this half's columns, in column order: the
             // best value, the base column of the chunk holding it and, in shared
-            // memory, a copy of that chunk's scores (eight predicated vector
-            // stores instead of a per-chunk index search, which every chunk would
-            // run: some lane of the warp almost always improves); the index is
-            // searched once per item
+            // memory, a copy of that chunk's scores (eight vector stores by the
+            // lanes that move, instead of a per-chunk index search, which every
+            // chunk would run: some lane of the warp almost always improves); the
+            // index is searched once per item
             float best = -INFINITY;
             int bcb = 0;
             float* dbg_row = (DBG && valid) ? dbg_scores + ((size_t)bh * N + p) * C : nullptr;

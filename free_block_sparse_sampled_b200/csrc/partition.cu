@@ -457,39 +457,49 @@ __global__ void __launch_bounds__(1024) label_offsets_kernel(int32_t* __restrict
 }
 
 // Scatter of one tile's points to their sorted positions: the label's group
-// offset + the counts of earlier tiles + the rank among equal labels of
-// lower index in this tile (warps in order), so the sort is stable.
-__global__ void __launch_bounds__(1024) label_scatter_kernel(const int32_t* __restrict__ labels, int N,
-                                                             int C, int n_tiles,
-                                                             const int32_t* __restrict__ hist,
-                                                             const int32_t* __restrict__ offs,
-                                                             int32_t* __restrict__ sorted,
-                                                             const int32_t* __restrict__ ctl) {
+// offset + the counts of earlier tiles + the rank among equal labels of lower
+// index in this tile, so the sort is stable.  The in-tile rank is the count in
+// earlier warps (a per-label scan over the warps of per-warp counts, uint16
+// table [warp][label] in dynamic shared memory) plus the rank among lower lanes
+// of the same warp; three block barriers per tile.
+__global__ void __launch_bounds__(kSortTile) label_scatter_kernel(const int32_t* __restrict__ labels, int N,
+                                                                  int C, int n_tiles,
+                                                                  const int32_t* __restrict__ hist,
+                                                                  const int32_t* __restrict__ offs,
+                                                                  int32_t* __restrict__ sorted,
+                                                                  const int32_t* __restrict__ ctl) {
+    constexpr int W = kSortTile / 32;
     const int bh = blockIdx.y, tile = blockIdx.x;
     if (ctl != nullptr && ctl[bh * kCtlStride + kCtlDone]) return;
-    __shared__ int cnt[kMaxGroups];
+    extern __shared__ int32_t sort_smem[];
+    int32_t* cnt = sort_smem;                                          // [C]: group offset + earlier tiles
+    uint16_t* wc = reinterpret_cast<uint16_t*>(sort_smem + C);         // [W][C]: per-warp counts, then prefix
     const int32_t* base = hist + ((size_t)bh * n_tiles + tile) * C;
     const int32_t* go = offs + (size_t)bh * (C + 1);
-    for (int c = threadIdx.x; c < C; c += blockDim.x) cnt[c] = base[c] + go[c];
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        cnt[c] = base[c] + go[c];
+#pragma unroll
+        for (int w = 0; w < W; ++w) wc[w * C + c] = 0;
+    }
     __syncthreads();
     const int i = tile * kSortTile + threadIdx.x;
     const int lab = (i < N) ? labels[(size_t)bh * N + i] : -1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-        if (warp == w) {
-            const unsigned m = __match_any_sync(0xffffffffu, lab);
-            const int leader = __ffs(m) - 1;
-            const int rank = __popc(m & ((1u << lane) - 1u));
-            int start = 0;
-            if (lane == leader && lab >= 0) {
-                start = cnt[lab];
-                cnt[lab] = start + __popc(m);
-            }
-            start = __shfl_sync(0xffffffffu, start, leader);
-            if (lab >= 0) sorted[(size_t)bh * N + start + rank] = i;
+    const unsigned m = __match_any_sync(0xffffffffu, lab);
+    const int rank = __popc(m & ((1u << lane) - 1u));
+    if (lab >= 0 && lane == __ffs(m) - 1) wc[warp * C + lab] = (uint16_t)__popc(m);
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {   // exclusive scan over the warps, per label
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+            const int v = wc[w * C + c];
+            wc[w * C + c] = (uint16_t)run;
+            run += v;
         }
-        __syncthreads();
     }
+    __syncthreads();
+    if (lab >= 0) sorted[(size_t)bh * N + cnt[lab] + wc[warp * C + lab] + rank] = i;
 }
 
 // Centre update: member mean, rounded to TF32; empty centres keep their
@@ -750,6 +760,14 @@ void launch_jacobi_factor(const float* A, float* F, int Rp, int r, int BH, int d
 
 namespace {
 
+// Dynamic shared memory of label_scatter_kernel for C labels: the offsets
+// (int32) and the per-warp counts (uint16).
+size_t scatter_smem(int C) {
+    const size_t bytes = (size_t)C * (4 + 2 * (kSortTile / 32));
+    cudaFuncSetAttribute(label_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    return bytes;
+}
+
 inline int grid_for(size_t total, int threads) {
     size_t g = (total + threads - 1) / threads;
     return (int)(g > 148 * 64 ? 148 * 64 : (g == 0 ? 1 : g));
@@ -778,8 +796,8 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
             count_launch(), label_hist_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, ctl);
             count_launch(), label_colscan_kernel<<<cgrid, 256, 0, st>>>(hist, C, pl.n_sort_tiles, offs, ctl);
             count_launch(), label_offsets_kernel<<<BH, 1024, 0, st>>>(offs, N, C, ctl);
-            count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, offs,
-                                                                              sorted, ctl);
+            count_launch(), label_scatter_kernel<<<tgrid, kSortTile, scatter_smem(C), st>>>(raw, N, C, pl.n_sort_tiles,
+                                                                                             hist, offs, sorted, ctl);
             count_launch(), centre_update_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, sorted, offs, N, C, cen, hn, ctl);
         }
         if (!launch_kmeans_assign_tc(phi, cen, hn, at<float>(ws, pl.o_hs), BH, N, C, R, raw, ctl, first, dbg_scores, dbg_hist,
@@ -831,8 +849,8 @@ void finalize_groups(const Plan& pl, void* ws, int C, int which, int32_t* label_
     count_launch(), label_colscan_kernel<<<dim3((C + 255) / 256, BH), 256, 0, st>>>(hist, C, pl.n_sort_tiles, offs,
                                                                                    nullptr);
     count_launch(), label_offsets_kernel<<<BH, 1024, 0, st>>>(offs, N, C, nullptr);
-    count_launch(), label_scatter_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, offs, sorted,
-                                                                      nullptr);
+    count_launch(), label_scatter_kernel<<<tgrid, kSortTile, scatter_smem(C), st>>>(raw, N, C, pl.n_sort_tiles, hist,
+                                                                                     offs, sorted, nullptr);
     count_launch(), compact_groups_kernel<<<BH, 1024, 0, st>>>(offs, C, N, newid, offs_out, ng, which);
     count_launch(), relabel_kernel<<<grid_for((size_t)BH * N, 256), 256, 0, st>>>(raw, newid, sorted, BH, N, C,
                                                                   label_out, perm_out, pos_out);
