@@ -94,6 +94,13 @@ bool make_plan(const sparsepr_params& p, Plan& pl) {
     pl.o_pbits = bump(c, BH * ((N + 31) / 32) * 4);
     pl.o_S = bump(c, p.residual_rank > 0 ? BH * d * d * 8 : 256);
     pl.o_rawkv = bump(c, pl.G > 1 ? BH / pl.G * N * 4 : 256);
+    {
+        const size_t Rmax = pl.RKp > pl.RQp ? pl.RKp : pl.RQp;
+        pl.o_csum = bump(c, BH * Cm * Rmax * 8);
+        pl.o_ccnt = bump(c, BH * Cm * 4);
+        pl.o_prev = bump(c, BH * N * 4);
+        pl.o_cscale = bump(c, BH * 4);
+    }
     // outputs owned by the workspace (fused call)
     pl.o_Qp = bump(c, BH * N * d * es);
     pl.o_Kp = bump(c, BHk * N * d * es);

@@ -113,7 +113,11 @@ struct Plan {
         o_warm,   // [0]: kWarmMagic when the fused call's state is complete; [1 + bh], [1 + BH + bh]: cold K / Q factor
         o_pbits,  // [BH][ceil(N/32)] probe membership bits (random / uniform probes)
         o_S,      // [BH][d][d] fp64 Rbar^T W Rbar (rank truncation)
-        o_rawkv;  // [BH/G][N] K/V k-means labels per K/V head (GQA)
+        o_rawkv,  // [BH/G][N] K/V k-means labels per K/V head (GQA)
+        o_csum,   // [BH][Cmax][Rmax] int64 member sums of the k-means centres (fixed point)
+        o_ccnt,   // [BH][Cmax] member counts
+        o_prev,   // [BH][N] the labels the sums hold
+        o_cscale; // [BH] fixed-point exponent of each head's coordinates
     // outputs owned by the workspace for sparsepr_call
     size_t o_Qp, o_Kp, o_Vp, o_qlab, o_kvlab, o_permq, o_permk, o_posq, o_qoff, o_kvoff, o_ng, o_its,
         o_qcen, o_kcen, o_vcen, o_qdist, o_score, o_mask, o_selc, o_selg, o_pairs, o_pidx, o_pgrp,

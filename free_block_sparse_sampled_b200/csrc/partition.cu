@@ -502,78 +502,129 @@ __global__ void __launch_bounds__(kSortTile) label_scatter_kernel(const int32_t*
     if (lab >= 0) sorted[(size_t)bh * N + cnt[lab] + wc[warp * C + lab] + rank] = i;
 }
 
-// Centre update: member mean, rounded to TF32; empty centres keep their
-// value.  One warp per centre: a member row is read as R/4 float4 lanes, so
-// one warp load covers 32/(R/4) rows (lanes past that stay idle for R = 48).
-// Rows are assigned to (load, row slot) by their position in the sorted
-// member list and the partial sums are combined in a fixed order, so the
-// result depends only on the labels.
+// ---- exact member sums for the centre updates
+// Coordinates of head bh are taken as the integers q = rint(phi * 2^S_bh),
+// with S_bh chosen so that a sum of N of them stays below 2^62 in magnitude.
+// Integer sums are exact: they do not depend on the order of the members, so
+// after the first update only the points whose label changed move their q
+// from one centre's sum to the other's.  A centre is the member mean
+// (sum * 2^-S / count in fp64, rounded to fp32 and then TF32); empty centres
+// keep their value.
+
+// S_bh = 62 - (bits of max |phi|) - (bits of N).
+__global__ void coord_scale_kernel(const float* __restrict__ phi, int N, int R, int32_t* __restrict__ S_out) {
+    const int bh = blockIdx.x;
+    const float* ph = phi + (size_t)bh * N * R;
+    float m = 0.f;
+    for (size_t e = threadIdx.x; e < (size_t)N * R; e += blockDim.x) m = fmaxf(m, fabsf(ph[e]));
+    m = warp_max(m);
+    __shared__ float red[32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+        m = fmaxf(m, red[0]);
+        const int eb = m > 0.f ? ilogbf(m) + 1 : 0;   // max |phi| < 2^eb
+        const int nb = 32 - __clz(N);                   // N < 2^nb
+        S_out[bh] = 62 - eb - nb;
+    }
+}
+
+__device__ __forceinline__ long long fixed_coord(float x, int S) { return __double2ll_rn(scalbn((double)x, S)); }
+
+// First update of a run: the member sums and counts from the sorted member
+// lists (one warp per centre; lane k holds coordinates k, k + 32, ...).
 template <int R>
-__global__ void centre_update_kernel(const float* __restrict__ phi, const int32_t* __restrict__ sorted,
-                                     const int32_t* __restrict__ offs, int N, int C,
-                                     float* __restrict__ cen, float* __restrict__ hn,
-                                     const int32_t* __restrict__ ctl) {
-    static_assert(R % 16 == 0 && R >= 16 && R <= 128, "coordinate rows of 16..128 floats");
-    constexpr int LPR = R / 4;        // lanes per row
-    constexpr int RPL = 32 / LPR;     // rows per warp load
-    constexpr int LOADS = 32 / RPL;   // loads per 32 listed members
-    constexpr int U = 4;              // independent accumulators per lane
+__global__ void centre_sums_kernel(const float* __restrict__ phi, const int32_t* __restrict__ sorted,
+                                   const int32_t* __restrict__ offs, const int32_t* __restrict__ S_in, int N, int C,
+                                   long long* __restrict__ csum, int32_t* __restrict__ ccnt,
+                                   const int32_t* __restrict__ ctl) {
+    constexpr int KPL = (R + 31) / 32;   // coordinates per lane
     const int bh = blockIdx.y, lane = threadIdx.x & 31;
     if (ctl[bh * kCtlStride + kCtlDone]) return;
     const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (c >= C) return;
     const int s = offs[(size_t)bh * (C + 1) + c], e = offs[(size_t)bh * (C + 1) + c + 1];
-    if (e == s) return;
-    const int slot = lane / LPR, part = lane % LPR;
-    const bool active = slot < RPL;
-    float4 acc[U];
+    const int S = S_in[bh];
+    long long acc[KPL];
 #pragma unroll
-    for (int k = 0; k < U; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* ph = reinterpret_cast<const float4*>(phi + (size_t)bh * N * R) + part;
+    for (int k = 0; k < KPL; ++k) acc[k] = 0;
+    const float* ph = phi + (size_t)bh * N * R;
     const int32_t* so = sorted + (size_t)bh * N;
     for (int p0 = s; p0 < e; p0 += 32) {
-        const int my = (p0 + lane < e) ? so[p0 + lane] : 0;   // 32 member indices per load
+        const int my = (p0 + lane < e) ? so[p0 + lane] : 0;
         const int n = min(32, e - p0);
+#pragma unroll 4
+        for (int q = 0; q < n; ++q) {
+            const int row = __shfl_sync(0xffffffffu, my, q);
 #pragma unroll
-        for (int k = 0; k < LOADS; ++k) {
-            const int q = RPL * k + slot;
-            const int row = __shfl_sync(0xffffffffu, my, q & 31);
-            if (active && q < n) {
-                const float4 x = ph[(size_t)row * LPR];
-                float4& a = acc[k % U];
-                a.x += x.x;
-                a.y += x.y;
-                a.z += x.z;
-                a.w += x.w;
-            }
+            for (int k = 0; k < KPL; ++k)
+                if (32 * k + lane < R) acc[k] += fixed_coord(ph[(size_t)row * R + 32 * k + lane], S);
         }
     }
-    float4 t = acc[0];
+    long long* cs = csum + ((size_t)bh * C + c) * R;
 #pragma unroll
-    for (int k = 1; k < U; ++k) {
-        t.x += acc[k].x;
-        t.y += acc[k].y;
-        t.z += acc[k].z;
-        t.w += acc[k].w;
+    for (int k = 0; k < KPL; ++k)
+        if (32 * k + lane < R) cs[32 * k + lane] = acc[k];
+    if (lane == 0) ccnt[(size_t)bh * C + c] = e - s;
+}
+
+// Later updates: every point whose label differs from the one its sums hold
+// (prev) moves its coordinates from the old centre's sum to the new one's.
+// One warp per 32 points; the warp takes the moving points one at a time,
+// a lane per coordinate.
+__global__ void centre_delta_kernel(const float* __restrict__ phi, const int32_t* __restrict__ labels,
+                                    int32_t* __restrict__ prev, const int32_t* __restrict__ S_in, int N, int C, int R,
+                                    long long* __restrict__ csum, int32_t* __restrict__ ccnt,
+                                    const int32_t* __restrict__ ctl) {
+    const int bh = blockIdx.y, lane = threadIdx.x & 31;
+    if (ctl[bh * kCtlStride + kCtlDone]) return;
+    const int p0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32;
+    if (p0 >= N) return;
+    const int p = p0 + lane;
+    const size_t hb = (size_t)bh * N;
+    const int nw = p < N ? labels[hb + p] : 0, od = p < N ? prev[hb + p] : 0;
+    const bool mv = p < N && nw != od;
+    unsigned moving = __ballot_sync(0xffffffffu, mv);
+    if (moving == 0u) return;
+    if (mv) {
+        prev[hb + p] = nw;
+        atomicAdd(&ccnt[(size_t)bh * C + nw], 1);
+        atomicSub(&ccnt[(size_t)bh * C + od], 1);
     }
-    // row slots -> slot 0 (lane = slot * LPR + part), fixed tree order
-#pragma unroll
-    for (int o = LPR; o < RPL * LPR; o <<= 1) {
-        t.x += __shfl_down_sync(0xffffffffu, t.x, o);
-        t.y += __shfl_down_sync(0xffffffffu, t.y, o);
-        t.z += __shfl_down_sync(0xffffffffu, t.z, o);
-        t.w += __shfl_down_sync(0xffffffffu, t.w, o);
+    const int S = S_in[bh];
+    const float* ph = phi + hb * R;
+    unsigned long long* cs = reinterpret_cast<unsigned long long*>(csum) + (size_t)bh * C * R;
+    while (moving != 0u) {
+        const int j = __ffs(moving) - 1;
+        moving &= moving - 1u;
+        const int n = __shfl_sync(0xffffffffu, nw, j), o = __shfl_sync(0xffffffffu, od, j);
+        for (int k = lane; k < R; k += 32) {
+            const long long q = fixed_coord(ph[(size_t)(p0 + j) * R + k], S);
+            atomicAdd(&cs[(size_t)n * R + k], (unsigned long long)q);
+            atomicAdd(&cs[(size_t)o * R + k], (unsigned long long)(-q));
+        }
     }
-    const float count = (float)(e - s);
+}
+
+// Centres (and -|c|^2/2 halves, hn = |c|^2 / 2) from the sums; one warp per centre.
+__global__ void centre_from_sums_kernel(const long long* __restrict__ csum, const int32_t* __restrict__ ccnt,
+                                        const int32_t* __restrict__ S_in, int C, int R, float* __restrict__ cen,
+                                        float* __restrict__ hn, const int32_t* __restrict__ ctl) {
+    const int bh = blockIdx.y, lane = threadIdx.x & 31;
+    if (ctl[bh * kCtlStride + kCtlDone]) return;
+    const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (c >= C) return;
+    const int cnt = ccnt[(size_t)bh * C + c];
+    if (cnt <= 0) return;   // empty: keeps its value
+    const int S = S_in[bh];
+    const long long* cs = csum + ((size_t)bh * C + c) * R;
+    float* cc = cen + ((size_t)bh * C + c) * R;
     float ss = 0.f;
-    if (lane < LPR) {
-        float4 m;
-        m.x = tf32_round(t.x / count);
-        m.y = tf32_round(t.y / count);
-        m.z = tf32_round(t.z / count);
-        m.w = tf32_round(t.w / count);
-        reinterpret_cast<float4*>(cen + ((size_t)bh * C + c) * R)[part] = m;
-        ss = fmaf(m.x, m.x, fmaf(m.y, m.y, fmaf(m.z, m.z, m.w * m.w)));
+    for (int k = lane; k < R; k += 32) {
+        const float m = tf32_round((float)(scalbn((double)cs[k], -S) / (double)cnt));
+        cc[k] = m;
+        ss = fmaf(m, m, ss);
     }
     ss = warp_sum(ss);
     if (lane == 0) hn[(size_t)bh * C + c] = 0.5f * ss;
@@ -789,16 +840,27 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
     else
         count_launch(), kmeans_init_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, N, C, p.seed, stage, cen, hn);
     const dim3 agrid((N + 127) / 128, BH);
-    const dim3 tgrid(pl.n_sort_tiles, BH), cgrid((C + 255) / 256, BH);
+    const dim3 tgrid(pl.n_sort_tiles, BH), cgrid((C + 255) / 256, BH), wgrid((C + 7) / 8, BH);
+    long long* csum = at<long long>(ws, pl.o_csum);
+    int32_t* ccnt = at<int32_t>(ws, pl.o_ccnt);
+    int32_t* prev = at<int32_t>(ws, pl.o_prev);
+    int32_t* cscale = at<int32_t>(ws, pl.o_cscale);
+    if (p.kmeans_iters > 1) count_launch(), coord_scale_kernel<<<BH, 1024, 0, st>>>(phi, N, R, cscale);
     for (int it = 0; it < p.kmeans_iters; ++it) {
         const int first = it == 0;
-        if (!first) {
+        if (it == 1) {   // first update: sums and counts from the sorted member lists
             count_launch(), label_hist_kernel<<<tgrid, kSortTile, 0, st>>>(raw, N, C, pl.n_sort_tiles, hist, ctl);
             count_launch(), label_colscan_kernel<<<cgrid, 256, 0, st>>>(hist, C, pl.n_sort_tiles, offs, ctl);
             count_launch(), label_offsets_kernel<<<BH, 1024, 0, st>>>(offs, N, C, ctl);
             count_launch(), label_scatter_kernel<<<tgrid, kSortTile, scatter_smem(C), st>>>(raw, N, C, pl.n_sort_tiles,
                                                                                              hist, offs, sorted, ctl);
-            count_launch(), centre_update_kernel<R><<<dim3((C + 7) / 8, BH), 256, 0, st>>>(phi, sorted, offs, N, C, cen, hn, ctl);
+            count_launch(), centre_sums_kernel<R><<<wgrid, 256, 0, st>>>(phi, sorted, offs, cscale, N, C, csum, ccnt, ctl);
+            cudaMemcpyAsync(prev, raw, (size_t)BH * N * sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+            count_launch(), centre_from_sums_kernel<<<wgrid, 256, 0, st>>>(csum, ccnt, cscale, C, R, cen, hn, ctl);
+        } else if (it > 1) {   // later updates: only the points whose label changed
+            count_launch(), centre_delta_kernel<<<dim3((N + 255) / 256, BH), 256, 0, st>>>(phi, raw, prev, cscale, N, C,
+                                                                                          R, csum, ccnt, ctl);
+            count_launch(), centre_from_sums_kernel<<<wgrid, 256, 0, st>>>(csum, ccnt, cscale, C, R, cen, hn, ctl);
         }
         if (!launch_kmeans_assign_tc(phi, cen, hn, at<float>(ws, pl.o_hs), BH, N, C, R, raw, ctl, first, dbg_scores, dbg_hist,
                                      p.kmeans_iters, at<DevStatus>(ws, pl.o_status), st))
