@@ -238,9 +238,9 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
                 float v[32];
                 tmem_ld32(t_row + stage * BK + c4 * 32, v);
                 tmem_wait_ld(v);
+                const int nv = ncol - c4 * 32;   // valid columns of the chunk (uniform)
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (c4 * 32 + i < ncol) m4[i & 3] = fmaxf(m4[i & 3], v[i] * cs);
+                for (int i = 0; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], i < nv ? v[i] * cs : -INFINITY);
             }
             const float Mn = fmaxf(Mr, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
             if (Mn > Mr) {
@@ -254,27 +254,37 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
             const float* meta = reinterpret_cast<const float*>(sm + L::oMeta + ring * L::META);
             const uint32_t* endm = reinterpret_cast<const uint32_t*>(meta + 2 * BK);
             // pass 2, one 32-key chunk at a time (a rolled loop keeps the code small):
-            // segment sums, flushed at every key-group end
+            // the chunk's exponentials first (all independent), then the segment
+            // sums in key order, flushed at every key-group end.  Columns past the
+            // tile's keys give e = 0 and carry no group end, so no test branches.
+            const size_t row_idx = ((size_t)bh * Cq + a) * Ck;
+            const float m_nat = Mr * 0.6931471805599453f;   // back to natural-log units
 #pragma unroll 1
             for (int c4 = 0; c4 < BK / 32; ++c4) {
                 float v[32];
                 tmem_ld32(t_row + stage * BK + c4 * 32, v);
                 tmem_wait_ld(v);
-                const uint32_t em = endm[c4];
-                const float* u = meta + c4 * 32;
-                const float* wv = meta + BK + c4 * 32;
+                const int nv = ncol - c4 * 32;
+                const uint32_t em = endm[c4];   // group ends at these keys (same for every row)
+                const float4* u4 = reinterpret_cast<const float4*>(meta + c4 * 32);
+                const float4* w4 = reinterpret_cast<const float4*>(meta + BK + c4 * 32);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    if (c4 * 32 + i < ncol) {
-                        const float e = ex2_approx(fmaf(v[i], cs, -Mr));
-                        t1 = fmaf(e, u[i], t1);
-                        t2 = fmaf(e * e, wv[i], t2);
-                        if (em & (1u << i)) {   // group b ends at this key (same for every row)
+                for (int i = 0; i < 32; ++i) v[i] = i < nv ? ex2_approx(fmaf(v[i], cs, -Mr)) : 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 uq = u4[q], wq = w4[q];
+                    const float uu[4] = {uq.x, uq.y, uq.z, uq.w}, ww[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int i = 4 * q + k;
+                        const float e = v[i];
+                        t1 = fmaf(e, uu[k], t1);
+                        t2 = fmaf(e * e, ww[k], t2);
+                        if ((em >> i) & 1u) {   // uniform: group b ends at this key
                             if (a < Cqp) {
-                                const size_t idx = ((size_t)bh * Cq + a) * Ck + b;
-                                mloc[idx] = Mr * 0.6931471805599453f;   // back to natural-log units
-                                t1o[idx] = t1;
-                                t2o[idx] = t2;
+                                mloc[row_idx + b] = m_nat;
+                                t1o[row_idx + b] = t1;
+                                t2o[row_idx + b] = t2;
                             }
                             ++b;
                             t1 = 0.f;
