@@ -149,6 +149,10 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
                     tma_load_2d(s_base + L::oA + pc * L::AB + hh * BA * 128, &maps.a, bar(B_A), hh * 64,
                                 (bh * 3 + pc) * CqPad + at * BA);
         }
+        // the block's key-group ends, two per lane (GPB = 64), read once
+        static_assert(GPB == 64, "two group ends per lane");
+        const int ge0 = (g0 + lane < g1) ? ko[g0 + lane + 1] : -1;
+        const int ge1 = (g0 + lane + 32 < g1) ? ko[g0 + lane + 33] : -1;
         int issued = 0;
         for (int t = 0; t < n_tiles; ++t) {
             const int stage = t & 1, ring = t % RING, j0 = j_begin + t * BK;
@@ -172,8 +176,9 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
                 meta[c] = v.x;
                 meta[BK + c] = v.y;
             }
-            for (int g = g0 + lane; g < g1; g += 32) {   // key-group ends that fall in this tile
-                const int e = ko[g + 1];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {   // key-group ends that fall in this tile
+                const int e = h ? ge1 : ge0;
                 if (e > j0 && e <= j0 + BK) atomicOr(&endm[(e - 1 - j0) >> 5], 1u << ((e - 1 - j0) & 31));
             }
             __syncwarp();
@@ -194,18 +199,23 @@ __global__ void __launch_bounds__(192, 1) route_tc_kernel(
         // ------------------------------------------------ MMA: D[stage] = sum over pieces of A_piece K^T
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_f32acc(BA, BK, kFmtBF16, false);
+            // descriptors built once; each MMA adds a compile-time offset (>> 4) to
+            // the start-address field, which never carries out (shared < 2^18)
+            const uint64_t dA = smem_desc(s_base + L::oA, 16, 1024), dK = smem_desc(s_base + L::oK, 16, 1024);
             bool ok = mbar_wait(bar(B_A), 0, abort_flag, kSpin);
             for (int t = 0; ok && t < n_tiles; ++t) {
                 const int stage = t & 1;
                 if (!mbar_wait(bar(B_BF + stage), (t >> 1) & 1, abort_flag, kSpin)) { ok = false; break; }
                 if (t >= 2 && !mbar_wait(bar(B_DE + stage), ((t >> 1) - 1) & 1, abort_flag, kSpin)) { ok = false; break; }
                 tc_fence_after();
-                int n = 0;
+                const uint64_t b0 = dK + (uint64_t)((stage * L::KB) >> 4);
+#pragma unroll
                 for (int pc = 0; pc < 3; ++pc)
-                    for (int kk = 0; kk < D / 16; ++kk, ++n) {
-                        const uint64_t a = smem_desc(s_base + L::oA + pc * L::AB + (kk / 4) * BA * 128 + (kk % 4) * 32, 16, 1024);
-                        const uint64_t b = smem_desc(s_base + L::oK + stage * L::KB + (kk / 4) * BK * 128 + (kk % 4) * 32, 16, 1024);
-                        mma_f16_ss(tmem + stage * BK, a, b, idesc, n > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t oa = (uint64_t)((pc * L::AB + (kk / 4) * BA * 128 + (kk % 4) * 32) >> 4);
+                        const uint64_t ob = (uint64_t)(((kk / 4) * BK * 128 + (kk % 4) * 32) >> 4);
+                        mma_f16_ss(tmem + stage * BK, dA + oa, b0 + ob, idesc, (pc | kk) ? 1u : 0u);
                     }
                 mma_commit(bar(B_DF + stage));
                 mma_commit(bar(B_BE + stage));
