@@ -117,7 +117,7 @@ struct Plan {
         o_csum,   // [BH][Cmax][Rmax] int64 member sums of the k-means centres (fixed point)
         o_ccnt,   // [BH][Cmax] member counts
         o_prev,   // [BH][N] the labels the sums hold
-        o_cscale; // [BH] fixed-point exponent of each head's coordinates
+        o_cscale; // [BH] largest |coordinate| of each head (float bits): its fixed-point exponent
     // outputs owned by the workspace for sparsepr_call
     size_t o_Qp, o_Kp, o_Vp, o_qlab, o_kvlab, o_permq, o_permk, o_posq, o_qoff, o_kvoff, o_ng, o_its,
         o_qcen, o_kcen, o_vcen, o_qdist, o_score, o_mask, o_selc, o_selg, o_pairs, o_pidx, o_pgrp,

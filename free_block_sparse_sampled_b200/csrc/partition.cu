@@ -511,41 +511,56 @@ __global__ void __launch_bounds__(kSortTile) label_scatter_kernel(const int32_t*
 // (sum * 2^-S / count in fp64, rounded to fp32 and then TF32); empty centres
 // keep their value.
 
-// S_bh = 62 - (bits of max |phi|) - (bits of N).
-__global__ void coord_scale_kernel(const float* __restrict__ phi, int N, int R, int32_t* __restrict__ S_out) {
-    const int bh = blockIdx.x;
-    const float* ph = phi + (size_t)bh * N * R;
+// Largest |phi| of each head, as float bits (non-negative floats order as
+// unsigned integers): grid (blocks, BH), atomicMax into amax[bh] (zeroed first).
+__global__ void coord_absmax_kernel(const float* __restrict__ phi, size_t per_head, uint32_t* __restrict__ amax) {
+    const int bh = blockIdx.y;
+    const float4* ph = reinterpret_cast<const float4*>(phi + (size_t)bh * per_head);
     float m = 0.f;
-    for (size_t e = threadIdx.x; e < (size_t)N * R; e += blockDim.x) m = fmaxf(m, fabsf(ph[e]));
-    m = warp_max(m);
-    __shared__ float red[32];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
-        m = fmaxf(m, red[0]);
-        const int eb = m > 0.f ? ilogbf(m) + 1 : 0;   // max |phi| < 2^eb
-        const int nb = 32 - __clz(N);                   // N < 2^nb
-        S_out[bh] = 62 - eb - nb;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < per_head / 4; e += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = ph[e];
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
     }
+    m = warp_max(m);
+    if ((threadIdx.x & 31) == 0) atomicMax(&amax[bh], __float_as_uint(m));
 }
 
-__device__ __forceinline__ long long fixed_coord(float x, int S) { return __double2ll_rn(scalbn((double)x, S)); }
+// S_bh = 62 - (bits of max |phi|) - (bits of N), from the head's max bits.
+__device__ __forceinline__ int fixed_exponent(uint32_t amax_bits, int N) {
+    const float m = __uint_as_float(amax_bits);
+    const int eb = m > 0.f ? ilogbf(m) + 1 : 0;   // max |phi| < 2^eb
+    return 62 - eb - (32 - __clz(N));               // N < 2^(32 - clz(N))
+}
+
+// q = rint(x * 2^S): two exact multiplications by powers of two (each factor
+// in float range for the S above) and one rounding conversion.
+struct FixedScale {
+    float s1, s2;
+};
+__device__ __forceinline__ FixedScale fixed_scale(int S) {
+    FixedScale f;
+    f.s1 = __int_as_float((S / 2 + 127) << 23);
+    f.s2 = __int_as_float((S - S / 2 + 127) << 23);
+    return f;
+}
+__device__ __forceinline__ long long fixed_coord(float x, const FixedScale& f) { return __float2ll_rn((x * f.s1) * f.s2); }
 
 // First update of a run: the member sums and counts from the sorted member
-// lists (one warp per centre; lane k holds coordinates k, k + 32, ...).
+// lists (one warp per centre; lane k holds coordinates k, k + 32, ...; eight
+// member rows in flight per step).
 template <int R>
 __global__ void centre_sums_kernel(const float* __restrict__ phi, const int32_t* __restrict__ sorted,
-                                   const int32_t* __restrict__ offs, const int32_t* __restrict__ S_in, int N, int C,
+                                   const int32_t* __restrict__ offs, const uint32_t* __restrict__ amax, int N, int C,
                                    long long* __restrict__ csum, int32_t* __restrict__ ccnt,
                                    const int32_t* __restrict__ ctl) {
     constexpr int KPL = (R + 31) / 32;   // coordinates per lane
+    constexpr int U = 8;                 // member rows per step
     const int bh = blockIdx.y, lane = threadIdx.x & 31;
     if (ctl[bh * kCtlStride + kCtlDone]) return;
     const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (c >= C) return;
     const int s = offs[(size_t)bh * (C + 1) + c], e = offs[(size_t)bh * (C + 1) + c + 1];
-    const int S = S_in[bh];
+    const FixedScale S = fixed_scale(fixed_exponent(amax[bh], N));
     long long acc[KPL];
 #pragma unroll
     for (int k = 0; k < KPL; ++k) acc[k] = 0;
@@ -554,12 +569,19 @@ __global__ void centre_sums_kernel(const float* __restrict__ phi, const int32_t*
     for (int p0 = s; p0 < e; p0 += 32) {
         const int my = (p0 + lane < e) ? so[p0 + lane] : 0;
         const int n = min(32, e - p0);
-#pragma unroll 4
-        for (int q = 0; q < n; ++q) {
-            const int row = __shfl_sync(0xffffffffu, my, q);
+        for (int q0 = 0; q0 < n; q0 += U) {
+            float x[U][KPL];
 #pragma unroll
-            for (int k = 0; k < KPL; ++k)
-                if (32 * k + lane < R) acc[k] += fixed_coord(ph[(size_t)row * R + 32 * k + lane], S);
+            for (int u = 0; u < U; ++u) {
+                const int row = __shfl_sync(0xffffffffu, my, (q0 + u) & 31);
+#pragma unroll
+                for (int k = 0; k < KPL; ++k)
+                    x[u][k] = (q0 + u < n && 32 * k + lane < R) ? ph[(size_t)row * R + 32 * k + lane] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int k = 0; k < KPL; ++k) acc[k] += fixed_coord(x[u][k], S);
         }
     }
     long long* cs = csum + ((size_t)bh * C + c) * R;
@@ -574,7 +596,7 @@ __global__ void centre_sums_kernel(const float* __restrict__ phi, const int32_t*
 // One warp per 32 points; the warp takes the moving points one at a time,
 // a lane per coordinate.
 __global__ void centre_delta_kernel(const float* __restrict__ phi, const int32_t* __restrict__ labels,
-                                    int32_t* __restrict__ prev, const int32_t* __restrict__ S_in, int N, int C, int R,
+                                    int32_t* __restrict__ prev, const uint32_t* __restrict__ amax, int N, int C, int R,
                                     long long* __restrict__ csum, int32_t* __restrict__ ccnt,
                                     const int32_t* __restrict__ ctl) {
     const int bh = blockIdx.y, lane = threadIdx.x & 31;
@@ -592,7 +614,7 @@ __global__ void centre_delta_kernel(const float* __restrict__ phi, const int32_t
         atomicAdd(&ccnt[(size_t)bh * C + nw], 1);
         atomicSub(&ccnt[(size_t)bh * C + od], 1);
     }
-    const int S = S_in[bh];
+    const FixedScale S = fixed_scale(fixed_exponent(amax[bh], N));
     const float* ph = phi + hb * R;
     unsigned long long* cs = reinterpret_cast<unsigned long long*>(csum) + (size_t)bh * C * R;
     while (moving != 0u) {
@@ -609,7 +631,7 @@ __global__ void centre_delta_kernel(const float* __restrict__ phi, const int32_t
 
 // Centres (and -|c|^2/2 halves, hn = |c|^2 / 2) from the sums; one warp per centre.
 __global__ void centre_from_sums_kernel(const long long* __restrict__ csum, const int32_t* __restrict__ ccnt,
-                                        const int32_t* __restrict__ S_in, int C, int R, float* __restrict__ cen,
+                                        const uint32_t* __restrict__ amax, int N, int C, int R, float* __restrict__ cen,
                                         float* __restrict__ hn, const int32_t* __restrict__ ctl) {
     const int bh = blockIdx.y, lane = threadIdx.x & 31;
     if (ctl[bh * kCtlStride + kCtlDone]) return;
@@ -617,7 +639,7 @@ __global__ void centre_from_sums_kernel(const long long* __restrict__ csum, cons
     if (c >= C) return;
     const int cnt = ccnt[(size_t)bh * C + c];
     if (cnt <= 0) return;   // empty: keeps its value
-    const int S = S_in[bh];
+    const int S = fixed_exponent(amax[bh], N);
     const long long* cs = csum + ((size_t)bh * C + c) * R;
     float* cc = cen + ((size_t)bh * C + c) * R;
     float ss = 0.f;
@@ -844,8 +866,11 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
     long long* csum = at<long long>(ws, pl.o_csum);
     int32_t* ccnt = at<int32_t>(ws, pl.o_ccnt);
     int32_t* prev = at<int32_t>(ws, pl.o_prev);
-    int32_t* cscale = at<int32_t>(ws, pl.o_cscale);
-    if (p.kmeans_iters > 1) count_launch(), coord_scale_kernel<<<BH, 1024, 0, st>>>(phi, N, R, cscale);
+    uint32_t* amax = at<uint32_t>(ws, pl.o_cscale);
+    if (p.kmeans_iters > 1) {
+        cudaMemsetAsync(amax, 0, (size_t)BH * sizeof(uint32_t), st);
+        count_launch(), coord_absmax_kernel<<<dim3(16, BH), 512, 0, st>>>(phi, (size_t)N * R, amax);
+    }
     for (int it = 0; it < p.kmeans_iters; ++it) {
         const int first = it == 0;
         if (it == 1) {   // first update: sums and counts from the sorted member lists
@@ -854,13 +879,13 @@ void kmeans_run(const Plan& pl, const sparsepr_params& p, void* ws, const float*
             count_launch(), label_offsets_kernel<<<BH, 1024, 0, st>>>(offs, N, C, ctl);
             count_launch(), label_scatter_kernel<<<tgrid, kSortTile, scatter_smem(C), st>>>(raw, N, C, pl.n_sort_tiles,
                                                                                              hist, offs, sorted, ctl);
-            count_launch(), centre_sums_kernel<R><<<wgrid, 256, 0, st>>>(phi, sorted, offs, cscale, N, C, csum, ccnt, ctl);
+            count_launch(), centre_sums_kernel<R><<<wgrid, 256, 0, st>>>(phi, sorted, offs, amax, N, C, csum, ccnt, ctl);
             cudaMemcpyAsync(prev, raw, (size_t)BH * N * sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
-            count_launch(), centre_from_sums_kernel<<<wgrid, 256, 0, st>>>(csum, ccnt, cscale, C, R, cen, hn, ctl);
+            count_launch(), centre_from_sums_kernel<<<wgrid, 256, 0, st>>>(csum, ccnt, amax, N, C, R, cen, hn, ctl);
         } else if (it > 1) {   // later updates: only the points whose label changed
-            count_launch(), centre_delta_kernel<<<dim3((N + 255) / 256, BH), 256, 0, st>>>(phi, raw, prev, cscale, N, C,
+            count_launch(), centre_delta_kernel<<<dim3((N + 255) / 256, BH), 256, 0, st>>>(phi, raw, prev, amax, N, C,
                                                                                           R, csum, ccnt, ctl);
-            count_launch(), centre_from_sums_kernel<<<wgrid, 256, 0, st>>>(csum, ccnt, cscale, C, R, cen, hn, ctl);
+            count_launch(), centre_from_sums_kernel<<<wgrid, 256, 0, st>>>(csum, ccnt, amax, N, C, R, cen, hn, ctl);
         }
         if (!launch_kmeans_assign_tc(phi, cen, hn, at<float>(ws, pl.o_hs), BH, N, C, R, raw, ctl, first, dbg_scores, dbg_hist,
                                      p.kmeans_iters, at<DevStatus>(ws, pl.o_status), st))
